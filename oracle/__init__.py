@@ -1,0 +1,174 @@
+"""CPU fp64 oracle for the causal FFT long convolution (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this package.  The CUDA library never imports it and shares no code with it.
+
+Definitions (see fftconv_oracle.c for the page citations):
+
+* ``causal_conv1d``: y[b,h,t] = sum_{s<=t, s<L} k[h,s] x[b,h,t-s] (+ D[h] x[b,h,t]),
+  x = u (ungated) or u*w (gated, then y *= v).  This is
+  irfft(rfft(x,2N) * rfft(k,2N))[:N] (+ D x) evaluated as the direct sum.
+* ``causal_conv2d``: y[b,c,i,j] = sum_{p<=i,q<=j} k[c,p,q] u[b,c,i-p,j-q].
+* ``dft_causal_conv1d`` / ``dft_causal_conv2d``: the same results through an
+  explicit O(M^2) DFT product (tiny sizes only), the independent second route.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+
+def bind(path):
+    """Open an oracle shared library at ``path`` and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_causal_conv1d.argtypes = [_i64] * 4 + [_f64p] * 6
+    lib.oracle_causal_conv1d_points.argtypes = [_i64] * 4 + [_f64p] * 5 + [_i64] + [_i64p] * 3 + [_f64p]
+    lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
+    lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
+    lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
+    lib.oracle_dft_causal_conv2d.argtypes = [_i64] * 4 + [_f64p] * 3
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = bind(_build.build())
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_f64p)
+
+
+def _ip(a):
+    return a.ctypes.data_as(_i64p)
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs with."""
+    return int(_load().oracle_num_threads())
+
+
+def _check_1d(u, k, D, w, v):
+    u = _f64(u)
+    k = _f64(k)
+    if u.ndim != 3 or k.ndim != 2:
+        raise ValueError("u must be [B,H,N] and k [H,L]")
+    B, H, N = u.shape
+    if k.shape[0] != H or k.shape[1] > N or k.shape[1] < 1:
+        raise ValueError("k must be [H,L] with 1 <= L <= N")
+    if (w is None) != (v is None):
+        raise ValueError("gated form needs both w and v")
+    w, v, D = _f64(w), _f64(v), _f64(D)
+    for a in (w, v):
+        if a is not None and a.shape != u.shape:
+            raise ValueError("w, v must have u's shape")
+    if D is not None and D.shape != (H,):
+        raise ValueError("D must be [H]")
+    return u, k, D, w, v
+
+
+def causal_conv1d(u, k, D=None, w=None, v=None) -> np.ndarray:
+    """Full fp64 direct-sum oracle; returns y [B,H,N]."""
+    u, k, D, w, v = _check_1d(u, k, D, w, v)
+    B, H, N = u.shape
+    y = np.empty_like(u)
+    _load().oracle_causal_conv1d(B, H, N, k.shape[1], _p(u), _p(w), _p(v), _p(k), _p(D), _p(y))
+    return y
+
+
+def causal_conv1d_points(u, k, b_idx, h_idx, t_idx, D=None, w=None, v=None) -> np.ndarray:
+    """fp64 oracle at the sampled outputs y[b_idx[i], h_idx[i], t_idx[i]]."""
+    u, k, D, w, v = _check_1d(u, k, D, w, v)
+    B, H, N = u.shape
+    bi = np.ascontiguousarray(b_idx, dtype=np.int64)
+    hi = np.ascontiguousarray(h_idx, dtype=np.int64)
+    ti = np.ascontiguousarray(t_idx, dtype=np.int64)
+    if not (bi.shape == hi.shape == ti.shape) or bi.ndim != 1:
+        raise ValueError("index arrays must be 1-D and of equal length")
+    if bi.size and (bi.min() < 0 or bi.max() >= B or hi.min() < 0 or hi.max() >= H
+                    or ti.min() < 0 or ti.max() >= N):
+        raise ValueError("sample index out of range")
+    out = np.empty(bi.size, dtype=np.float64)
+    _load().oracle_causal_conv1d_points(B, H, N, k.shape[1], _p(u), _p(w), _p(v), _p(k), _p(D),
+                                        bi.size, _ip(bi), _ip(hi), _ip(ti), _p(out))
+    return out
+
+
+def _check_2d(u, k):
+    u = _f64(u)
+    k = _f64(k)
+    if u.ndim != 4 or k.ndim != 3:
+        raise ValueError("u must be [B,C,Hs,Ws] and k [C,Kh,Kw]")
+    B, C, Hs, Ws = u.shape
+    if k.shape[0] != C or not (1 <= k.shape[1] <= Hs) or not (1 <= k.shape[2] <= Ws):
+        raise ValueError("k must be [C,Kh,Kw] with Kh <= Hs, Kw <= Ws")
+    return u, k
+
+
+def causal_conv2d(u, k) -> np.ndarray:
+    """Full fp64 2-D oracle (first-quadrant crop of the zero-padded linear conv)."""
+    u, k = _check_2d(u, k)
+    B, C, Hs, Ws = u.shape
+    y = np.empty_like(u)
+    _load().oracle_causal_conv2d(B, C, Hs, Ws, k.shape[1], k.shape[2], _p(u), _p(k), _p(y))
+    return y
+
+
+def causal_conv2d_points(u, k, b_idx, c_idx, i_idx, j_idx) -> np.ndarray:
+    """fp64 2-D oracle at sampled pixels."""
+    u, k = _check_2d(u, k)
+    B, C, Hs, Ws = u.shape
+    idx = [np.ascontiguousarray(a, dtype=np.int64) for a in (b_idx, c_idx, i_idx, j_idx)]
+    n = idx[0].size
+    if any(a.shape != (n,) for a in idx):
+        raise ValueError("index arrays must be 1-D and of equal length")
+    lims = (B, C, Hs, Ws)
+    if n and any(a.min() < 0 or a.max() >= m for a, m in zip(idx, lims)):
+        raise ValueError("sample index out of range")
+    out = np.empty(n, dtype=np.float64)
+    _load().oracle_causal_conv2d_points(B, C, Hs, Ws, k.shape[1], k.shape[2], _p(u), _p(k), n,
+                                        *[_ip(a) for a in idx], _p(out))
+    return out
+
+
+def dft_causal_conv1d(x, k) -> np.ndarray:
+    """Second route (tiny N): explicit length-2N DFT product, inverse, crop."""
+    x = _f64(x)
+    k = _f64(k)
+    if x.ndim != 1 or k.ndim != 1 or not (1 <= k.size <= x.size):
+        raise ValueError("x [N], k [L] with L <= N")
+    y = np.empty_like(x)
+    _load().oracle_dft_causal_conv1d(x.size, k.size, _p(x), _p(k), _p(y))
+    return y
+
+
+def dft_causal_conv2d(x, k) -> np.ndarray:
+    """Second route for 2-D (tiny sizes): explicit (2Hs x 2Ws) DFT product, crop."""
+    x = _f64(x)
+    k = _f64(k)
+    if x.ndim != 2 or k.ndim != 2 or k.shape[0] > x.shape[0] or k.shape[1] > x.shape[1]:
+        raise ValueError("x [Hs,Ws], k [Kh,Kw] with Kh <= Hs, Kw <= Ws")
+    y = np.empty_like(x)
+    _load().oracle_dft_causal_conv2d(x.shape[0], x.shape[1], k.shape[0], k.shape[1],
+                                     _p(x), _p(k), _p(y))
+    return y
+
+
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv2d", "causal_conv2d_points",
+           "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

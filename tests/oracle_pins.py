@@ -1,0 +1,252 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each check raises AssertionError on failure.  They are collected as tests in
+test_oracle_pins.py and re-run against deliberately broken copies of the
+oracle in test_oracle_mutants.py, which shows that a plausible mistake anywhere
+in the oracle fails at least one of them.
+
+What pins what:
+* the numpy FFT route of the defining formula y = irfft(rfft(x,2N) rfft(k,2N))[:N]
+  (+ D x), written literally with numpy.fft ("FlashFFTConv: Efficient
+  Convolutions for Long Sequences with Tensor Cores", abstract; causal padding:
+  "RubiConv -- Efficient Boundary-Respecting Convolutions", Caracal abstract);
+* numpy.convolve / scipy.signal.convolve2d, the library linear convolutions;
+* closed forms (geometric kernel on a constant input; the first-order
+  recursion that a geometric kernel satisfies, exact at any N);
+* identities the definition fixes: delta kernel / delta input, linearity,
+  commutativity, causality, shift invariance, 2-D separability;
+* hand-derived fixtures in tests/golden/hand_examples.json.
+"""
+import json
+import os
+
+import numpy as np
+import scipy.signal
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_examples.json")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _fft_formula_1d(x, k, D=None):
+    """The defining formula with numpy's FFT as the library step (fp64)."""
+    N = x.shape[-1]
+    M = 2 * N
+    y = np.fft.irfft(np.fft.rfft(x, M) * np.fft.rfft(k, M), M)[..., :N]
+    if D is not None:
+        y = y + D * x
+    return y
+
+
+def check_golden_1d():
+    cases = json.load(open(GOLDEN))["cases_1d"]
+    for c in cases:
+        u = np.array(c["u"], float)[None, None]
+        k = np.array(c["k"], float)[None]
+        D = None if c["D"] is None else np.array([c["D"]], float)
+        w = None if c["w"] is None else np.array(c["w"], float)[None, None]
+        v = None if c["v"] is None else np.array(c["v"], float)[None, None]
+        y = oracle.causal_conv1d(u, k, D=D, w=w, v=v)[0, 0]
+        assert np.array_equal(y, np.array(c["y"], float)), (c["name"], y, c["y"])
+
+
+def check_golden_2d():
+    for c in json.load(open(GOLDEN))["cases_2d"]:
+        u = np.array(c["u"], float)[None, None]
+        k = np.array(c["k"], float)[None]
+        y = oracle.causal_conv2d(u, k)[0, 0]
+        assert np.array_equal(y, np.array(c["y"], float)), (c["name"], y, c["y"])
+
+
+def check_fft_formula_1d():
+    """Direct sum == the FFT formula written with numpy.fft, ungated and gated,
+    L = N and L < N, with and without D, several N (powers of two and not)."""
+    r = _rng(11)
+    for (B, H, N, L) in [(2, 3, 64, 64), (1, 2, 1000, 1000), (2, 2, 256, 37), (1, 1, 1024, 1024)]:
+        u = r.standard_normal((B, H, N))
+        k = r.standard_normal((H, L)) * np.exp(-0.01 * np.arange(L))
+        D = r.standard_normal(H)
+        got = oracle.causal_conv1d(u, k, D=D)
+        kp = np.zeros((H, N))
+        kp[:, :L] = k
+        want = np.stack([_fft_formula_1d(u[b], kp, D[:, None]) for b in range(B)])
+        assert np.allclose(got, want, rtol=1e-11, atol=1e-11 * np.abs(want).max()), (B, H, N, L)
+        got0 = oracle.causal_conv1d(u, k)
+        want0 = np.stack([_fft_formula_1d(u[b], kp) for b in range(B)])
+        assert np.allclose(got0, want0, rtol=1e-11, atol=1e-11 * np.abs(want0).max())
+        # gated: y = v * ((u*w) conv k + D (u*w))
+        w = r.standard_normal((B, H, N))
+        v = r.standard_normal((B, H, N))
+        gotg = oracle.causal_conv1d(u, k, D=D, w=w, v=v)
+        wantg = np.stack([v[b] * _fft_formula_1d(u[b] * w[b], kp, D[:, None]) for b in range(B)])
+        assert np.allclose(gotg, wantg, rtol=1e-11, atol=1e-11 * np.abs(wantg).max())
+
+
+def check_numpy_convolve_1d():
+    r = _rng(12)
+    for N, L in [(1, 1), (5, 3), (64, 64), (300, 17)]:
+        x = r.standard_normal(N)
+        k = r.standard_normal(L)
+        got = oracle.causal_conv1d(x[None, None], k[None])[0, 0]
+        want = np.convolve(x, k)[:N]
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-12), (N, L)
+
+
+def check_dft_route_1d():
+    """The oracle's explicit-DFT route equals numpy's FFT formula and the direct sum."""
+    r = _rng(13)
+    for N, L in [(1, 1), (4, 4), (16, 9), (64, 64), (33, 33)]:
+        x = r.standard_normal(N)
+        k = r.standard_normal(L)
+        kp = np.zeros(N)
+        kp[:L] = k
+        d = oracle.dft_causal_conv1d(x, k)
+        f = _fft_formula_1d(x, kp)
+        s = oracle.causal_conv1d(x[None, None], k[None])[0, 0]
+        scale = max(1.0, np.abs(f).max())
+        assert np.allclose(d, f, rtol=0, atol=1e-12 * scale * N), (N, L)
+        assert np.allclose(d, s, rtol=0, atol=1e-12 * scale * N), (N, L)
+
+
+def check_delta_identities():
+    r = _rng(14)
+    B, H, N = 2, 3, 97
+    u = r.standard_normal((B, H, N))
+    k = r.standard_normal((H, N))
+    delta_k = np.zeros((H, N))
+    delta_k[:, 0] = 1.0
+    assert np.array_equal(oracle.causal_conv1d(u, delta_k), u)
+    D = r.standard_normal(H)
+    assert np.allclose(oracle.causal_conv1d(u, delta_k, D=D), u * (1.0 + D[:, None]), rtol=1e-15, atol=0)
+    delta_u = np.zeros((B, H, N))
+    delta_u[:, :, 0] = 1.0
+    assert np.array_equal(oracle.causal_conv1d(delta_u, k), np.broadcast_to(k, (B, H, N)))
+    # kernel shorter than the sequence: u = delta returns k followed by zeros
+    ks = r.standard_normal((H, 40))
+    want = np.zeros((B, H, N))
+    want[:, :, :40] = ks
+    assert np.array_equal(oracle.causal_conv1d(delta_u, ks), want)
+
+
+def check_linearity_commutativity():
+    r = _rng(15)
+    B, H, N = 1, 2, 128
+    u1, u2 = r.standard_normal((2, B, H, N))
+    k1, k2 = r.standard_normal((2, H, N))
+    a, b = 0.75, -1.25
+    lhs = oracle.causal_conv1d(a * u1 + b * u2, k1)
+    rhs = a * oracle.causal_conv1d(u1, k1) + b * oracle.causal_conv1d(u2, k1)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+    lhs = oracle.causal_conv1d(u1, a * k1 + b * k2)
+    rhs = a * oracle.causal_conv1d(u1, k1) + b * oracle.causal_conv1d(u1, k2)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+    # commutativity u*k = k*u (both length N, one row per channel)
+    yk = oracle.causal_conv1d(u1, k1)
+    ku = oracle.causal_conv1d(k1[None], u1[0])
+    assert np.allclose(yk, ku, rtol=1e-12, atol=1e-12)
+
+
+def check_causality_shift():
+    r = _rng(16)
+    H, N = 2, 200
+    u = r.standard_normal((1, H, N))
+    k = r.standard_normal((H, N))
+    y = oracle.causal_conv1d(u, k)
+    for t0 in (0, 1, 57, N - 1):
+        up = u.copy()
+        up[:, :, t0] += 3.0
+        yp = oracle.causal_conv1d(up, k)
+        assert np.array_equal(yp[:, :, :t0], y[:, :, :t0]), t0
+        assert not np.array_equal(yp[:, :, t0], y[:, :, t0]), t0
+    # delaying u by s delays y by s
+    s = 13
+    us = np.zeros_like(u)
+    us[:, :, s:] = u[:, :, :N - s]
+    ys = oracle.causal_conv1d(us, k)
+    assert np.allclose(ys[:, :, s:], y[:, :, :N - s], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(ys[:, :, :s], np.zeros((1, H, s)))
+
+
+def check_closed_forms():
+    # k[t] = a^t on u = 1: y[t] = (1 - a^(t+1)) / (1 - a)
+    N, a = 500, 0.97
+    t = np.arange(N)
+    y = oracle.causal_conv1d(np.ones((1, 1, N)), (a ** t)[None])[0, 0]
+    assert np.allclose(y, (1 - a ** (t + 1)) / (1 - a), rtol=1e-12, atol=0)
+    # k[t] = c a^t on any u: y[t] = a y[t-1] + c u[t]  (exact at any N)
+    r = _rng(17)
+    N, a, c = 4096, 0.999, -0.7
+    u = r.standard_normal(N)
+    y = oracle.causal_conv1d(u[None, None], (c * a ** np.arange(N))[None])[0, 0]
+    rec = np.empty(N)
+    acc = 0.0
+    for i in range(N):
+        acc = a * acc + c * u[i]
+        rec[i] = acc
+    assert np.allclose(y, rec, rtol=1e-9, atol=1e-9 * np.abs(rec).max())
+
+
+def check_points_match_full_1d():
+    r = _rng(18)
+    B, H, N = 3, 4, 150
+    u, w, v = r.standard_normal((3, B, H, N))
+    k = r.standard_normal((H, 120))
+    D = r.standard_normal(H)
+    full = oracle.causal_conv1d(u, k, D=D, w=w, v=v)
+    bi = r.integers(0, B, 200)
+    hi = r.integers(0, H, 200)
+    ti = r.integers(0, N, 200)
+    pts = oracle.causal_conv1d_points(u, k, bi, hi, ti, D=D, w=w, v=v)
+    assert np.array_equal(pts, full[bi, hi, ti])
+
+
+def check_conv2d_library():
+    r = _rng(19)
+    for (Hs, Ws, Kh, Kw) in [(1, 1, 1, 1), (7, 5, 7, 5), (16, 16, 16, 16), (12, 20, 5, 9)]:
+        u = r.standard_normal((2, 2, Hs, Ws))
+        k = r.standard_normal((2, Kh, Kw))
+        got = oracle.causal_conv2d(u, k)
+        for b in range(2):
+            for c in range(2):
+                want = scipy.signal.convolve2d(u[b, c], k[c], mode="full")[:Hs, :Ws]
+                assert np.allclose(got[b, c], want, rtol=1e-12, atol=1e-12), (Hs, Ws, Kh, Kw)
+
+
+def check_conv2d_separable_and_dft():
+    r = _rng(20)
+    Hs, Ws = 12, 10
+    u1, k1 = r.standard_normal((2, Hs))
+    u2, k2 = r.standard_normal((2, Ws))
+    y = oracle.causal_conv2d(np.outer(u1, u2)[None, None], np.outer(k1, k2)[None])[0, 0]
+    y1 = oracle.causal_conv1d(u1[None, None], k1[None])[0, 0]
+    y2 = oracle.causal_conv1d(u2[None, None], k2[None])[0, 0]
+    assert np.allclose(y, np.outer(y1, y2), rtol=1e-12, atol=1e-12)
+    x = r.standard_normal((6, 5))
+    k = r.standard_normal((4, 5))
+    d = oracle.dft_causal_conv2d(x, k)
+    s = oracle.causal_conv2d(x[None, None], k[None])[0, 0]
+    f = np.fft.irfft2(np.fft.rfft2(x, (12, 10)) * np.fft.rfft2(k, (12, 10)), (12, 10))[:6, :5]
+    assert np.allclose(d, f, rtol=0, atol=1e-11)
+    assert np.allclose(s, f, rtol=0, atol=1e-11)
+
+
+def check_points_match_full_2d():
+    r = _rng(21)
+    u = r.standard_normal((2, 3, 9, 11))
+    k = r.standard_normal((3, 9, 11))
+    full = oracle.causal_conv2d(u, k)
+    idx = [r.integers(0, m, 100) for m in (2, 3, 9, 11)]
+    pts = oracle.causal_conv2d_points(u, k, *idx)
+    assert np.array_equal(pts, full[tuple(idx)])
+
+
+ALL_CHECKS = [
+    check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
+    check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
+    check_causality_shift, check_closed_forms, check_points_match_full_1d,
+    check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
+]
