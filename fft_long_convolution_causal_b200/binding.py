@@ -1,0 +1,255 @@
+"""ctypes binding of libfftconv_b200.so (the C ABI in include/fftconv.h).
+
+Argument marshalling only: every step of the convolution runs in the CUDA
+library.  torch supplies device memory and the current stream.  If the
+library is missing the calls raise -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+_LIB = None
+
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "kernel spectrum not computed for this plan",
+    4: "out of device memory", 5: "CUDA error", 6: "device wait timed out",
+}
+DTYPES = {"f32": 0, "bf16": 1}
+TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+# name -> (restype, argtypes); mirrors include/fftconv.h
+_vp = ctypes.c_void_p
+_SIGS = {
+    "fftconv_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                           ctypes.c_int, ctypes.c_int]),
+    "fftconv2d_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int]),
+    "fftconv_plan_destroy": (ctypes.c_int, [_vp]),
+    "fftconv_spectrum_bytes": (ctypes.c_size_t, [_vp]),
+    "fftconv_workspace_bytes": (ctypes.c_size_t, [_vp]),
+    "fftconv_plan_path": (ctypes.c_char_p, [_vp]),
+    "fftconv_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, _vp, _vp, _vp]),
+    "fftconv_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv2d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
+    "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fftconv_version": (ctypes.c_int, []),
+}
+
+
+class FFTConvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, 'unknown')} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
+    """Load the CUDA library; raises if it is not built."""
+    global _LIB
+    if _LIB is None:
+        path = _build.LIB
+        if not os.path.exists(path):
+            if not build_if_missing:
+                raise FileNotFoundError(
+                    f"{path} is missing: build it with `python -m fft_long_convolution_causal_b200.build`")
+            _build.build()
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    return load_library().fftconv_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise FFTConvError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class _PlanBase:
+    _handle: ctypes.c_void_p
+
+    def __del__(self):
+        h = getattr(self, "_handle", None)
+        if h is not None and h.value and _LIB is not None:
+            _LIB.fftconv_plan_destroy(h)
+            self._handle = None
+
+    def destroy(self):
+        self.__del__()
+
+    @property
+    def spectrum_bytes(self) -> int:
+        return int(self.lib.fftconv_spectrum_bytes(self._handle))
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self.lib.fftconv_workspace_bytes(self._handle))
+
+    @property
+    def path(self) -> str:
+        return self.lib.fftconv_plan_path(self._handle).decode()
+
+    def new_spectrum(self, device=None) -> torch.Tensor:
+        return torch.empty(self.spectrum_bytes, dtype=torch.uint8, device=device or "cuda")
+
+    def new_workspace(self, device=None) -> Optional[torch.Tensor]:
+        n = self.workspace_bytes
+        return torch.empty(n, dtype=torch.uint8, device=device or "cuda") if n else None
+
+    def _ws(self, workspace):
+        if workspace is None and self.workspace_bytes:
+            if self._workspace is None:
+                self._workspace = self.new_workspace()
+            workspace = self._workspace
+        if workspace is not None and workspace.numel() * workspace.element_size() < self.workspace_bytes:
+            raise ValueError("workspace too small")
+        return workspace
+
+
+class Plan(_PlanBase):
+    """1-D plan: fftconv_plan_create(B, H, N, dtype, gated)."""
+
+    def __init__(self, B: int, H: int, N: int, dtype: str = "bf16", gated: bool = False):
+        self.lib = load_library()
+        self.B, self.H, self.N, self.dtype, self.gated = B, H, N, dtype, bool(gated)
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv_plan_create(ctypes.byref(h), B, H, N, DTYPES[dtype], int(bool(gated))),
+               "fftconv_plan_create")
+        self._handle = h
+        self._workspace = None
+
+    def kernel_spectrum(self, k: torch.Tensor, khat: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """khat <- spectrum of k [H, L] (fp32, L <= N)."""
+        if k.dim() != 2:
+            raise ValueError("k must be [H, L]")
+        _need(k, "k", (self.H, k.shape[1]), torch.float32)
+        if khat is None:
+            khat = self.new_spectrum(k.device)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv_kernel_spectrum(self._handle, _ptr(k), k.shape[1], _ptr(khat), _ptr(workspace),
+                                                _stream(stream)), "fftconv_kernel_spectrum")
+        return khat
+
+    def fwd(self, u: torch.Tensor, khat: torch.Tensor, D: Optional[torch.Tensor] = None,
+            v: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None,
+            y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+        """y = v * ((u*w) conv k + D (u*w)) (gated) or (u conv k) + D u."""
+        shape = (self.B, self.H, self.N)
+        _need(u, "u", shape, self.torch_dtype)
+        if self.gated:
+            _need(v, "v", shape, self.torch_dtype)
+            _need(w, "w", shape, self.torch_dtype)
+        elif v is not None or w is not None:
+            raise ValueError("v and w are only for a gated plan")
+        if D is not None:
+            _need(D, "D", (self.H,), torch.float32)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        _need(y, "y", shape, self.torch_dtype)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv_fwd(self._handle, _ptr(u), _ptr(v), _ptr(w), _ptr(khat), _ptr(D), _ptr(y),
+                                    _ptr(workspace), _stream(stream)), "fftconv_fwd")
+        return y
+
+
+class Plan2D(_PlanBase):
+    """2-D plan: fftconv2d_plan_create(B, C, Hs, Ws, dtype)."""
+
+    def __init__(self, B: int, C: int, Hs: int, Ws: int, dtype: str = "bf16"):
+        self.lib = load_library()
+        self.B, self.C, self.Hs, self.Ws, self.dtype = B, C, Hs, Ws, dtype
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv2d_plan_create(ctypes.byref(h), B, C, Hs, Ws, DTYPES[dtype]),
+               "fftconv2d_plan_create")
+        self._handle = h
+        self._workspace = None
+
+    def kernel_spectrum(self, k: torch.Tensor, khat: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        if k.dim() != 3:
+            raise ValueError("k must be [C, Kh, Kw]")
+        _need(k, "k", (self.C, k.shape[1], k.shape[2]), torch.float32)
+        if khat is None:
+            khat = self.new_spectrum(k.device)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv2d_kernel_spectrum(self._handle, _ptr(k), k.shape[1], k.shape[2], _ptr(khat),
+                                                  _ptr(workspace), _stream(stream)), "fftconv2d_kernel_spectrum")
+        return khat
+
+    def fwd(self, u: torch.Tensor, khat: torch.Tensor, y: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        shape = (self.B, self.C, self.Hs, self.Ws)
+        _need(u, "u", shape, self.torch_dtype)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        _need(y, "y", shape, self.torch_dtype)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv2d_fwd(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace),
+                                      _stream(stream)), "fftconv2d_fwd")
+        return y
+
+
+def fftconv(u: torch.Tensor, k: torch.Tensor, D: Optional[torch.Tensor] = None,
+            v: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One-shot causal long convolution (plan + spectrum + forward)."""
+    B, H, N = u.shape
+    dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[u.dtype]
+    plan = Plan(B, H, N, dtype, gated=v is not None)
+    khat = plan.kernel_spectrum(k.contiguous())
+    y = plan.fwd(u, khat, D=D, v=v, w=w)
+    torch.cuda.current_stream().synchronize()  # the plan's tables are freed on return
+    return y
+
+
+def fftconv2d(u: torch.Tensor, k: torch.Tensor) -> torch.Tensor:
+    """One-shot 2-D causal convolution (plan + spectrum + forward)."""
+    B, C, Hs, Ws = u.shape
+    dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[u.dtype]
+    plan = Plan2D(B, C, Hs, Ws, dtype)
+    khat = plan.kernel_spectrum(k.contiguous())
+    y = plan.fwd(u, khat)
+    torch.cuda.current_stream().synchronize()  # the plan's tables are freed on return
+    return y

@@ -1,0 +1,423 @@
+// conv1d_simt.cu -- fp32 SIMT kernels of the 1-D causal FFT convolution.
+//
+// Two batch rows b, b+1 of one channel h are packed as one complex sequence
+// z = x_b + i x_{b+1}; because k is real, iDFT(DFT(z) . K) = (x_b * k) + i (x_{b+1} * k),
+// so one complex transform of length M = 2N serves two rows.  The input is
+// zero-padded to 2N and the output truncated to [:N] ("RubiConv -- Efficient
+// Boundary-Respecting Convolutions", Caracal abstract: causal masking by
+// asymmetric padding and truncation); FFT, pointwise product and inverse
+// FFT are fused with no intermediate off-chip traffic ("FlashConv",
+// Mechanism).  The skip term D x is folded into the pointwise product as the
+// constant spectrum D/M of D.delta, so x is never re-read.
+//
+// Fused path (2N <= 16384): one CTA per (pair, channel) holds the whole
+// transform in shared memory.
+//
+// Multi-pass path (2N > 16384): M = N1 x N2, n = N2 n1 + n2, k = k1 + N1 k2
+// (the four-step / Monarch split of the DFT that "FlashFFTConv" (abstract)
+// uses to map the FFT onto matrix units and to fuse long sequences):
+//   pass 1: per column n2, DFT_N1 over n1 < N1/2 (the nonzero half), times
+//           W_M^{n2 k1}, into the workspace as [k1][n2];
+//   pass 2: per row k1, DFT_N2 over n2, times Khat[k1][k2] (+ D/M), inverse
+//           DFT_N2, times W_M^{-n2 k1}, back into the workspace;
+//   pass 3: per column n2, inverse DFT_N1, only n1 < N1/2 (n < N) kept.
+// Pairs are processed in groups so the workspace of one group stays small
+// (L2-sized) and is reused group after group.
+#include "fft_simt.cuh"
+#include "plan.h"
+
+namespace fftc {
+
+// Load x = u (or u*w) of the pair (row0, row1) at position n.
+template <typename IO, bool GATED>
+__device__ __forceinline__ float2 load_pair(const IO* __restrict__ u, const IO* __restrict__ w,
+                                            size_t row0, size_t row1, bool has1, size_t n) {
+    float a = to_f(u[row0 + n]);
+    if (GATED) a *= to_f(w[row0 + n]);
+    float b = 0.f;
+    if (has1) {
+        b = to_f(u[row1 + n]);
+        if (GATED) b *= to_f(w[row1 + n]);
+    }
+    return make_float2(a, b);
+}
+
+// Store the pair (re -> row0, im -> row1) at position n, gated by v.
+template <typename IO, bool GATED>
+__device__ __forceinline__ void store_pair(IO* __restrict__ y, const IO* __restrict__ v, size_t row0,
+                                           size_t row1, bool has1, size_t n, float2 z) {
+    float a = z.x, b = z.y;
+    if (GATED) a *= to_f(v[row0 + n]);
+    y[row0 + n] = from_f<IO>(a);
+    if (has1) {
+        if (GATED) b *= to_f(v[row1 + n]);
+        y[row1 + n] = from_f<IO>(b);
+    }
+}
+
+template <class G>
+constexpr int first_radix() { return 1 << G::Plan::log2r(0); }
+template <class G>
+constexpr int last_radix() { return 1 << G::Plan::log2r(G::Plan::kStages - 1); }
+
+// ============================================================== fused path
+template <int LOG2M>
+using FusedG = Geometry<LOG2M, 1, false>;
+
+template <int LOG2M, typename IO, bool GATED>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+fused_fwd_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __restrict__ w,
+               const float2* __restrict__ khat, const float* __restrict__ D, IO* __restrict__ y,
+               const float2* __restrict__ tw, int B, int H) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, N = M / 2, NS = G::Plan::kStages;
+    static_assert(NS >= 2, "transform too short");
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, h = blockIdx.y;
+    const int b0 = 2 * blockIdx.x;
+    const bool has1 = b0 + 1 < B;
+    const size_t row0 = ((size_t)b0 * H + h) * N;
+    const size_t row1 = ((size_t)(b0 + 1) * H + h) * N;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+
+    // forward DFT_M; stage 0 reads the nonzero half straight from global memory
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return load_pair<IO, GATED>(u, w, row0, row1, has1, n); }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(smem, tid, tw);
+
+    // pointwise product with (Khat + D/M), fused into the first inverse stage
+    const float dm = D ? D[h] * (1.0f / M) : 0.f;
+    const float2* __restrict__ kh = khat + (size_t)h * M;
+    stage<G, 0, true, R0, R0, true>(
+        tid, tw,
+        [&](int i, int) {
+            float2 kk = __ldg(&kh[i]);
+            kk.x += dm;
+            return cmul(smem[Lay::at(i, 0)], kk);
+        },
+        sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, true>(smem, tid, tw);
+    // last inverse stage writes only n < N to global memory
+    stage<G, NS - 1, true, RL, RL / 2, false>(
+        tid, tw, lds, [&](int n, int, float2 z) { store_pair<IO, GATED>(y, v, row0, row1, has1, n, z); });
+}
+
+template <int LOG2M>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+fused_spectrum_simt(const float* __restrict__ k, int L, float2* __restrict__ khat,
+                    const float2* __restrict__ tw) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, NS = G::Plan::kStages;
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, h = blockIdx.x;
+    const float* __restrict__ kr = k + (size_t)h * L;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return make_float2(n < L ? kr[n] : 0.f, 0.f); }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, false>(smem, tid, tw);
+    float2* __restrict__ out = khat + (size_t)h * M;
+    stage<G, NS - 1, false, RL, RL, false>(
+        tid, tw, lds, [&](int i, int, float2 z) { out[i] = cscale(z, 1.0f / M); });
+}
+
+template <int LOG2M>
+static size_t fused_smem() { return FusedG<LOG2M>::Lay::kWords * sizeof(float2); }
+
+template <class K>
+static void ensure_smem(K kern, size_t bytes) {
+    if (bytes > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int LOG2M, typename IO, bool GATED>
+static cudaError_t fused_fwd_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                                const float2* khat, const float* D, void* y, cudaStream_t s) {
+    auto kern = fused_fwd_simt<LOG2M, IO, GATED>;
+    const size_t smem = fused_smem<LOG2M>();
+    ensure_smem(kern, smem);
+    dim3 grid((p.B + 1) / 2, p.H);
+    kern<<<grid, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)v, (const IO*)w, khat, D, (IO*)y,
+                                               p.tw.wL, p.B, p.H);
+    return cudaGetLastError();
+}
+
+template <int LOG2M>
+static cudaError_t fused_fwd_dtype(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                                   const float2* khat, const float* D, void* y, cudaStream_t s) {
+    if (p.dtype == FFTCONV_F32)
+        return p.gated ? fused_fwd_go<LOG2M, float, true>(p, u, v, w, khat, D, y, s)
+                       : fused_fwd_go<LOG2M, float, false>(p, u, v, w, khat, D, y, s);
+    return p.gated ? fused_fwd_go<LOG2M, __nv_bfloat16, true>(p, u, v, w, khat, D, y, s)
+                   : fused_fwd_go<LOG2M, __nv_bfloat16, false>(p, u, v, w, khat, D, y, s);
+}
+
+template <int LOG2M>
+static cudaError_t fused_spec_go(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,
+                                 cudaStream_t s) {
+    auto kern = fused_spectrum_simt<LOG2M>;
+    const size_t smem = fused_smem<LOG2M>();
+    ensure_smem(kern, smem);
+    kern<<<p.H, FusedG<LOG2M>::T, smem, s>>>(k, (int)L, khat, p.tw.wL);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fused_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                             const float2* khat, const float* D, void* y, cudaStream_t s) {
+    switch (p.log2M) {
+        case 7: return fused_fwd_dtype<7>(p, u, v, w, khat, D, y, s);
+        case 8: return fused_fwd_dtype<8>(p, u, v, w, khat, D, y, s);
+        case 9: return fused_fwd_dtype<9>(p, u, v, w, khat, D, y, s);
+        case 10: return fused_fwd_dtype<10>(p, u, v, w, khat, D, y, s);
+        case 11: return fused_fwd_dtype<11>(p, u, v, w, khat, D, y, s);
+        case 12: return fused_fwd_dtype<12>(p, u, v, w, khat, D, y, s);
+        case 13: return fused_fwd_dtype<13>(p, u, v, w, khat, D, y, s);
+        case 14: return fused_fwd_dtype<14>(p, u, v, w, khat, D, y, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_fused_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,
+                                  cudaStream_t s) {
+    switch (p.log2M) {
+        case 7: return fused_spec_go<7>(p, k, L, khat, s);
+        case 8: return fused_spec_go<8>(p, k, L, khat, s);
+        case 9: return fused_spec_go<9>(p, k, L, khat, s);
+        case 10: return fused_spec_go<10>(p, k, L, khat, s);
+        case 11: return fused_spec_go<11>(p, k, L, khat, s);
+        case 12: return fused_spec_go<12>(p, k, L, khat, s);
+        case 13: return fused_spec_go<13>(p, k, L, khat, s);
+        case 14: return fused_spec_go<14>(p, k, L, khat, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// ========================================================== multi-pass path
+constexpr int kColTile = 16;  // columns per CTA in the column passes (128 B of fp32 complex)
+
+template <int LOG2N1>
+using ColG = Geometry<LOG2N1, kColTile, true>;
+template <int LOG2N2>
+using RowG = Geometry<LOG2N2, 1, false>;
+
+// W_M^e from the two-level table, e reduced mod M.
+__device__ __forceinline__ float2 twiddle_M(const float2* __restrict__ lo, const float2* __restrict__ hi,
+                                            uint32_t e, int log2M, int log2S) {
+    e &= (1u << log2M) - 1u;
+    return cmul(__ldg(&lo[e & ((1u << log2S) - 1u)]), __ldg(&hi[e >> log2S]));
+}
+
+// Pass 1.  MODE 0: x from (u[,w]) rows of pair P = first + blockIdx.y;
+//          MODE 1: real kernel taps k[h] (h = first + blockIdx.y), n < L.
+template <int LOG2N1, int LOG2N2, typename IO, bool GATED, int MODE>
+__global__ void __launch_bounds__(ColG<LOG2N1>::T)
+mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __restrict__ k, int L,
+         float2* __restrict__ work, const float2* __restrict__ twC, const float2* __restrict__ lo,
+         const float2* __restrict__ hi, int log2S, int B, int H, int64_t first) {
+    using G = ColG<LOG2N1>;
+    using Lay = typename G::Lay;
+    constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2, LOG2M = LOG2N1 + LOG2N2;
+    constexpr int64_t N = (int64_t)N1 * N2 / 2;
+    constexpr int NS = G::Plan::kStages, R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x;
+    const int64_t P = first + blockIdx.y;
+    const int n2_0 = blockIdx.x * kColTile;
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    if constexpr (MODE == 0) {
+        const int h = (int)(P % H);
+        const int b0 = (int)(P / H) * 2;
+        const bool has1 = b0 + 1 < B;
+        const size_t row0 = ((size_t)b0 * H + h) * N, row1 = ((size_t)(b0 + 1) * H + h) * N;
+        stage<G, 0, false, R0 / 2, R0, false>(
+            tid, twC,
+            [&](int n1, int c) {
+                return load_pair<IO, GATED>(u, w, row0, row1, has1, (size_t)n1 * N2 + n2_0 + c);
+            },
+            sts);
+    } else {
+        const float* __restrict__ kr = k + (size_t)P * L;
+        stage<G, 0, false, R0 / 2, R0, false>(
+            tid, twC,
+            [&](int n1, int c) {
+                const int64_t n = (int64_t)n1 * N2 + n2_0 + c;
+                return make_float2(n < L ? kr[n] : 0.f, 0.f);
+            },
+            sts);
+    }
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, false>(smem, tid, twC);
+    float2* __restrict__ out = work + (size_t)blockIdx.y * ((size_t)N1 * N2);
+    stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int k1, int c, float2 z) {
+        const int n2 = n2_0 + c;
+        out[(size_t)k1 * N2 + n2] = cmul(z, twiddle_M(lo, hi, (uint32_t)n2 * (uint32_t)k1, LOG2M, log2S));
+    });
+}
+
+// Pass 2.  MODE 0: forward row DFT, product with Khat (+D/M), inverse, conj
+// twiddle, in place.  MODE 1: forward row DFT only, Khat[k1][k2] = X / M.
+template <int LOG2N1, int LOG2N2, int MODE>
+__global__ void __launch_bounds__(RowG<LOG2N2>::T)
+mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __restrict__ khat_out,
+         const float* __restrict__ D, const float2* __restrict__ twR, const float2* __restrict__ lo,
+         const float2* __restrict__ hi, int log2S, int H, int64_t first) {
+    using G = RowG<LOG2N2>;
+    using Lay = typename G::Lay;
+    constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2, LOG2M = LOG2N1 + LOG2N2;
+    constexpr int M = N1 * N2;
+    constexpr int NS = G::Plan::kStages, R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x;
+    const int k1 = blockIdx.x;
+    const int64_t P = first + blockIdx.y;
+    float2* __restrict__ row = work + ((size_t)blockIdx.y * N1 + k1) * N2;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    stage<G, 0, false, R0, R0, false>(tid, twR, [&](int n2, int) { return row[n2]; }, sts);
+    __syncthreads();
+    if constexpr (MODE == 1) {
+        smem_stages<G, 1, NS - 1, false>(smem, tid, twR);
+        float2* __restrict__ out = khat_out + ((size_t)P * N1 + k1) * N2;
+        stage<G, NS - 1, false, RL, RL, false>(tid, twR, lds,
+                                                [&](int k2, int, float2 z) { out[k2] = cscale(z, 1.0f / M); });
+    } else {
+        smem_stages<G, 1, NS, false>(smem, tid, twR);
+        const int h = (int)(P % H);
+        const float dm = D ? D[h] * (1.0f / M) : 0.f;
+        const float2* __restrict__ kh = khat + ((size_t)h * N1 + k1) * N2;
+        stage<G, 0, true, R0, R0, true>(
+            tid, twR,
+            [&](int k2, int) {
+                float2 kk = __ldg(&kh[k2]);
+                kk.x += dm;
+                return cmul(smem[Lay::at(k2, 0)], kk);
+            },
+            sts);
+        __syncthreads();
+        smem_stages<G, 1, NS - 1, true>(smem, tid, twR);
+        stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int n2, int, float2 z) {
+            row[n2] = cmulc(z, twiddle_M(lo, hi, (uint32_t)n2 * (uint32_t)k1, LOG2M, log2S));
+        });
+    }
+}
+
+// Pass 3: inverse column DFT; outputs n1 < N1/2 (n < N) to y.
+template <int LOG2N1, int LOG2N2, typename IO, bool GATED>
+__global__ void __launch_bounds__(ColG<LOG2N1>::T)
+mp_pass3(const float2* __restrict__ work, const IO* __restrict__ v, IO* __restrict__ y,
+         const float2* __restrict__ twC, int B, int H, int64_t first) {
+    using G = ColG<LOG2N1>;
+    using Lay = typename G::Lay;
+    constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2;
+    constexpr int64_t N = (int64_t)N1 * N2 / 2;
+    constexpr int NS = G::Plan::kStages, R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x;
+    const int64_t P = first + blockIdx.y;
+    const int n2_0 = blockIdx.x * kColTile;
+    const float2* __restrict__ in = work + (size_t)blockIdx.y * ((size_t)N1 * N2);
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    stage<G, 0, true, R0, R0, false>(
+        tid, twC, [&](int k1, int c) { return in[(size_t)k1 * N2 + n2_0 + c]; }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, true>(smem, tid, twC);
+    const int h = (int)(P % H);
+    const int b0 = (int)(P / H) * 2;
+    const bool has1 = b0 + 1 < B;
+    const size_t row0 = ((size_t)b0 * H + h) * N, row1 = ((size_t)(b0 + 1) * H + h) * N;
+    stage<G, NS - 1, true, RL, RL / 2, false>(tid, twC, lds, [&](int n1, int c, float2 z) {
+        store_pair<IO, GATED>(y, v, row0, row1, has1, (size_t)n1 * N2 + n2_0 + c, z);
+    });
+}
+
+template <int LOG2N1, int LOG2N2, typename IO, bool GATED>
+static cudaError_t mp_fwd_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                             const float2* khat, const float* D, void* y, float2* work, cudaStream_t s) {
+    constexpr int N2 = 1 << LOG2N2, N1 = 1 << LOG2N1;
+    auto k1 = mp_pass1<LOG2N1, LOG2N2, IO, GATED, 0>;
+    auto k2 = mp_pass2<LOG2N1, LOG2N2, 0>;
+    auto k3 = mp_pass3<LOG2N1, LOG2N2, IO, GATED>;
+    const size_t sc = ColG<LOG2N1>::Lay::kWords * sizeof(float2);
+    const size_t sr = RowG<LOG2N2>::Lay::kWords * sizeof(float2);
+    ensure_smem(k1, sc);
+    ensure_smem(k2, sr);
+    ensure_smem(k3, sc);
+    for (int64_t first = 0; first < p.pairs; first += p.group) {
+        const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
+        k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
+                                                               p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S, p.B,
+                                                               p.H, first);
+        k2<<<dim3(N1, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
+                                                    p.log2S, p.H, first);
+        k3<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
+                                                               p.H, first);
+    }
+    return cudaGetLastError();
+}
+
+template <int LOG2N1, int LOG2N2>
+static cudaError_t mp_fwd_dtype(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                                const float2* khat, const float* D, void* y, float2* work, cudaStream_t s) {
+    if (p.dtype == FFTCONV_F32)
+        return p.gated ? mp_fwd_go<LOG2N1, LOG2N2, float, true>(p, u, v, w, khat, D, y, work, s)
+                       : mp_fwd_go<LOG2N1, LOG2N2, float, false>(p, u, v, w, khat, D, y, work, s);
+    return p.gated ? mp_fwd_go<LOG2N1, LOG2N2, __nv_bfloat16, true>(p, u, v, w, khat, D, y, work, s)
+                   : mp_fwd_go<LOG2N1, LOG2N2, __nv_bfloat16, false>(p, u, v, w, khat, D, y, work, s);
+}
+
+template <int LOG2N1, int LOG2N2>
+static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat, float2* work,
+                              cudaStream_t s) {
+    constexpr int N2 = 1 << LOG2N2, N1 = 1 << LOG2N1;
+    auto k1 = mp_pass1<LOG2N1, LOG2N2, float, false, 1>;
+    auto k2 = mp_pass2<LOG2N1, LOG2N2, 1>;
+    const size_t sc = ColG<LOG2N1>::Lay::kWords * sizeof(float2);
+    const size_t sr = RowG<LOG2N2>::Lay::kWords * sizeof(float2);
+    ensure_smem(k1, sc);
+    ensure_smem(k2, sr);
+    for (int64_t first = 0; first < p.H; first += p.group) {
+        const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
+        k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(nullptr, nullptr, k, (int)L, work, p.tw.wC,
+                                                               p.tw.wLo, p.tw.wHi, p.log2S, p.B, p.H, first);
+        k2<<<dim3(N1, g), RowG<LOG2N2>::T, sr, s>>>(work, nullptr, khat, nullptr, p.tw.wL, p.tw.wLo, p.tw.wHi,
+                                                    p.log2S, p.H, first);
+    }
+    return cudaGetLastError();
+}
+
+#define FFTC_MP_SWITCH(CALL)             \
+    switch (p.log2M) {                   \
+        case 15: return CALL(7, 8);      \
+        case 16: return CALL(8, 8);      \
+        case 17: return CALL(8, 9);      \
+        case 18: return CALL(9, 9);      \
+        case 19: return CALL(9, 10);     \
+        case 20: return CALL(10, 10);    \
+        case 21: return CALL(10, 11);    \
+        default: return cudaErrorInvalidValue; \
+    }
+
+cudaError_t launch_multipass_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                                 const float2* khat, const float* D, void* y, float2* work, cudaStream_t s) {
+#define FFTC_CALL(a, b) mp_fwd_dtype<a, b>(p, u, v, w, khat, D, y, work, s)
+    FFTC_MP_SWITCH(FFTC_CALL)
+#undef FFTC_CALL
+}
+
+cudaError_t launch_multipass_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,
+                                      float2* work, cudaStream_t s) {
+#define FFTC_CALL(a, b) mp_spec_go<a, b>(p, k, L, khat, work, s)
+    FFTC_MP_SWITCH(FFTC_CALL)
+#undef FFTC_CALL
+}
+
+}  // namespace fftc

@@ -1,0 +1,255 @@
+// fftconv_api.cu -- the extern "C" boundary declared in include/fftconv.h:
+// argument checks, path selection, twiddle tables, dispatch to the kernels.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "fftconv.h"
+#include "plan.h"
+
+namespace {
+
+// Largest transform the fused kernel holds in shared memory (complex fp32).
+constexpr int kFusedMaxLog2M = 14;
+// Workspace target of one multi-pass / 2-D group (L2-sized).
+constexpr size_t kGroupBytes = size_t(64) << 20;
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+int log2i(int64_t x) {
+    int r = 0;
+    while ((int64_t(1) << r) < x) ++r;
+    return r;
+}
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// exp(-2 pi i m / L), m in [0, count), computed in fp64 and rounded to fp32.
+void fill_roots(std::vector<float2>& out, int64_t L, int64_t count, int64_t stride = 1) {
+    for (int64_t m = 0; m < count; ++m) {
+        const int64_t e = (m * stride) % L;
+        const double a = 2.0 * M_PI * (double)e / (double)L;
+        out.push_back(make_float2((float)cos(a), (float)-sin(a)));
+    }
+}
+
+fftconv_status upload_tables(fftconv_plan_s* p, const std::vector<float2>& host) {
+    void* d = nullptr;
+    if (cudaMalloc(&d, host.size() * sizeof(float2)) != cudaSuccess) {
+        cudaGetLastError();
+        return FFTCONV_ERR_OOM;
+    }
+    if (cudaMemcpy(d, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(d);
+        cudaGetLastError();
+        return FFTCONV_ERR_CUDA;
+    }
+    p->d_tables = d;
+    return FFTCONV_OK;
+}
+
+fftconv_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return FFTCONV_OK;
+    return FFTCONV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fftconv_status_string(fftconv_status s) {
+    switch (s) {
+        case FFTCONV_OK: return "ok";
+        case FFTCONV_ERR_INVALID_ARG: return "invalid argument";
+        case FFTCONV_ERR_UNSUPPORTED: return "unsupported size";
+        case FFTCONV_ERR_NOT_READY: return "kernel spectrum not computed for this plan";
+        case FFTCONV_ERR_OOM: return "out of device memory";
+        case FFTCONV_ERR_CUDA: return "CUDA error";
+        case FFTCONV_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int fftconv_version(void) { return 100; }
+
+fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N, fftconv_dtype dtype,
+                                   int gated) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
+    if (!is_pow2(N) || N < FFTCONV_MIN_N || N > FFTCONV_MAX_N) return FFTCONV_ERR_UNSUPPORTED;
+    fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
+    if (!p) return FFTCONV_ERR_OOM;
+    p->kind = 1;
+    p->B = B;
+    p->H = H;
+    p->N = N;
+    p->dtype = dtype;
+    p->gated = gated ? 1 : 0;
+    p->log2M = log2i(2 * N);
+    p->pairs = (int64_t)((B + 1) / 2) * H;
+    cudaGetDevice(&p->device);
+    std::vector<float2> host;
+    const int64_t M = int64_t(1) << p->log2M;
+    if (p->log2M <= kFusedMaxLog2M) {
+        p->path = fftc::PATH_FUSED;
+        fill_roots(host, M, M);
+        p->spectrum_bytes = (size_t)H * M * sizeof(float2);
+        p->workspace_bytes = 0;
+    } else {
+        p->path = fftc::PATH_MULTIPASS;
+        p->log2N1 = p->log2M / 2;
+        p->log2N2 = p->log2M - p->log2N1;
+        p->log2S = (p->log2M + 1) / 2;
+        const int64_t N1 = int64_t(1) << p->log2N1, N2 = int64_t(1) << p->log2N2;
+        const int64_t S = int64_t(1) << p->log2S;
+        fill_roots(host, N2, N2);                 // wL
+        fill_roots(host, N1, N1);                 // wC
+        fill_roots(host, M, S);                   // wLo: W_M^e, e < S
+        fill_roots(host, M, M / S, S);            // wHi: W_M^(e S)
+        const size_t per_pair = (size_t)M * sizeof(float2);
+        int64_t g = (int64_t)(kGroupBytes / per_pair);
+        if (g < 1) g = 1;
+        const int64_t most = p->pairs > H ? p->pairs : H;
+        if (g > most) g = most;
+        p->group = (int)g;
+        p->spectrum_bytes = (size_t)H * M * sizeof(float2);
+        p->workspace_bytes = (size_t)g * per_pair;
+    }
+    fftconv_status st = upload_tables(p, host);
+    if (st != FFTCONV_OK) {
+        delete p;
+        return st;
+    }
+    const float2* base = (const float2*)p->d_tables;
+    if (p->path == fftc::PATH_FUSED) {
+        p->tw.wL = base;
+    } else {
+        const int64_t N1 = int64_t(1) << p->log2N1, N2 = int64_t(1) << p->log2N2;
+        const int64_t S = int64_t(1) << p->log2S;
+        p->tw.wL = base;
+        p->tw.wC = base + N2;
+        p->tw.wLo = base + N2 + N1;
+        p->tw.wHi = base + N2 + N1 + S;
+    }
+    *out = p;
+    return FFTCONV_OK;
+}
+
+fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, int Ws, fftconv_dtype dtype) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || C < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
+    if (!is_pow2(Hs) || !is_pow2(Ws) || Hs < FFTCONV2D_MIN_SIDE || Ws < FFTCONV2D_MIN_SIDE ||
+        Hs > FFTCONV2D_MAX_SIDE || Ws > FFTCONV2D_MAX_SIDE)
+        return FFTCONV_ERR_UNSUPPORTED;
+    fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
+    if (!p) return FFTCONV_ERR_OOM;
+    p->kind = 2;
+    p->path = fftc::PATH_2D;
+    p->B = B;
+    p->H = C;
+    p->Hs = Hs;
+    p->Ws = Ws;
+    p->dtype = dtype;
+    p->pairs = (int64_t)((B + 1) / 2) * C;
+    cudaGetDevice(&p->device);
+    const int64_t LR = 2 * (int64_t)Ws, LC = 2 * (int64_t)Hs;
+    std::vector<float2> host;
+    fill_roots(host, LR, LR);
+    fill_roots(host, LC, LC);
+    const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
+    int64_t g = (int64_t)(kGroupBytes / per_pair);
+    if (g < 1) g = 1;
+    const int64_t most = p->pairs > C ? p->pairs : C;
+    if (g > most) g = most;
+    p->group = (int)g;
+    p->spectrum_bytes = (size_t)C * LC * LR * sizeof(float2);
+    p->workspace_bytes = (size_t)g * per_pair;
+    fftconv_status st = upload_tables(p, host);
+    if (st != FFTCONV_OK) {
+        delete p;
+        return st;
+    }
+    p->tw.wL = (const float2*)p->d_tables;
+    p->tw.wC = (const float2*)p->d_tables + LR;
+    *out = p;
+    return FFTCONV_OK;
+}
+
+fftconv_status fftconv_plan_destroy(fftconv_plan_t p) {
+    if (!p) return FFTCONV_OK;
+    cudaError_t e = cudaSuccess;
+    if (p->d_tables) e = cudaFree(p->d_tables);
+    delete p;
+    return e == cudaSuccess ? FFTCONV_OK : FFTCONV_ERR_CUDA;
+}
+
+size_t fftconv_spectrum_bytes(fftconv_plan_t p) { return p ? p->spectrum_bytes : 0; }
+size_t fftconv_workspace_bytes(fftconv_plan_t p) { return p ? p->workspace_bytes : 0; }
+
+const char* fftconv_plan_path(fftconv_plan_t p) {
+    if (!p) return "none";
+    switch (p->path) {
+        case fftc::PATH_FUSED: return "fused";
+        case fftc::PATH_MULTIPASS: return "multipass";
+        case fftc::PATH_2D: return "2d";
+    }
+    return "unknown";
+}
+
+fftconv_status fftconv_kernel_spectrum(fftconv_plan_t p, const float* k, int64_t L, void* khat, void* work,
+                                       void* stream) {
+    if (!p || p->kind != 1 || !k || !khat || L < 1 || L > p->N) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(khat)) return FFTCONV_ERR_INVALID_ARG;
+    if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (p->path == fftc::PATH_FUSED)
+        e = fftc::launch_fused_spectrum(*p, k, L, (float2*)khat, s);
+    else
+        e = fftc::launch_multipass_spectrum(*p, k, L, (float2*)khat, (float2*)work, s);
+    if (e == cudaSuccess) p->spectrum_ready = true;
+    return cuda_status(e);
+}
+
+fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const void* w, const void* khat,
+                           const float* D, void* y, void* work, void* stream) {
+    if (!p || p->kind != 1 || !u || !khat || !y) return FFTCONV_ERR_INVALID_ARG;
+    if (p->gated ? (!v || !w) : (v || w)) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || (v && !aligned16(v)) || (w && !aligned16(w)) ||
+        (D && !aligned16(D)))
+        return FFTCONV_ERR_INVALID_ARG;
+    if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
+    if (y == u || y == v || y == w) return FFTCONV_ERR_INVALID_ARG;
+    if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (p->path == fftc::PATH_FUSED)
+        e = fftc::launch_fused_fwd(*p, u, v, w, (const float2*)khat, D, y, s);
+    else
+        e = fftc::launch_multipass_fwd(*p, u, v, w, (const float2*)khat, D, y, (float2*)work, s);
+    return cuda_status(e);
+}
+
+fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t p, const float* k, int Kh, int Kw, void* khat, void* work,
+                                         void* stream) {
+    if (!p || p->kind != 2 || !k || !khat || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (Kh < 1 || Kw < 1 || Kh > p->Hs || Kw > p->Ws) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(khat) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    cudaError_t e = fftc::launch_conv2d_spectrum(*p, k, Kh, Kw, (float2*)khat, (float2*)work, (cudaStream_t)stream);
+    if (e == cudaSuccess) p->spectrum_ready = true;
+    return cuda_status(e);
+}
+
+fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work, void* stream) {
+    if (!p || p->kind != 2 || !u || !khat || !y || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (y == u) return FFTCONV_ERR_INVALID_ARG;
+    if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
+    return cuda_status(
+        fftc::launch_conv2d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fft_long_convolution_causal_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fftconv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"FFTCONV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ("fftconv_plan_create", "fftconv_kernel_spectrum", "fftconv_fwd", "fftconv2d_plan_create",
+              "fftconv2d_kernel_spectrum", "fftconv2d_fwd", "fftconv_plan_destroy", "fftconv_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in binding._SIGS, f"binding does not declare {n}"
+
+
+def test_no_internal_symbols_leak(lib):
+    # C++ internals are hidden; only the fftconv_* C names are exported.
+    out = os.popen(f"nm -D --defined-only {build.LIB}").read()
+    exported = [l.split()[-1] for l in out.splitlines() if l.split() and l.split()[1] in "TtWw"]
+    assert exported and all(n.startswith("fftconv") for n in exported), exported
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert binding.status_string(code) == binding.STATUS[code]
+    assert lib.fftconv_version() >= 100
+
+
+def _create(lib, B, H, N, dtype=0, gated=0, null_out=False):
+    h = ctypes.c_void_p()
+    ref = None if null_out else ctypes.byref(h)
+    return lib.fftconv_plan_create(ref, B, H, N, dtype, gated), h
+
+
+@pytest.mark.parametrize("B,H,N,dtype,want", [
+    (0, 4, 1024, 0, 1), (1, 0, 1024, 0, 1), (1, 4, 1024, 7, 1),
+    (1, 4, 1000, 0, 2), (1, 4, 32, 0, 2), (1, 4, 1 << 21, 0, 2), (1, 4, 0, 0, 2), (1, 4, -1024, 0, 2),
+])
+def test_plan_create_rejects_before_any_cuda_call(lib, B, H, N, dtype, want):
+    st, h = _create(lib, B, H, N, dtype)
+    assert st == want
+    assert not h.value
+
+
+def test_plan_create_null_out(lib):
+    st, _ = _create(lib, 1, 4, 1024, null_out=True)
+    assert st == 1
+
+
+@pytest.mark.parametrize("B,C,Hs,Ws,want", [
+    (0, 1, 16, 16, 1), (1, 0, 16, 16, 1), (1, 1, 8, 16, 2), (1, 1, 16, 512, 2), (1, 1, 48, 64, 2),
+])
+def test_plan2d_create_rejects(lib, B, C, Hs, Ws, want):
+    h = ctypes.c_void_p()
+    assert lib.fftconv2d_plan_create(ctypes.byref(h), B, C, Hs, Ws, 1) == want
+    assert not h.value
+
+
+def test_null_plan_calls(lib):
+    assert lib.fftconv_fwd(None, None, None, None, None, None, None, None, None) == 1
+    assert lib.fftconv_kernel_spectrum(None, None, 1, None, None, None) == 1
+    assert lib.fftconv2d_fwd(None, None, None, None, None, None) == 1
+    assert lib.fftconv2d_kernel_spectrum(None, None, 1, 1, None, None, None) == 1
+    assert lib.fftconv_spectrum_bytes(None) == 0
+    assert lib.fftconv_workspace_bytes(None) == 0
+    assert lib.fftconv_plan_path(None) == b"none"
+    assert lib.fftconv_plan_destroy(None) == 0
+
+
+def test_binding_refuses_missing_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(build, "LIB", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(binding, "_LIB", None)
+    with pytest.raises(FileNotFoundError):
+        binding.load_library()

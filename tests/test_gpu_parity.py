@@ -1,0 +1,230 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU fp64 oracle.
+
+Small sizes are compared element by element over the whole output; the five
+named workloads run at full size in the launch configuration bench.py times
+and are compared on seeded samples of outputs that the oracle computes one by
+one, plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import scipy.signal
+import torch
+
+import oracle
+from fft_long_convolution_causal_b200 import workloads as wlmod
+from parity import assert_close, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fft_long_convolution_causal_b200 import binding
+    binding.load_library()
+
+
+def run_1d(wl, khat_plan=None):
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan(wl.B, wl.H, wl.N, wl.dtype, gated=wl.gated)
+    k = torch.from_numpy(wl.k).cuda()
+    khat = plan.kernel_spectrum(k)
+    u = to_dev(wl.u, wl.dtype)
+    v = to_dev(wl.v, wl.dtype)
+    w = to_dev(wl.w, wl.dtype)
+    D = torch.from_numpy(wl.D).cuda() if wl.D is not None else None
+    y = plan.fwd(u, khat, D=D, v=v, w=w)
+    torch.cuda.synchronize()
+    return to_host(y), plan.path
+
+
+def oracle_full(wl):
+    return oracle.causal_conv1d(wl.u, wl.k, D=wl.D, w=wl.w, v=wl.v)
+
+
+# ------------------------------------------------------------- small, full
+FUSED_N = [64, 128, 256, 512, 1024, 2048, 4096, 8192]
+
+
+@pytest.mark.parametrize("N", FUSED_N)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fused_full_compare(N, dtype):
+    wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
+    y, path = run_1d(wl)
+    assert path == "fused"
+    assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}")
+
+
+@pytest.mark.parametrize("N", [256, 4096, 8192])
+def test_fused_gated_full_compare(N):
+    wl = wlmod.make_1d(3, 3, N, dtype="bf16", gated=True, seed=7 + N, with_D=True)
+    y, _ = run_1d(wl)
+    assert_close(y, oracle_full(wl), "bf16", f"fused gated N={N}")
+    wl = wlmod.make_1d(2, 2, N, dtype="f32", gated=True, seed=8 + N, with_D=False)
+    y, _ = run_1d(wl)
+    assert_close(y, oracle_full(wl), "f32", f"fused gated f32 N={N}")
+
+
+@pytest.mark.parametrize("N,L", [(1024, 1), (1024, 100), (4096, 4095), (32768, 777), (65536, 40000)])
+def test_partial_kernel(N, L):
+    """k shorter than the sequence (a partial convolution): taps past L are zero."""
+    wl = wlmod.make_1d(2, 2, N, dtype="f32", seed=L, L=L, kernel="normal")
+    y, _ = run_1d(wl)
+    if N <= 32768:
+        ref = oracle_full(wl)
+        assert_close(y, ref, "f32", f"partial N={N} L={L}")
+    else:
+        b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 256, seed=L)
+        ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
+        assert_close(y[b, h, t], ref, "f32", f"partial N={N} L={L}")
+
+
+def test_no_skip_term_and_single_row():
+    wl = wlmod.make_1d(1, 5, 2048, dtype="f32", seed=3, with_D=False)
+    y, _ = run_1d(wl)
+    assert_close(y, oracle_full(wl), "f32", "B=1 no D")
+
+
+@pytest.mark.parametrize("N", [16384, 32768])
+@pytest.mark.parametrize("dtype,gated", [("f32", False), ("bf16", True), ("bf16", False)])
+def test_multipass_full_compare(N, dtype, gated):
+    wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=gated, seed=N + gated, with_D=True)
+    y, path = run_1d(wl)
+    assert path == "multipass"
+    assert_close(y, oracle_full(wl), dtype, f"multipass N={N} {dtype} gated={gated}")
+
+
+@pytest.mark.parametrize("log2N", [16, 17, 18, 19, 20])
+def test_multipass_sampled(log2N):
+    N = 1 << log2N
+    wl = wlmod.make_1d(3, 1, N, dtype="f32", seed=log2N, alpha=1e-5)
+    y, path = run_1d(wl)
+    assert path == "multipass"
+    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 400, seed=log2N)
+    ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
+    assert_close(y[b, h, t], ref, "f32", f"multipass N=2^{log2N}")
+
+
+def test_multipass_ragged_groups():
+    """More pairs than one workspace group holds, with a short last group."""
+    N = 1 << 20
+    wl = wlmod.make_1d(3, 5, N, dtype="bf16", seed=99, alpha=1e-5)
+    y, _ = run_1d(wl)
+    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 64, seed=99)
+    ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
+    assert_close(y[b, h, t], ref, "bf16", "ragged groups")
+
+
+@pytest.mark.parametrize("N", [4096, 1 << 20])
+def test_geometric_kernel_recursion_full_length(N):
+    """k[t] = c a^t gives y[t] = a y[t-1] + c u[t] (+ D u[t]): every output of a
+    full-length launch is checked against this O(N) recursion in fp64."""
+    rng = np.random.default_rng(5)
+    B, H = 2, 2
+    u = rng.standard_normal((B, H, N), dtype=np.float32)
+    a = np.array([0.9999, 0.99])
+    c = np.array([0.5, -1.5])
+    t = np.arange(N)
+    k = (c[:, None] * a[:, None] ** t[None, :]).astype(np.float32)
+    D = np.array([0.25, -2.0], dtype=np.float32)
+    wl = wlmod.Workload1D("geometric", B, H, N, "f32", False, u, k, D)
+    y, _ = run_1d(wl)
+    ref = np.empty((B, H, N))
+    for h in range(H):
+        # y[t] = a y[t-1] + c u[t], run as a first-order IIR filter in fp64
+        ref[:, h, :] = scipy.signal.lfilter([c[h]], [1.0, -a[h]], u[:, h, :].astype(np.float64), axis=-1)
+    ref += D[None, :, None].astype(np.float64) * u.astype(np.float64)
+    # k was rounded to fp32 (<= 2^-24 relative per tap); the error that induces
+    # in y is orders of magnitude inside the fp32 tolerance.
+    assert_close(y, ref, "f32", f"geometric recursion N={N}")
+
+
+# ------------------------------------------------ the named workloads, full size
+def _named(name):
+    return wlmod.make_config(name)
+
+
+def test_pr1_full():
+    wl = _named("pr1_b1_h4_n1024_f32")
+    y, path = run_1d(wl)
+    assert path == "fused"
+    assert_close(y, oracle_full(wl), "f32", wl.name)
+
+
+@pytest.mark.parametrize("name,per_row", [("hyena_b8_h768_n4096_bf16", 12),
+                                          ("gated_b4_h1024_n16384_bf16", 6),
+                                          ("long_b2_h64_n1048576_f32", 96)])
+def test_named_1d_sampled(name, per_row):
+    wl = _named(name)
+    y, _ = run_1d(wl)
+    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, wl.N, per_row, seed=1)
+    ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D, w=wl.w, v=wl.v)
+    assert_close(y[b, h, t], ref, wl.dtype, wl.name)
+
+
+# ------------------------------------------------------------------ 2-D
+def run_2d(wl):
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, wl.dtype)
+    khat = plan.kernel_spectrum(torch.from_numpy(wl.k).cuda())
+    y = plan.fwd(to_dev(wl.u, wl.dtype), khat)
+    torch.cuda.synchronize()
+    return to_host(y)
+
+
+@pytest.mark.parametrize("Hs,Ws", [(16, 16), (32, 64), (64, 32), (128, 128)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv2d_full_compare(Hs, Ws, dtype):
+    wl = wlmod.make_2d(3, 2, Hs, Ws, dtype=dtype, seed=Hs + Ws, sigma=Hs / 4)
+    y = run_2d(wl)
+    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), dtype, f"2d {Hs}x{Ws} {dtype}")
+
+
+def test_conv2d_small_kernel():
+    wl = wlmod.make_2d(2, 3, 64, 64, dtype="f32", seed=2, Kh=5, Kw=17)
+    y = run_2d(wl)
+    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel")
+
+
+def test_conv2d_named_sampled():
+    wl = _named("conv2d_b4_c256_256x256_bf16")
+    y = run_2d(wl)
+    idx = wlmod.sample_points_2d(wl.B, wl.C, wl.Hs, wl.Ws, 4096, seed=4)
+    ref = oracle.causal_conv2d_points(wl.u, wl.k, *idx)
+    assert_close(y[idx], ref, "bf16", wl.name)
+
+
+# ------------------------------------------------------------------ API on GPU
+def test_fwd_before_spectrum_is_not_ready():
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan(2, 2, 1024, "f32")
+    u = torch.zeros(2, 2, 1024, device="cuda")
+    khat = plan.new_spectrum()
+    with pytest.raises(binding.FFTConvError) as e:
+        plan.fwd(u, khat)
+    assert e.value.status == 3
+
+
+def test_misaligned_and_aliased_pointers_rejected():
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan(1, 1, 1024, "f32")
+    k = torch.randn(1, 1024, device="cuda")
+    khat = plan.kernel_spectrum(k)
+    buf = torch.zeros(1025 + 4, device="cuda")
+    lib = binding.load_library()
+    import ctypes
+    bad = ctypes.c_void_p(buf.data_ptr() + 4)
+    ok = ctypes.c_void_p(buf.data_ptr())
+    st = lib.fftconv_fwd(plan._handle, bad, None, None, ctypes.c_void_p(khat.data_ptr()), None, ok, None,
+                         None)
+    assert st == 1
+    st = lib.fftconv_fwd(plan._handle, ok, None, None, ctypes.c_void_p(khat.data_ptr()), None, ok, None, None)
+    assert st == 1
+
+
+def test_repeated_calls_are_deterministic():
+    wl = wlmod.make_1d(4, 8, 4096, dtype="bf16", seed=17)
+    y1, _ = run_1d(wl)
+    y2, _ = run_1d(wl)
+    assert np.array_equal(y1, y2)
