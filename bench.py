@@ -40,7 +40,7 @@ METRIC = "FFT-conv output elems/s and % of HBM roofline (1 B200), N=1K–1M and 
 DEFAULT_CONFIG = "hyena_b8_h768_n4096_bf16"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ["fft_simt.cuh", "conv1d_simt.cu", "conv2d_simt.cu"]
+KERNEL_SOURCES = ["fft_simt.cuh", "conv1d_simt.cu", "conv2d_simt.cu", "conv1d_mma.cu"]
 
 
 def parse():
@@ -200,7 +200,7 @@ class Runner:
                           y=y, workspace=self.ws)
 
     def launches_per_step(self):
-        if self.plan.path == "fused":
+        if self.plan.path in ("fused", "fused_tc"):
             return 1
         pairs = ((self.wl.B + 1) // 2) * (self.wl.C if self.is2d else self.wl.H)
         group = max(1, self.plan.workspace_bytes // self._pair_bytes())
@@ -212,10 +212,11 @@ class Runner:
         return 2 * self.wl.N * 8
 
     def compute_dtype(self):
-        return {"fused": "f32", "multipass": "f32", "2d": "f32"}.get(self.plan.path, "f32")
+        return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16"}.get(self.plan.path, "f32")
 
     def dominant_kernel(self):
-        return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2"}.get(self.plan.path)
+        return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2",
+                "fused_tc": "fused_fwd_tc"}.get(self.plan.path)
 
 
 def time_steps(r, steps, torch, flush):
@@ -299,7 +300,7 @@ class OracleSampler:
         while dt < 0.25 and n < 1 << 26:
             n *= 4
             dt = self.run(n)
-        return int(min(max(n * target_s / max(dt, 1e-6), 64), 1 << 27))
+        return int(min(max(n * target_s / max(dt, 1e-6), 64), self.total))
 
     def describe(self, n, dt):
         return (f"{n} uniformly drawn outputs of {self.total} (direct fp64 sum per output), "

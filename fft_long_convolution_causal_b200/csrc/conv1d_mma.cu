@@ -1,0 +1,558 @@
+// conv1d_mma.cu -- fused bf16 tensor-core kernel of the 1-D causal FFT convolution.
+//
+// The DFT of length M = 2N is computed as a Monarch (four-step) product of
+// small dense DFT matrices on the tensor cores, the matrix decomposition that
+// "FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores"
+// (abstract) uses to run the FFT on matrix-multiply units, fused with the
+// pointwise product and the inverse in one kernel as in "FlashConv"
+// (Mechanism: FFT, pointwise product and inverse FFT on chip; block FFT as
+// matrix multiplications).  Two batch rows b, b+1 of channel h travel as one
+// complex sequence z = x_b + i x_{b+1}; x is zero-padded to M and y truncated
+// to [:N] ("RubiConv -- Efficient Boundary-Respecting Convolutions", Caracal
+// abstract).
+//
+// Index split, M = P * 256:   n = 256 p + q,  k = k_p + P (c + 16 d),  q = 16 a + b.
+//   step 1 (outer): for each q, DFT_P over p < P/2 (the nonzero half), times
+//                   W_M^{q k_p}  -> S[k_p][q]
+//   step 3 (inner, one warp per row k_p): 256-point DFT as 16 x 16:
+//                   over a -> c, times W_256^{b c}, transpose, over b -> d;
+//                   times Khat[k] (+ D/M); inverse in reverse order; times
+//                   W_M^{-q k_p}                                 -> S[k_p][q]
+//   step 1' (outer inverse): for each q, inverse DFT_P over k_p, only p < P/2.
+// Every DFT stage is a complex product of a bf16 tile (data, the A operand
+// of mma.sync m16n8k16) with a bf16 DFT matrix (the B operand), accumulated
+// in fp32: Yr = Xr Fr - Xi Fi, Yi = Xr Fi + Xi Fr.  Accumulator fragments are
+// reused directly as the next A fragments; the 16 x 16 transpose between the
+// inner stages is done in registers (movmatrix).  S lives in shared memory as
+// two bf16 planes (re, im), rows k_p of 256 q, 16-byte chunks XOR-swizzled so
+// that both the row-wise (step 3) and the column-wise (steps 1, 1')
+// ldmatrix / stmatrix accesses are free of bank conflicts.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "fft_simt.cuh"
+#include "plan.h"
+#include "tables.h"
+
+namespace fftc {
+namespace tc {
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t movt(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+// two fp32 -> packed bf16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ __nv_bfloat162 as_b2(uint32_t x) { return *reinterpret_cast<__nv_bfloat162*>(&x); }
+__device__ __forceinline__ uint32_t as_u(__nv_bfloat162 x) { return *reinterpret_cast<uint32_t*>(&x); }
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Packed complex multiply on two adjacent elements: (re, im) pairs times
+// (cos, sin) pairs.  FWD: z (c - i s);  otherwise z (c + i s).
+template <bool FWD>
+__device__ __forceinline__ void twiddle2(uint32_t& re, uint32_t& im, uint2 cs) {
+    const __nv_bfloat162 r = as_b2(re), i = as_b2(im), c = as_b2(cs.x), s = as_b2(cs.y);
+    if (FWD) {
+        re = as_u(__hfma2(r, c, __hmul2(i, s)));
+        im = as_u(__hfma2(i, c, __hneg2(__hmul2(r, s))));
+    } else {
+        re = as_u(__hfma2(r, c, __hneg2(__hmul2(i, s))));
+        im = as_u(__hfma2(i, c, __hmul2(r, s)));
+    }
+}
+
+// Complex tile product on one 16 x 8 output tile:
+//   yr += Ar Br + Ai Bni,   yi += Ar Bi + Ai Br     (Bni = -Bi)
+__device__ __forceinline__ void cmma(float (&yr)[4], float (&yi)[4], const uint32_t (&ar)[4],
+                                     const uint32_t (&ai)[4], uint2 br, uint2 bi, uint2 bni) {
+    mma16816(yr, ar, br.x, br.y);
+    mma16816(yr, ai, bni.x, bni.y);
+    mma16816(yi, ar, bi.x, bi.y);
+    mma16816(yi, ai, br.x, br.y);
+}
+
+// ------------------------------------------------------------ smem layout
+// Plane row = 256 bf16 = 32 chunks of 16 B.  Chunk c of row r is stored at
+// chunk (c4 c0 ((c3 c2 c1) ^ r)) -- a bijection per row that makes 8 chunks
+// {2a + cb : 8 consecutive a} of one row, and one chunk of 8 consecutive rows,
+// land on 8 distinct 16-byte bank groups.
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
+    return (chunk & 16u) | ((chunk & 1u) << 3) | (((chunk >> 1) ^ row) & 7u);
+}
+__device__ __forceinline__ uint32_t plane_addr(uint32_t base, uint32_t row, uint32_t chunk) {
+    return base + row * 512u + swz(row, chunk) * 16u;
+}
+
+using TcTables = TcTablePtrs;
+
+template <int P>
+struct TcShape {
+    static constexpr int kLog2P = ilog2(P);
+    static constexpr int M = P * 256;
+    static constexpr int N = M / 2;
+    static constexpr int NT1 = P / 8;                   // step-1 output n-tiles (k_p)
+    static constexpr int KS1 = (P / 2 + 15) / 16;       // step-1 k-steps (p < P/2)
+    static constexpr int NT3 = (P / 2 + 7) / 8;         // step-1' output n-tiles (p < P/2)
+    static constexpr int KS3 = P / 16;                  // step-1' k-steps (k_p)
+    static constexpr int kPlaneBytes = P * 512;         // one bf16 plane, P rows of 256
+    static constexpr int kSmemPerPair = 2 * kPlaneBytes;
+};
+
+// ================================================================== kernel
+template <int P, int NW, bool GATED>
+__global__ void __launch_bounds__(NW * 32)
+fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
+             const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
+             __nv_bfloat16* __restrict__ y, TcTables tb, int B, int H) {
+    using S = TcShape<P>;
+    static_assert(P >= 16 && P <= 64, "outer factor");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.y;
+    const int b0 = 2 * blockIdx.x;
+    const bool has1 = b0 + 1 < B;
+    const size_t row0 = ((size_t)b0 * H + h) * S::N;
+    const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
+    const uint32_t sre = smem_u32(smem), sim = sre + S::kPlaneBytes;
+
+    // ---- stage x = u (or u*w) into the planes: rows p < P/2, natural q
+    {
+        constexpr int CH = S::N / 8;  // 16-byte chunks per row of u
+        for (int i = tid; i < 2 * CH; i += NW * 32) {
+            const int plane = i / CH, ci = i % CH;  // plane 0: row b (re), 1: row b+1 (im)
+            const int n0 = ci * 8;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (plane == 0 || has1) {
+                const size_t off = (plane ? row1 : row0) + n0;
+                val = __ldg(reinterpret_cast<const uint4*>(u + off));
+                if (GATED) {
+                    const uint4 ww = __ldg(reinterpret_cast<const uint4*>(w + off));
+                    val.x = as_u(__hmul2(as_b2(val.x), as_b2(ww.x)));
+                    val.y = as_u(__hmul2(as_b2(val.y), as_b2(ww.y)));
+                    val.z = as_u(__hmul2(as_b2(val.z), as_b2(ww.z)));
+                    val.w = as_u(__hmul2(as_b2(val.w), as_b2(ww.w)));
+                }
+            }
+            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+            const uint32_t addr = plane_addr(plane ? sim : sre, p, chunk);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(val.x), "r"(val.y), "r"(val.z),
+                         "r"(val.w)
+                         : "memory");
+        }
+    }
+    // inner DFT_16 fragments and W_256 twiddles (same for every row)
+    uint2 f16[3][2], w256[4];
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+    __syncthreads();
+
+    const int m8 = lane >> 3, r8 = lane & 7;
+
+    // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
+    for (int qt = warp; qt < 16; qt += NW) {
+        uint32_t ar[S::KS1][4], ai[S::KS1][4];
+#pragma unroll
+        for (int ks = 0; ks < S::KS1; ++ks) {
+            // A[q][p]: matrices (q 0-7|8-15) x (p 0-7|8-15) from rows p, chunks 2 qt (+1)
+            // rows p >= P/2 are the zero padding: those lanes point at row 0 (a
+            // select, not a branch: ldmatrix must run warp-converged) and the
+            // registers they feed are zeroed below
+            const uint32_t prow0 = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+            const uint32_t prow = prow0 < (uint32_t)(P / 2) ? prow0 : 0u;
+            ldsm_x4_t(ar[ks], plane_addr(sre, prow, chunk));
+            ldsm_x4_t(ai[ks], plane_addr(sim, prow, chunk));
+            if (16 * ks + 8 >= P / 2) {  // p 8-15 of this k-step are padding
+                ar[ks][2] = ar[ks][3] = ai[ks][2] = ai[ks][3] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < S::NT1; ++j) {
+            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < S::KS1; ++ks) {
+                const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
+                cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+            }
+            // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
+            uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
+            uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                twiddle2<true>(pr[hh], pi[hh], __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + hh) * 32 + lane]));
+            // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
+            const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
+        }
+    }
+    __syncthreads();
+
+    // ---- step 3: inner 256-point DFT, product with Khat, inverse, per row k_p
+    const float dm = D ? D[h] * (1.0f / S::M) : 0.f;
+    const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
+    for (int kp = warp; kp < P; kp += NW) {
+        uint32_t xr[4], xi[4];
+        {
+            const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
+            ldsm_x4_t(xr, plane_addr(sre, kp, chunk));
+            ldsm_x4_t(xi, plane_addr(sim, kp, chunk));
+        }
+        // stage i: [b][a] x F16 -> [b][c]
+        float ur[2][4] = {}, ui[2][4] = {};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) cmma(ur[j], ui[j], xr, xi, f16[0][j], f16[1][j], f16[2][j]);
+        uint32_t tr[4] = {pack2(ur[0][0], ur[0][1]), pack2(ur[0][2], ur[0][3]), pack2(ur[1][0], ur[1][1]),
+                          pack2(ur[1][2], ur[1][3])};
+        uint32_t ti[4] = {pack2(ui[0][0], ui[0][1]), pack2(ui[0][2], ui[0][3]), pack2(ui[1][0], ui[1][1]),
+                          pack2(ui[1][2], ui[1][3])};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+        // transpose [b][c] -> [c][b]
+        uint32_t cr[4] = {movt(tr[0]), movt(tr[2]), movt(tr[1]), movt(tr[3])};
+        uint32_t ci[4] = {movt(ti[0]), movt(ti[2]), movt(ti[1]), movt(ti[3])};
+        // stage ii: [c][b] x F16 -> [c][d]  (spectrum at k = k_p + P (c + 16 d))
+        float vr[2][4] = {}, vi[2][4] = {};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) cmma(vr[j], vi[j], cr, ci, f16[0][j], f16[1][j], f16[2][j]);
+        // pointwise product with Khat (+ D/M), in fp32
+        const uint4 k0 = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
+        const uint4 k1 = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
+        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t kk = kw[j * 4 + e];
+                const float kr = __uint_as_float(kk << 16) + dm, ki = __uint_as_float(kk & 0xffff0000u);
+                const float zr = vr[j][e], zi = vi[j][e];
+                vr[j][e] = fmaf(zr, kr, -zi * ki);
+                vi[j][e] = fmaf(zr, ki, zi * kr);
+            }
+        // inverse stage ii: [c][d] x conj(F16) -> [c][b]
+        uint32_t zr4[4] = {pack2(vr[0][0], vr[0][1]), pack2(vr[0][2], vr[0][3]), pack2(vr[1][0], vr[1][1]),
+                           pack2(vr[1][2], vr[1][3])};
+        uint32_t zi4[4] = {pack2(vi[0][0], vi[0][1]), pack2(vi[0][2], vi[0][3]), pack2(vi[1][0], vi[1][1]),
+                           pack2(vi[1][2], vi[1][3])};
+        float sr[2][4] = {}, si[2][4] = {};
+        // conj(F16) = Fr - i Fi: parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
+#pragma unroll
+        for (int j = 0; j < 2; ++j) cmma(sr[j], si[j], zr4, zi4, f16[0][j], f16[2][j], f16[1][j]);
+        uint32_t gr[4] = {pack2(sr[0][0], sr[0][1]), pack2(sr[0][2], sr[0][3]), pack2(sr[1][0], sr[1][1]),
+                          pack2(sr[1][2], sr[1][3])};
+        uint32_t gi[4] = {pack2(si[0][0], si[0][1]), pack2(si[0][2], si[0][3]), pack2(si[1][0], si[1][1]),
+                          pack2(si[1][2], si[1][3])};
+        // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
+        uint32_t hr[4] = {movt(gr[0]), movt(gr[2]), movt(gr[1]), movt(gr[3])};
+        uint32_t hi[4] = {movt(gi[0]), movt(gi[2]), movt(gi[1]), movt(gi[3])};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<false>(hr[i], hi[i], w256[i]);
+        // inverse stage i: [b][c] x conj(F16) -> [b][a]
+        float or_[2][4] = {}, oi[2][4] = {};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) cmma(or_[j], oi[j], hr, hi, f16[0][j], f16[2][j], f16[1][j]);
+        uint32_t qr[4] = {pack2(or_[0][0], or_[0][1]), pack2(or_[0][2], or_[0][3]), pack2(or_[1][0], or_[1][1]),
+                          pack2(or_[1][2], or_[1][3])};
+        uint32_t qi[4] = {pack2(oi[0][0], oi[0][1]), pack2(oi[0][2], oi[0][3]), pack2(oi[1][0], oi[1][1]),
+                          pack2(oi[1][2], oi[1][3])};
+        // conj twiddle W_M^{-q k_p}, q = 16 a + b
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]));
+        // back to row k_p (fragment [b][a] stored transposed: rows a, natural q)
+        {
+            const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
+            // registers: 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3 (b 8-15, a 8-15)
+            stsm_x4_t(plane_addr(sre, kp, chunk), qr[0], qr[1], qr[2], qr[3]);
+            stsm_x4_t(plane_addr(sim, kp, chunk), qi[0], qi[1], qi[2], qi[3]);
+        }
+    }
+    __syncthreads();
+
+    // ---- step 1': inverse outer DFT over k_p, outputs p < P/2, into rows p
+    for (int qt = warp; qt < 16; qt += NW) {
+        uint32_t ar[S::KS3][4], ai[S::KS3][4];
+#pragma unroll
+        for (int ks = 0; ks < S::KS3; ++ks) {
+            const uint32_t krow = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+            ldsm_x4_t(ar[ks], plane_addr(sre, krow, chunk));
+            ldsm_x4_t(ai[ks], plane_addr(sim, krow, chunk));
+        }
+#pragma unroll
+        for (int j = 0; j < S::NT3; ++j) {
+            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < S::KS3; ++ks) {
+                const uint2* fb = tb.fpi + ((size_t)(ks * S::NT3 + j) * 3) * 32 + lane;
+                cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+            }
+            // rows q = 16 qt + g (+8), cols p = 8 j + 2t (+1) -> rows p, chunk 2 qt (+1)
+            const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk), pack2(yr[0], yr[1]), pack2(yr[2], yr[3]),
+                      pack2(yi[0], yi[1]), pack2(yi[2], yi[3]));
+        }
+    }
+    __syncthreads();
+
+    // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
+    {
+        constexpr int CH = S::N / 8;
+        for (int i = tid; i < 2 * CH; i += NW * 32) {
+            const int plane = i / CH, ci = i % CH;
+            if (plane == 1 && !has1) continue;
+            const int n0 = ci * 8;
+            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(plane_addr(plane ? sim : sre, p, chunk)));
+            const size_t off = (plane ? row1 : row0) + n0;
+            if (GATED) {
+                const uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + off));
+                val.x = as_u(__hmul2(as_b2(val.x), as_b2(vv.x)));
+                val.y = as_u(__hmul2(as_b2(val.y), as_b2(vv.y)));
+                val.z = as_u(__hmul2(as_b2(val.z), as_b2(vv.z)));
+                val.w = as_u(__hmul2(as_b2(val.w), as_b2(vv.w)));
+            }
+            *reinterpret_cast<uint4*>(y + off) = val;
+        }
+    }
+}
+
+// Spectrum in the kernel's fragment order: the SIMT transform of k[h]
+// (natural order, fp32, in shared memory), then per row k_p and lane the 8
+// values (j, e) at k = k_p + P (c + 16 d), c = g + 8 (e >> 1),
+// d = 8 j + 2 t + (e & 1), scaled by 1/M and rounded to bf16 (re, im).
+template <int LOG2M>
+__global__ void __launch_bounds__(Geometry<LOG2M, 1, false>::T)
+tc_spectrum(const float* __restrict__ k, int L, uint32_t* __restrict__ khat, const float2* __restrict__ tw) {
+    using G = Geometry<LOG2M, 1, false>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, NS = G::Plan::kStages, P = M / 256;
+    constexpr int R0 = 1 << G::Plan::log2r(0);
+    extern __shared__ float2 smem2[];
+    const int tid = threadIdx.x, h = blockIdx.x;
+    const float* __restrict__ kr = k + (size_t)h * L;
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return make_float2(n < L ? kr[n] : 0.f, 0.f); },
+        [&](int i, int, float2 z) { smem2[Lay::at(i, 0)] = z; });
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(smem2, tid, tw);
+    uint32_t* out = khat + (size_t)h * M;
+    for (int o = tid; o < M; o += G::T) {
+        const int kp = o / 256, rem = o % 256, lane = rem / 8, je = rem % 8;
+        const int j = je / 4, e = je % 4, g = lane >> 2, t = lane & 3;
+        const int c = g + 8 * (e >> 1), d = 8 * j + 2 * t + (e & 1);
+        const float2 z = cscale(smem2[Lay::at(kp + P * (c + 16 * d), 0)], 1.0f / M);
+        out[o] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.x)) |
+                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.y)) << 16);
+    }
+}
+
+}  // namespace tc
+
+// ================================================================== host side
+namespace {
+
+uint16_t bf16_bits(double x) {
+    const float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+uint32_t pack_host(double lo, double hi) { return (uint32_t)bf16_bits(lo) | ((uint32_t)bf16_bits(hi) << 16); }
+
+void push_u2(std::vector<float2>& out, uint32_t x, uint32_t y) {
+    float2 f;
+    memcpy(&f.x, &x, 4);
+    memcpy(&f.y, &y, 4);
+    out.push_back(f);
+}
+
+// cos and sin of 2 pi e / L, e reduced mod L, in fp64
+void cs(int64_t e, int64_t L, double* c, double* s) {
+    int64_t r = e % L;
+    if (r < 0) r += L;
+    const double a = 2.0 * M_PI * (double)r / (double)L;
+    *c = cos(a);
+    *s = sin(a);
+}
+
+// B fragments of a complex K x N matrix G given by value(k, n) -> (re, im):
+// [ks][ntile][part (Re, Im, -Im)][lane] with b0b1 = (k = 2t, 2t+1), b2b3 = (k = 2t+8, 2t+9), n = g.
+template <class F>
+void push_bfrags(std::vector<float2>& out, int ksteps, int ntiles, F value) {
+    for (int ks = 0; ks < ksteps; ++ks)
+        for (int j = 0; j < ntiles; ++j)
+            for (int part = 0; part < 3; ++part)
+                for (int lane = 0; lane < 32; ++lane) {
+                    const int g = lane >> 2, t = lane & 3, n = 8 * j + g;
+                    double v[4];
+                    const int ks4[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+                    for (int q = 0; q < 4; ++q) {
+                        double re, im;
+                        value(16 * ks + ks4[q], n, &re, &im);
+                        v[q] = part == 0 ? re : (part == 1 ? im : -im);
+                    }
+                    push_u2(out, pack_host(v[0], v[1]), pack_host(v[2], v[3]));
+                }
+}
+
+}  // namespace
+
+bool tc_supported(int log2M) { return log2M >= 12 && log2M <= 14; }
+
+bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]) {
+    if (!tc_supported(log2M)) return false;
+    const int64_t M = int64_t(1) << log2M;
+    const int P = (int)(M / 256);
+    const int NT1 = P / 8, KS1 = (P / 2 + 15) / 16, NT3 = (P / 2 + 7) / 8, KS3 = P / 16;
+    // f16: DFT_16, B[k][n] = W_16^{k n}
+    off[0] = out.size();
+    push_bfrags(out, 1, 2, [](int k, int n, double* re, double* im) {
+        double c, s;
+        cs((int64_t)k * n, 16, &c, &s);
+        *re = c;
+        *im = -s;
+    });
+    // w256: (cos, sin) pairs of W_256^{b c}; reg i: b = g + 8 (i & 1), c = 2t + 8 (i >> 1) + {0, 1}
+    off[1] = out.size();
+    for (int i = 0; i < 4; ++i)
+        for (int lane = 0; lane < 32; ++lane) {
+            const int g = lane >> 2, t = lane & 3, b = g + 8 * (i & 1), c0 = 2 * t + 8 * (i >> 1);
+            double ca, sa, cb, sb;
+            cs((int64_t)b * c0, 256, &ca, &sa);
+            cs((int64_t)b * (c0 + 1), 256, &cb, &sb);
+            push_u2(out, pack_host(ca, cb), pack_host(sa, sb));
+        }
+    // fp: outer forward, B[k = p][n = k_p] = W_P^{p k_p} for p < P/2, else 0
+    off[2] = out.size();
+    push_bfrags(out, KS1, NT1, [P](int k, int n, double* re, double* im) {
+        if (k >= P / 2) {
+            *re = *im = 0.0;
+            return;
+        }
+        double c, s;
+        cs((int64_t)k * n, P, &c, &s);
+        *re = c;
+        *im = -s;
+    });
+    // fpi: outer inverse, B[k = k_p][n = p] = conj(W_P^{k_p p}) for p < P/2, else 0
+    off[3] = out.size();
+    push_bfrags(out, KS3, NT3, [P](int k, int n, double* re, double* im) {
+        if (n >= P / 2) {
+            *re = *im = 0.0;
+            return;
+        }
+        double c, s;
+        cs((int64_t)k * n, P, &c, &s);
+        *re = c;
+        *im = s;
+    });
+    // tw1: (cos, sin) of W_M^{q k_p}, [qt][j][hh][lane]: q = 16 qt + g + 8 hh, k_p = 8 j + 2 t + {0, 1}
+    off[4] = out.size();
+    for (int qt = 0; qt < 16; ++qt)
+        for (int j = 0; j < NT1; ++j)
+            for (int hh = 0; hh < 2; ++hh)
+                for (int lane = 0; lane < 32; ++lane) {
+                    const int g = lane >> 2, t = lane & 3;
+                    const int64_t q = 16 * qt + g + 8 * hh, k0 = 8 * j + 2 * t;
+                    double ca, sa, cb, sb;
+                    cs(q * k0, M, &ca, &sa);
+                    cs(q * (k0 + 1), M, &cb, &sb);
+                    push_u2(out, pack_host(ca, cb), pack_host(sa, sb));
+                }
+    // tw3: (cos, sin) of W_M^{q k_p}, [k_p][reg][lane]: b = g + 8 (i & 1), a = 2t + 8 (i >> 1) + {0, 1}
+    off[5] = out.size();
+    for (int kp = 0; kp < P; ++kp)
+        for (int i = 0; i < 4; ++i)
+            for (int lane = 0; lane < 32; ++lane) {
+                const int g = lane >> 2, t = lane & 3, b = g + 8 * (i & 1), a0 = 2 * t + 8 * (i >> 1);
+                double ca, sa, cb, sb;
+                cs((int64_t)(16 * a0 + b) * kp, M, &ca, &sa);
+                cs((int64_t)(16 * (a0 + 1) + b) * kp, M, &cb, &sb);
+                push_u2(out, pack_host(ca, cb), pack_host(sa, sb));
+            }
+    return true;
+}
+
+template <int P, bool GATED>
+static cudaError_t tc_fwd_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                             const void* khat, const float* D, void* y, cudaStream_t s) {
+    constexpr int NW = 4;
+    auto kern = tc::fused_fwd_tc<P, NW, GATED>;
+    const size_t smem = tc::TcShape<P>::kSmemPerPair;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((p.B + 1) / 2, p.H);
+    kern<<<grid, NW * 32, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
+                                     (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.B, p.H);
+    return cudaGetLastError();
+}
+
+template <int P>
+static cudaError_t tc_fwd_g(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
+                            const float* D, void* y, cudaStream_t s) {
+    return p.gated ? tc_fwd_go<P, true>(p, u, v, w, khat, D, y, s) : tc_fwd_go<P, false>(p, u, v, w, khat, D, y, s);
+}
+
+cudaError_t launch_tc_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
+                          const float* D, void* y, cudaStream_t s) {
+    switch (p.log2M) {
+        case 12: return tc_fwd_g<16>(p, u, v, w, khat, D, y, s);
+        case 13: return tc_fwd_g<32>(p, u, v, w, khat, D, y, s);
+        case 14: return tc_fwd_g<64>(p, u, v, w, khat, D, y, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int LOG2M>
+static cudaError_t tc_spec_go(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s) {
+    using G = Geometry<LOG2M, 1, false>;
+    auto kern = tc::tc_spectrum<LOG2M>;
+    const size_t smem = G::Lay::kWords * sizeof(float2);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<p.H, G::T, smem, s>>>(k, (int)L, (uint32_t*)khat, p.tw.wL);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s) {
+    switch (p.log2M) {
+        case 12: return tc_spec_go<12>(p, k, L, khat, s);
+        case 13: return tc_spec_go<13>(p, k, L, khat, s);
+        case 14: return tc_spec_go<14>(p, k, L, khat, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace fftc

@@ -25,6 +25,7 @@
 // (L2-sized) and is reused group after group.
 #include "fft_simt.cuh"
 #include "plan.h"
+#include "tables.h"
 
 namespace fftc {
 
@@ -167,6 +168,16 @@ static cudaError_t fused_spec_go(const fftconv_plan_s& p, const float* k, int64_
     ensure_smem(kern, smem);
     kern<<<p.H, FusedG<LOG2M>::T, smem, s>>>(k, (int)L, khat, p.tw.wL);
     return cudaGetLastError();
+}
+
+bool fused_tables(int log2M, std::vector<float2>& out, size_t* offL) {
+    *offL = out.size();
+    switch (log2M) {
+#define FFTC_T(X) case X: append_stage_twiddles<FusedG<X>>(out); return true;
+        FFTC_T(7) FFTC_T(8) FFTC_T(9) FFTC_T(10) FFTC_T(11) FFTC_T(12) FFTC_T(13) FFTC_T(14)
+#undef FFTC_T
+        default: return false;
+    }
 }
 
 cudaError_t launch_fused_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
@@ -405,6 +416,28 @@ static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L
         case 21: return CALL(10, 11);    \
         default: return cudaErrorInvalidValue; \
     }
+
+template <int LOG2N1, int LOG2N2>
+static bool mp_tables_go(std::vector<float2>& out, size_t* offC, size_t* offR) {
+    *offC = out.size();
+    append_stage_twiddles<ColG<LOG2N1>>(out);
+    *offR = out.size();
+    append_stage_twiddles<RowG<LOG2N2>>(out);
+    return true;
+}
+
+bool multipass_tables(int log2M, std::vector<float2>& out, size_t* offC, size_t* offR) {
+    switch (log2M) {
+        case 15: return mp_tables_go<7, 8>(out, offC, offR);
+        case 16: return mp_tables_go<8, 8>(out, offC, offR);
+        case 17: return mp_tables_go<8, 9>(out, offC, offR);
+        case 18: return mp_tables_go<9, 9>(out, offC, offR);
+        case 19: return mp_tables_go<9, 10>(out, offC, offR);
+        case 20: return mp_tables_go<10, 10>(out, offC, offR);
+        case 21: return mp_tables_go<10, 11>(out, offC, offR);
+        default: return false;
+    }
+}
 
 cudaError_t launch_multipass_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
                                  const float2* khat, const float* D, void* y, float2* work, cudaStream_t s) {

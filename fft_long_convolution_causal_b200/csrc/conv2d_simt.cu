@@ -13,6 +13,7 @@
 //   pass 3: inverse row DFT_{2Ws} of the Hs rows, keeping j < Ws -> y.
 #include "fft_simt.cuh"
 #include "plan.h"
+#include "tables.h"
 
 namespace fftc {
 
@@ -227,6 +228,37 @@ static cudaError_t c2_spec_w(const fftconv_plan_s& p, const float* k, int Kh, in
         FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
 #undef FFTC_C
         default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int LOG2LC, int LOG2LR>
+static bool c2_tables_go(std::vector<float2>& out, size_t* offR, size_t* offC) {
+    constexpr int RB = rows_per_cta<LOG2LR>((1 << LOG2LC) / 2);
+    *offR = out.size();
+    append_stage_twiddles<Row2G<LOG2LR, RB>>(out);
+    *offC = out.size();
+    append_stage_twiddles<Col2G<LOG2LC>>(out);
+    return true;
+}
+
+template <int LOG2LC>
+static bool c2_tables_w(int Ws, std::vector<float2>& out, size_t* offR, size_t* offC) {
+    switch (ilog2_host(Ws)) {
+#define FFTC_C(LW) case LW: return c2_tables_go<LOG2LC, LW + 1>(out, offR, offC);
+        FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
+#undef FFTC_C
+        default: return false;
+    }
+}
+
+bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_t* offC) {
+    switch (ilog2_host(Hs)) {
+        case 4: return c2_tables_w<5>(Ws, out, offR, offC);
+        case 5: return c2_tables_w<6>(Ws, out, offR, offC);
+        case 6: return c2_tables_w<7>(Ws, out, offR, offC);
+        case 7: return c2_tables_w<8>(Ws, out, offR, offC);
+        case 8: return c2_tables_w<9>(Ws, out, offR, offC);
+        default: return false;
     }
 }
 

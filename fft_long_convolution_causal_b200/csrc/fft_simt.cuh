@@ -170,6 +170,18 @@ struct Geometry {
     using Lay = Layout<L, C, BF>;
 };
 
+// Twiddles of every stage of a geometry, one table: stage s holds
+// W_{Ns R}^{r k} at offset(s) + r Ns + k for r < R, k < Ns.
+template <class G>
+struct StageTwiddles {
+    static constexpr int offset(int s) {
+        int o = 0;
+        for (int i = 0; i < s; ++i) o += (1 << G::Plan::log2r(i)) << G::Plan::log2ns(i);
+        return o;
+    }
+    static constexpr int total() { return offset(G::Plan::kStages); }
+};
+
 // Butterfly id -> (j, c).  Consecutive ids walk the fast axis of the layout.
 template <class G, int R>
 __device__ __forceinline__ void bfly_coords(int bid, int& j, int& c) {
@@ -208,10 +220,11 @@ __device__ __forceinline__ void stage(int tid, const float2* __restrict__ tw, Lo
         bfly_coords<G, R>(tid + q * G::T, j, c);
         const int k = j & (NS - 1);
         if (LOG2NS > 0) {
-            // W_{Ns R}^{r k} = W_L^{r k L / (Ns R)}
-            const int step = k << (G::LOG2L - LOG2NS - LOG2R);
+            // W_{Ns R}^{r k} from the stage's table, laid out [r][k] so that the
+            // consecutive k of a warp read consecutive entries
+            constexpr int OFF = StageTwiddles<G>::offset(S);
 #pragma unroll
-            for (int r = 1; r < IN_R; ++r) v[q][r] = cmul_dir<INV>(v[q][r], __ldg(&tw[r * step]));
+            for (int r = 1; r < IN_R; ++r) v[q][r] = cmul_dir<INV>(v[q][r], __ldg(&tw[OFF + r * NS + k]));
         }
         dft<R, INV>(v[q]);
         const int base = ((j >> LOG2NS) << (LOG2NS + LOG2R)) + k;

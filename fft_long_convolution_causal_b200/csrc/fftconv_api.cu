@@ -92,9 +92,17 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
     cudaGetDevice(&p->device);
     std::vector<float2> host;
     const int64_t M = int64_t(1) << p->log2M;
-    if (p->log2M <= kFusedMaxLog2M) {
+    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[6] = {0, 0, 0, 0, 0, 0};
+    const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && !getenv("FFTCONV_NO_TC");
+    if (use_tc) {
+        p->path = fftc::PATH_FUSED_TC;
+        fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the spectrum transform
+        fftc::tc_tables(p->log2M, host, offTc);
+        p->spectrum_bytes = (size_t)H * M * sizeof(uint32_t);  // bf16 (re, im) in fragment order
+        p->workspace_bytes = 0;
+    } else if (p->log2M <= kFusedMaxLog2M) {
         p->path = fftc::PATH_FUSED;
-        fill_roots(host, M, M);
+        fftc::fused_tables(p->log2M, host, &offL);
         p->spectrum_bytes = (size_t)H * M * sizeof(float2);
         p->workspace_bytes = 0;
     } else {
@@ -102,11 +110,11 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         p->log2N1 = p->log2M / 2;
         p->log2N2 = p->log2M - p->log2N1;
         p->log2S = (p->log2M + 1) / 2;
-        const int64_t N1 = int64_t(1) << p->log2N1, N2 = int64_t(1) << p->log2N2;
         const int64_t S = int64_t(1) << p->log2S;
-        fill_roots(host, N2, N2);                 // wL
-        fill_roots(host, N1, N1);                 // wC
+        fftc::multipass_tables(p->log2M, host, &offC, &offL);
+        offLo = host.size();
         fill_roots(host, M, S);                   // wLo: W_M^e, e < S
+        offHi = host.size();
         fill_roots(host, M, M / S, S);            // wHi: W_M^(e S)
         const size_t per_pair = (size_t)M * sizeof(float2);
         int64_t g = (int64_t)(kGroupBytes / per_pair);
@@ -123,15 +131,19 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         return st;
     }
     const float2* base = (const float2*)p->d_tables;
-    if (p->path == fftc::PATH_FUSED) {
-        p->tw.wL = base;
-    } else {
-        const int64_t N1 = int64_t(1) << p->log2N1, N2 = int64_t(1) << p->log2N2;
-        const int64_t S = int64_t(1) << p->log2S;
-        p->tw.wL = base;
-        p->tw.wC = base + N2;
-        p->tw.wLo = base + N2 + N1;
-        p->tw.wHi = base + N2 + N1 + S;
+    p->tw.wL = base + offL;
+    if (p->path == fftc::PATH_MULTIPASS) {
+        p->tw.wC = base + offC;
+        p->tw.wLo = base + offLo;
+        p->tw.wHi = base + offHi;
+    }
+    if (p->path == fftc::PATH_FUSED_TC) {
+        p->tc.f16 = (const uint2*)(base + offTc[0]);
+        p->tc.w256 = (const uint2*)(base + offTc[1]);
+        p->tc.fp = (const uint2*)(base + offTc[2]);
+        p->tc.fpi = (const uint2*)(base + offTc[3]);
+        p->tc.tw1 = (const uint2*)(base + offTc[4]);
+        p->tc.tw3 = (const uint2*)(base + offTc[5]);
     }
     *out = p;
     return FFTCONV_OK;
@@ -157,8 +169,8 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     cudaGetDevice(&p->device);
     const int64_t LR = 2 * (int64_t)Ws, LC = 2 * (int64_t)Hs;
     std::vector<float2> host;
-    fill_roots(host, LR, LR);
-    fill_roots(host, LC, LC);
+    size_t offR = 0, offC = 0;
+    fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
     const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
     int64_t g = (int64_t)(kGroupBytes / per_pair);
     if (g < 1) g = 1;
@@ -172,8 +184,8 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
         delete p;
         return st;
     }
-    p->tw.wL = (const float2*)p->d_tables;
-    p->tw.wC = (const float2*)p->d_tables + LR;
+    p->tw.wL = (const float2*)p->d_tables + offR;
+    p->tw.wC = (const float2*)p->d_tables + offC;
     *out = p;
     return FFTCONV_OK;
 }
@@ -193,6 +205,7 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
     if (!p) return "none";
     switch (p->path) {
         case fftc::PATH_FUSED: return "fused";
+        case fftc::PATH_FUSED_TC: return "fused_tc";
         case fftc::PATH_MULTIPASS: return "multipass";
         case fftc::PATH_2D: return "2d";
     }
@@ -206,7 +219,9 @@ fftconv_status fftconv_kernel_spectrum(fftconv_plan_t p, const float* k, int64_t
     if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (p->path == fftc::PATH_FUSED)
+    if (p->path == fftc::PATH_FUSED_TC)
+        e = fftc::launch_tc_spectrum(*p, k, L, khat, s);
+    else if (p->path == fftc::PATH_FUSED)
         e = fftc::launch_fused_spectrum(*p, k, L, (float2*)khat, s);
     else
         e = fftc::launch_multipass_spectrum(*p, k, L, (float2*)khat, (float2*)work, s);
@@ -226,7 +241,9 @@ fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (p->path == fftc::PATH_FUSED)
+    if (p->path == fftc::PATH_FUSED_TC)
+        e = fftc::launch_tc_fwd(*p, u, v, w, khat, D, y, s);
+    else if (p->path == fftc::PATH_FUSED)
         e = fftc::launch_fused_fwd(*p, u, v, w, (const float2*)khat, D, y, s);
     else
         e = fftc::launch_multipass_fwd(*p, u, v, w, (const float2*)khat, D, y, (float2*)work, s);

@@ -5,19 +5,32 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "fftconv.h"
 
 namespace fftc {
 
-enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2 };
+enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2, PATH_FUSED_TC = 3 };
 
-// Twiddle tables of one plan (device pointers into one allocation).  A table
-// "W_L" holds exp(-2 pi i m / L) for m in [0, L), rounded from fp64.
+// Twiddle tables of one plan (device pointers into one allocation).  wL / wC
+// are per-stage tables of the row / column transforms (StageTwiddles layout);
+// wLo / wHi the two-level table of W_M^e (e = e_hi 2^S + e_lo).
 struct Tables {
-    const float2* wL = nullptr;     // fused: W_M;  multipass: W_N2 (rows);  2-D: W_{2Ws}
-    const float2* wC = nullptr;     // multipass: W_N1 (columns);  2-D: W_{2Hs}
+    const float2* wL = nullptr;     // fused: length-M stages;  multipass: rows N2;  2-D: rows 2Ws
+    const float2* wC = nullptr;     // multipass: columns N1;  2-D: columns 2Hs
     const float2* wLo = nullptr;    // multipass: W_M^e for e < 2^S
     const float2* wHi = nullptr;    // multipass: W_M^(e 2^S) for e < M / 2^S
+};
+
+// Constant tables of the tensor-core path, in per-lane fragment order.
+struct TcTablePtrs {
+    const uint2* f16 = nullptr;   // [ntile 2][part 3][lane]        DFT_16 B fragments (Re, Im, -Im)
+    const uint2* w256 = nullptr;  // [reg 4][lane]                  (cos, sin) pairs of W_256^{b c}
+    const uint2* fp = nullptr;    // [kstep][ntile][part 3][lane]   outer DFT_P, p < P/2
+    const uint2* fpi = nullptr;   // [kstep][ntile][part 3][lane]   outer inverse, conj(W_P^{k_p p}), p < P/2
+    const uint2* tw1 = nullptr;   // [qt 16][ntile][half 2][lane]   (cos, sin) of W_M^{q k_p}
+    const uint2* tw3 = nullptr;   // [k_p][reg 4][lane]             (cos, sin) of W_M^{q k_p}, q = 16 a + b
 };
 
 }  // namespace fftc
@@ -40,11 +53,25 @@ struct fftconv_plan_s {
     size_t workspace_bytes = 0;
     void* d_tables = nullptr;
     fftc::Tables tw;
+    fftc::TcTablePtrs tc;
     bool spectrum_ready = false;
     int device = 0;
 };
 
 namespace fftc {
+
+// Twiddle tables: each appends its geometry's stage tables to `out` and records
+// their offsets (in float2 entries).  Returns false for an unsupported size.
+bool fused_tables(int log2M, std::vector<float2>& out, size_t* offL);
+bool multipass_tables(int log2M, std::vector<float2>& out, size_t* offC, size_t* offR);
+bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_t* offC);
+
+// 1-D bf16 tensor-core fused path (2N in {4096, 8192, 16384}).
+bool tc_supported(int log2M);
+bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]);
+cudaError_t launch_tc_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s);
+cudaError_t launch_tc_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
+                          const float* D, void* y, cudaStream_t s);
 
 // 1-D fused path (one CTA per (pair of batch rows, channel)).
 cudaError_t launch_fused_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,

@@ -13,3 +13,19 @@ def pytest_configure(config):
 TESTS = os.path.dirname(os.path.abspath(__file__))
 if TESTS not in sys.path:
     sys.path.insert(0, TESTS)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With FFTCONV_PARITY_LOG=<path>, write every parity check's errors as JSON lines."""
+    path = os.environ.get("FFTCONV_PARITY_LOG")
+    if not path:
+        return
+    try:
+        import json
+        import parity
+    except Exception:
+        return
+    with open(path, "w") as f:
+        for what, dtype, rel, mx, rms, n in parity.RECORD:
+            f.write(json.dumps({"check": what, "dtype": dtype, "rel_l2": rel, "max_abs": mx, "rms_ref": rms,
+                                "n": n}) + "\n")

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from fft_long_convolution_causal_b200 import workloads as wlmod
-from parity import assert_close, to_dev, to_host
+from parity import assert_close, row_scale_1d, row_scale_2d, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -52,18 +52,19 @@ FUSED_N = [64, 128, 256, 512, 1024, 2048, 4096, 8192]
 def test_fused_full_compare(N, dtype):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
     y, path = run_1d(wl)
-    assert path == "fused"
-    assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}")
+    want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 8192) else "fused"
+    assert path == want
+    assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}", scale=row_scale_1d(wl))
 
 
 @pytest.mark.parametrize("N", [256, 4096, 8192])
 def test_fused_gated_full_compare(N):
     wl = wlmod.make_1d(3, 3, N, dtype="bf16", gated=True, seed=7 + N, with_D=True)
     y, _ = run_1d(wl)
-    assert_close(y, oracle_full(wl), "bf16", f"fused gated N={N}")
+    assert_close(y, oracle_full(wl), "bf16", f"fused gated N={N}", gate=wl.v, scale=row_scale_1d(wl))
     wl = wlmod.make_1d(2, 2, N, dtype="f32", gated=True, seed=8 + N, with_D=False)
     y, _ = run_1d(wl)
-    assert_close(y, oracle_full(wl), "f32", f"fused gated f32 N={N}")
+    assert_close(y, oracle_full(wl), "f32", f"fused gated f32 N={N}", gate=wl.v, scale=row_scale_1d(wl))
 
 
 @pytest.mark.parametrize("N,L", [(1024, 1), (1024, 100), (4096, 4095), (32768, 777), (65536, 40000)])
@@ -73,17 +74,38 @@ def test_partial_kernel(N, L):
     y, _ = run_1d(wl)
     if N <= 32768:
         ref = oracle_full(wl)
-        assert_close(y, ref, "f32", f"partial N={N} L={L}")
+        assert_close(y, ref, "f32", f"partial N={N} L={L}", scale=row_scale_1d(wl))
     else:
         b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 256, seed=L)
         ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
-        assert_close(y[b, h, t], ref, "f32", f"partial N={N} L={L}")
+        assert_close(y[b, h, t], ref, "f32", f"partial N={N} L={L}", scale=row_scale_1d(wl, b, h))
+
+
+@pytest.mark.parametrize("N", [2048, 4096, 8192])
+@pytest.mark.parametrize("B,gated,with_D,L", [(1, False, True, None), (5, True, True, None),
+                                             (2, False, False, 333), (3, True, False, None)])
+def test_tensor_core_path(N, B, gated, with_D, L):
+    """bf16 tensor-core fused kernel: odd/even/single batch, gate, skip term, partial kernel."""
+    wl = wlmod.make_1d(B, 3, N, dtype="bf16", gated=gated, seed=N + B, with_D=with_D, L=L)
+    y, path = run_1d(wl)
+    assert path == "fused_tc"
+    assert_close(y, oracle_full(wl), "bf16", f"tc N={N} B={B} gated={gated} D={with_D} L={L}",
+                 gate=wl.v if gated else None, scale=row_scale_1d(wl))
+
+
+def test_tensor_core_large_dynamic_range():
+    """Inputs far from unit scale: the bf16 path keeps fp32's exponent range."""
+    wl = wlmod.make_1d(2, 2, 4096, dtype="bf16", seed=11)
+    wl.u = wlmod.round_bf16(wl.u * np.float32(3.0e4))
+    wl.k = (wl.k * np.float32(1.0e-3)).astype(np.float32)
+    y, _ = run_1d(wl)
+    assert_close(y, oracle_full(wl), "bf16", "tc scaled inputs", scale=row_scale_1d(wl))
 
 
 def test_no_skip_term_and_single_row():
     wl = wlmod.make_1d(1, 5, 2048, dtype="f32", seed=3, with_D=False)
     y, _ = run_1d(wl)
-    assert_close(y, oracle_full(wl), "f32", "B=1 no D")
+    assert_close(y, oracle_full(wl), "f32", "B=1 no D", scale=row_scale_1d(wl))
 
 
 @pytest.mark.parametrize("N", [16384, 32768])
@@ -92,7 +114,8 @@ def test_multipass_full_compare(N, dtype, gated):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=gated, seed=N + gated, with_D=True)
     y, path = run_1d(wl)
     assert path == "multipass"
-    assert_close(y, oracle_full(wl), dtype, f"multipass N={N} {dtype} gated={gated}")
+    assert_close(y, oracle_full(wl), dtype, f"multipass N={N} {dtype} gated={gated}",
+                 gate=wl.v if gated else None, scale=row_scale_1d(wl))
 
 
 @pytest.mark.parametrize("log2N", [16, 17, 18, 19, 20])
@@ -103,7 +126,7 @@ def test_multipass_sampled(log2N):
     assert path == "multipass"
     b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 400, seed=log2N)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
-    assert_close(y[b, h, t], ref, "f32", f"multipass N=2^{log2N}")
+    assert_close(y[b, h, t], ref, "f32", f"multipass N=2^{log2N}", scale=row_scale_1d(wl, b, h))
 
 
 def test_multipass_ragged_groups():
@@ -113,7 +136,7 @@ def test_multipass_ragged_groups():
     y, _ = run_1d(wl)
     b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 64, seed=99)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
-    assert_close(y[b, h, t], ref, "bf16", "ragged groups")
+    assert_close(y[b, h, t], ref, "bf16", "ragged groups", scale=row_scale_1d(wl, b, h))
 
 
 @pytest.mark.parametrize("N", [4096, 1 << 20])
@@ -149,7 +172,7 @@ def test_pr1_full():
     wl = _named("pr1_b1_h4_n1024_f32")
     y, path = run_1d(wl)
     assert path == "fused"
-    assert_close(y, oracle_full(wl), "f32", wl.name)
+    assert_close(y, oracle_full(wl), "f32", wl.name, scale=row_scale_1d(wl))
 
 
 @pytest.mark.parametrize("name,per_row", [("hyena_b8_h768_n4096_bf16", 12),
@@ -160,7 +183,8 @@ def test_named_1d_sampled(name, per_row):
     y, _ = run_1d(wl)
     b, h, t = wlmod.sample_points_1d(wl.B, wl.H, wl.N, per_row, seed=1)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D, w=wl.w, v=wl.v)
-    assert_close(y[b, h, t], ref, wl.dtype, wl.name)
+    assert_close(y[b, h, t], ref, wl.dtype, wl.name, gate=None if wl.v is None else wl.v[b, h, t],
+                 scale=row_scale_1d(wl, b, h))
 
 
 # ------------------------------------------------------------------ 2-D
@@ -178,13 +202,13 @@ def run_2d(wl):
 def test_conv2d_full_compare(Hs, Ws, dtype):
     wl = wlmod.make_2d(3, 2, Hs, Ws, dtype=dtype, seed=Hs + Ws, sigma=Hs / 4)
     y = run_2d(wl)
-    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), dtype, f"2d {Hs}x{Ws} {dtype}")
+    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), dtype, f"2d {Hs}x{Ws} {dtype}", scale=row_scale_2d(wl))
 
 
 def test_conv2d_small_kernel():
     wl = wlmod.make_2d(2, 3, 64, 64, dtype="f32", seed=2, Kh=5, Kw=17)
     y = run_2d(wl)
-    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel")
+    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel", scale=row_scale_2d(wl))
 
 
 def test_conv2d_named_sampled():
@@ -192,7 +216,7 @@ def test_conv2d_named_sampled():
     y = run_2d(wl)
     idx = wlmod.sample_points_2d(wl.B, wl.C, wl.Hs, wl.Ws, 4096, seed=4)
     ref = oracle.causal_conv2d_points(wl.u, wl.k, *idx)
-    assert_close(y[idx], ref, "bf16", wl.name)
+    assert_close(y[idx], ref, "bf16", wl.name, scale=row_scale_2d(wl, idx[0], idx[1]))
 
 
 # ------------------------------------------------------------------ API on GPU
