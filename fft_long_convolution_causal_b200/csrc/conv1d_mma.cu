@@ -128,48 +128,61 @@ struct TcShape {
 };
 
 // ================================================================== kernel
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+template <int P, bool GATED>
+struct TcSmem {
+    static constexpr int kS = 2 * P * 512;      // S: re and im planes, P rows of 256 q
+    static constexpr int kX = P * 512;          // x staging: re and im planes, P/2 rows
+    static constexpr int kBytes = kS + kX * (GATED ? 2 : 1);
+};
+
+// Persistent: each CTA walks work items (pair pp of channel h) with stride
+// gridDim.x; items of one channel are consecutive so concurrent CTAs share
+// Khat[h] in L2.  The next item's input is fetched with cp.async into the
+// staging planes while the current item runs its inner transforms.
 template <int P, int NW, bool GATED>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, P <= 32 ? 4 : 2)
 fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
              const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
              __nv_bfloat16* __restrict__ y, TcTables tb, int B, int H) {
     using S = TcShape<P>;
+    using SM = TcSmem<P, GATED>;
     static_assert(P >= 16 && P <= 64, "outer factor");
+    constexpr int NT = NW * 32;
+    constexpr int CH = S::N / 8;                          // 16-byte chunks per row of u
+    constexpr bool PRE1 = S::NT1 * S::KS1 <= 4;           // keep step-1 B fragments in registers
+    constexpr bool PRE3 = S::NT3 * S::KS3 <= 4;           // keep step-1' B fragments in registers
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = blockIdx.y;
-    const int b0 = 2 * blockIdx.x;
-    const bool has1 = b0 + 1 < B;
-    const size_t row0 = ((size_t)b0 * H + h) * S::N;
-    const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const int npp = (B + 1) / 2;
+    const int items = npp * H;
     const uint32_t sre = smem_u32(smem), sim = sre + S::kPlaneBytes;
+    const uint32_t xre = sre + SM::kS, xim = xre + SM::kX / 2;
+    const uint32_t wre = xre + SM::kX, wim = wre + SM::kX / 2;
 
-    // ---- stage x = u (or u*w) into the planes: rows p < P/2, natural q
-    {
-        constexpr int CH = S::N / 8;  // 16-byte chunks per row of u
-        for (int i = tid; i < 2 * CH; i += NW * 32) {
-            const int plane = i / CH, ci = i % CH;  // plane 0: row b (re), 1: row b+1 (im)
-            const int n0 = ci * 8;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (plane == 0 || has1) {
-                const size_t off = (plane ? row1 : row0) + n0;
-                val = __ldg(reinterpret_cast<const uint4*>(u + off));
-                if (GATED) {
-                    const uint4 ww = __ldg(reinterpret_cast<const uint4*>(w + off));
-                    val.x = as_u(__hmul2(as_b2(val.x), as_b2(ww.x)));
-                    val.y = as_u(__hmul2(as_b2(val.y), as_b2(ww.y)));
-                    val.z = as_u(__hmul2(as_b2(val.z), as_b2(ww.z)));
-                    val.w = as_u(__hmul2(as_b2(val.w), as_b2(ww.w)));
-                }
-            }
+    auto stage_input = [&](int item) {
+        const int hh = item / npp, b0 = 2 * (item % npp);
+        const bool has1 = b0 + 1 < B;
+        const size_t r0 = ((size_t)b0 * H + hh) * S::N;
+        const size_t r1 = has1 ? ((size_t)(b0 + 1) * H + hh) * S::N : r0;
+        for (int i = tid; i < 2 * CH; i += NT) {
+            const int plane = i / CH, n0 = (i % CH) * 8;
             const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
-            const uint32_t addr = plane_addr(plane ? sim : sre, p, chunk);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(val.x), "r"(val.y), "r"(val.z),
-                         "r"(val.w)
-                         : "memory");
+            const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing row
+            const size_t off = (plane ? r1 : r0) + n0;
+            cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
+            if (GATED) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
         }
-    }
-    // inner DFT_16 fragments and W_256 twiddles (same for every row)
+        cp_async_commit();
+    };
+
+    // constants for the whole kernel: inner DFT_16 fragments, W_256 twiddles
     uint2 f16[3][2], w256[4];
 #pragma unroll
     for (int part = 0; part < 3; ++part)
@@ -177,160 +190,228 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
-    __syncthreads();
-
-    const int m8 = lane >> 3, r8 = lane & 7;
-
-    // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
-    for (int qt = warp; qt < 16; qt += NW) {
-        uint32_t ar[S::KS1][4], ai[S::KS1][4];
+    uint2 fp[PRE1 ? S::KS1 : 1][PRE1 ? S::NT1 : 1][3];
+    if (PRE1) {
 #pragma unroll
-        for (int ks = 0; ks < S::KS1; ++ks) {
-            // A[q][p]: matrices (q 0-7|8-15) x (p 0-7|8-15) from rows p, chunks 2 qt (+1)
-            // rows p >= P/2 are the zero padding: those lanes point at row 0 (a
-            // select, not a branch: ldmatrix must run warp-converged) and the
-            // registers they feed are zeroed below
-            const uint32_t prow0 = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
-            const uint32_t prow = prow0 < (uint32_t)(P / 2) ? prow0 : 0u;
-            ldsm_x4_t(ar[ks], plane_addr(sre, prow, chunk));
-            ldsm_x4_t(ai[ks], plane_addr(sim, prow, chunk));
-            if (16 * ks + 8 >= P / 2) {  // p 8-15 of this k-step are padding
-                ar[ks][2] = ar[ks][3] = ai[ks][2] = ai[ks][3] = 0u;
-            }
+        for (int ks = 0; ks < S::KS1; ++ks)
+#pragma unroll
+            for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+                    fp[PRE1 ? ks : 0][PRE1 ? j : 0][part] =
+                        __ldg(&tb.fp[((ks * S::NT1 + j) * 3 + part) * 32 + lane]);
+    }
+    uint2 fpi[PRE3 ? S::KS3 : 1][PRE3 ? S::NT3 : 1][3];
+    if (PRE3) {
+#pragma unroll
+        for (int ks = 0; ks < S::KS3; ++ks)
+#pragma unroll
+            for (int j = 0; j < S::NT3; ++j)
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+                    fpi[PRE3 ? ks : 0][PRE3 ? j : 0][part] =
+                        __ldg(&tb.fpi[((ks * S::NT3 + j) * 3 + part) * 32 + lane]);
+    }
+
+    if ((int)blockIdx.x < items) stage_input(blockIdx.x);
+
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int h = item / npp, b0 = 2 * (item % npp);
+        const bool has1 = b0 + 1 < B;
+        const size_t row0 = ((size_t)b0 * H + h) * S::N;
+        const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
+        cp_async_wait_all();
+        __syncthreads();
+
+        // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
+        uint2 twn[S::NT1][2];
+        if (warp < 16) {
+#pragma unroll
+            for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) twn[j][hh] = __ldg(&tb.tw1[((warp * S::NT1 + j) * 2 + hh) * 32 + lane]);
         }
+        for (int qt = warp; qt < 16; qt += NW) {
+            uint2 twc[S::NT1][2];
 #pragma unroll
-        for (int j = 0; j < S::NT1; ++j) {
-            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < S::NT1; ++j) {
+                twc[j][0] = twn[j][0];
+                twc[j][1] = twn[j][1];
+            }
+            if (qt + NW < 16) {
+#pragma unroll
+                for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        twn[j][hh] = __ldg(&tb.tw1[(((qt + NW) * S::NT1 + j) * 2 + hh) * 32 + lane]);
+            }
+            uint32_t ar[S::KS1][4], ai[S::KS1][4];
 #pragma unroll
             for (int ks = 0; ks < S::KS1; ++ks) {
-                const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
-                cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
-            }
-            // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
-            uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
-            uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
+                // A[q][p] from rows p, chunks 2 qt (+1).  Rows p >= P/2 are the
+                // zero padding: those lanes point at row 0 (a select -- ldmatrix
+                // must run warp-converged) and their registers are zeroed.
+                const uint32_t prow0 = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+                const uint32_t prow = prow0 < (uint32_t)(P / 2) ? prow0 : 0u;
+                ldsm_x4_t(ar[ks], plane_addr(xre, prow, chunk));
+                ldsm_x4_t(ai[ks], plane_addr(xim, prow, chunk));
+                if (GATED) {
+                    uint32_t gr[4], gi[4];
+                    ldsm_x4_t(gr, plane_addr(wre, prow, chunk));
+                    ldsm_x4_t(gi, plane_addr(wim, prow, chunk));
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                twiddle2<true>(pr[hh], pi[hh], __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + hh) * 32 + lane]));
-            // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
-            const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
-            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
+                    for (int r = 0; r < 4; ++r) {
+                        ar[ks][r] = as_u(__hmul2(as_b2(ar[ks][r]), as_b2(gr[r])));
+                        ai[ks][r] = as_u(__hmul2(as_b2(ai[ks][r]), as_b2(gi[r])));
+                    }
+                }
+                if (16 * ks + 8 >= P / 2) ar[ks][2] = ar[ks][3] = ai[ks][2] = ai[ks][3] = 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < S::NT1; ++j) {
+                float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < S::KS1; ++ks) {
+                    if (PRE1) {
+                        cmma(yr, yi, ar[ks], ai[ks], fp[PRE1 ? ks : 0][PRE1 ? j : 0][0],
+                             fp[PRE1 ? ks : 0][PRE1 ? j : 0][1], fp[PRE1 ? ks : 0][PRE1 ? j : 0][2]);
+                    } else {
+                        const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
+                        cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                    }
+                }
+                // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
+                uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
+                uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
+                twiddle2<true>(pr[0], pi[0], twc[j][0]);
+                twiddle2<true>(pr[1], pi[1], twc[j][1]);
+                // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
+                const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+                stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
+            }
         }
-    }
-    __syncthreads();
+        __syncthreads();
+        // the staging planes are free: fetch the next item while this one runs
+        if (item + (int)gridDim.x < items) stage_input(item + gridDim.x);
 
-    // ---- step 3: inner 256-point DFT, product with Khat, inverse, per row k_p
-    const float dm = D ? D[h] * (1.0f / S::M) : 0.f;
-    const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
-    for (int kp = warp; kp < P; kp += NW) {
-        uint32_t xr[4], xi[4];
-        {
+        // ---- step 3: inner 256-point DFT, product with Khat, inverse, per row k_p
+        const float dmf = D ? D[h] * (1.0f / S::M) : 0.f;
+        const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
+        const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
+        uint4 kn0 = __ldg(&kh[(size_t)warp * 64 + lane * 2]), kn1 = __ldg(&kh[(size_t)warp * 64 + lane * 2 + 1]);
+        uint2 tn[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tn[i] = __ldg(&tb.tw3[((size_t)warp * 4 + i) * 32 + lane]);
+        for (int kp = warp; kp < P; kp += NW) {
+            const uint4 kc0 = kn0, kc1 = kn1;
+            uint2 tc3[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tc3[i] = tn[i];
+            if (kp + NW < P) {
+                kn0 = __ldg(&kh[(size_t)(kp + NW) * 64 + lane * 2]);
+                kn1 = __ldg(&kh[(size_t)(kp + NW) * 64 + lane * 2 + 1]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tn[i] = __ldg(&tb.tw3[((size_t)(kp + NW) * 4 + i) * 32 + lane]);
+            }
+            uint32_t xr[4], xi[4];
             const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
             ldsm_x4_t(xr, plane_addr(sre, kp, chunk));
             ldsm_x4_t(xi, plane_addr(sim, kp, chunk));
-        }
-        // stage i: [b][a] x F16 -> [b][c]
-        float ur[2][4] = {}, ui[2][4] = {};
+            // stage i: [b][a] x F16 -> [b][c]
+            float ur[2][4] = {}, ui[2][4] = {};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) cmma(ur[j], ui[j], xr, xi, f16[0][j], f16[1][j], f16[2][j]);
-        uint32_t tr[4] = {pack2(ur[0][0], ur[0][1]), pack2(ur[0][2], ur[0][3]), pack2(ur[1][0], ur[1][1]),
-                          pack2(ur[1][2], ur[1][3])};
-        uint32_t ti[4] = {pack2(ui[0][0], ui[0][1]), pack2(ui[0][2], ui[0][3]), pack2(ui[1][0], ui[1][1]),
-                          pack2(ui[1][2], ui[1][3])};
+            for (int j = 0; j < 2; ++j) cmma(ur[j], ui[j], xr, xi, f16[0][j], f16[1][j], f16[2][j]);
+            uint32_t tr[4] = {pack2(ur[0][0], ur[0][1]), pack2(ur[0][2], ur[0][3]), pack2(ur[1][0], ur[1][1]),
+                              pack2(ur[1][2], ur[1][3])};
+            uint32_t ti[4] = {pack2(ui[0][0], ui[0][1]), pack2(ui[0][2], ui[0][3]), pack2(ui[1][0], ui[1][1]),
+                              pack2(ui[1][2], ui[1][3])};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
-        // transpose [b][c] -> [c][b]
-        uint32_t cr[4] = {movt(tr[0]), movt(tr[2]), movt(tr[1]), movt(tr[3])};
-        uint32_t ci[4] = {movt(ti[0]), movt(ti[2]), movt(ti[1]), movt(ti[3])};
-        // stage ii: [c][b] x F16 -> [c][d]  (spectrum at k = k_p + P (c + 16 d))
-        float vr[2][4] = {}, vi[2][4] = {};
+            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+            // transpose [b][c] -> [c][b]
+            uint32_t cr[4] = {movt(tr[0]), movt(tr[2]), movt(tr[1]), movt(tr[3])};
+            uint32_t ci[4] = {movt(ti[0]), movt(ti[2]), movt(ti[1]), movt(ti[3])};
+            // stage ii: [c][b] x F16 -> [c][d]  (spectrum at k = k_p + P (c + 16 d))
+            float vr[2][4] = {}, vi[2][4] = {};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) cmma(vr[j], vi[j], cr, ci, f16[0][j], f16[1][j], f16[2][j]);
-        // pointwise product with Khat (+ D/M), in fp32
-        const uint4 k0 = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
-        const uint4 k1 = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
-        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            for (int j = 0; j < 2; ++j) cmma(vr[j], vi[j], cr, ci, f16[0][j], f16[1][j], f16[2][j]);
+            uint32_t zr4[4] = {pack2(vr[0][0], vr[0][1]), pack2(vr[0][2], vr[0][3]), pack2(vr[1][0], vr[1][1]),
+                               pack2(vr[1][2], vr[1][3])};
+            uint32_t zi4[4] = {pack2(vi[0][0], vi[0][1]), pack2(vi[0][2], vi[0][3]), pack2(vi[1][0], vi[1][1]),
+                               pack2(vi[1][2], vi[1][3])};
+            // pointwise product with (Khat + D/M), packed: Khat regs i hold (re pair, im pair)
+            {
+                const uint32_t kre[4] = {kc0.x, kc0.z, kc1.x, kc1.z}, kim[4] = {kc0.y, kc0.w, kc1.y, kc1.w};
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t kk = kw[j * 4 + e];
-                const float kr = __uint_as_float(kk << 16) + dm, ki = __uint_as_float(kk & 0xffff0000u);
-                const float zr = vr[j][e], zi = vi[j][e];
-                vr[j][e] = fmaf(zr, kr, -zi * ki);
-                vi[j][e] = fmaf(zr, ki, zi * kr);
+                for (int i = 0; i < 4; ++i) {
+                    const __nv_bfloat162 zr = as_b2(zr4[i]), zi = as_b2(zi4[i]);
+                    const __nv_bfloat162 kr = __hadd2(as_b2(kre[i]), dm2), ki = as_b2(kim[i]);
+                    zr4[i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
+                    zi4[i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
+                }
             }
-        // inverse stage ii: [c][d] x conj(F16) -> [c][b]
-        uint32_t zr4[4] = {pack2(vr[0][0], vr[0][1]), pack2(vr[0][2], vr[0][3]), pack2(vr[1][0], vr[1][1]),
-                           pack2(vr[1][2], vr[1][3])};
-        uint32_t zi4[4] = {pack2(vi[0][0], vi[0][1]), pack2(vi[0][2], vi[0][3]), pack2(vi[1][0], vi[1][1]),
-                           pack2(vi[1][2], vi[1][3])};
-        float sr[2][4] = {}, si[2][4] = {};
-        // conj(F16) = Fr - i Fi: parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
+            // inverse stage ii: [c][d] x conj(F16) -> [c][b]; conj parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
+            float sr[2][4] = {}, si[2][4] = {};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) cmma(sr[j], si[j], zr4, zi4, f16[0][j], f16[2][j], f16[1][j]);
-        uint32_t gr[4] = {pack2(sr[0][0], sr[0][1]), pack2(sr[0][2], sr[0][3]), pack2(sr[1][0], sr[1][1]),
-                          pack2(sr[1][2], sr[1][3])};
-        uint32_t gi[4] = {pack2(si[0][0], si[0][1]), pack2(si[0][2], si[0][3]), pack2(si[1][0], si[1][1]),
-                          pack2(si[1][2], si[1][3])};
-        // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
-        uint32_t hr[4] = {movt(gr[0]), movt(gr[2]), movt(gr[1]), movt(gr[3])};
-        uint32_t hi[4] = {movt(gi[0]), movt(gi[2]), movt(gi[1]), movt(gi[3])};
+            for (int j = 0; j < 2; ++j) cmma(sr[j], si[j], zr4, zi4, f16[0][j], f16[2][j], f16[1][j]);
+            uint32_t gr[4] = {pack2(sr[0][0], sr[0][1]), pack2(sr[0][2], sr[0][3]), pack2(sr[1][0], sr[1][1]),
+                              pack2(sr[1][2], sr[1][3])};
+            uint32_t gi[4] = {pack2(si[0][0], si[0][1]), pack2(si[0][2], si[0][3]), pack2(si[1][0], si[1][1]),
+                              pack2(si[1][2], si[1][3])};
+            // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
+            uint32_t hr[4] = {movt(gr[0]), movt(gr[2]), movt(gr[1]), movt(gr[3])};
+            uint32_t hi[4] = {movt(gi[0]), movt(gi[2]), movt(gi[1]), movt(gi[3])};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) twiddle2<false>(hr[i], hi[i], w256[i]);
-        // inverse stage i: [b][c] x conj(F16) -> [b][a]
-        float or_[2][4] = {}, oi[2][4] = {};
+            for (int i = 0; i < 4; ++i) twiddle2<false>(hr[i], hi[i], w256[i]);
+            // inverse stage i: [b][c] x conj(F16) -> [b][a]
+            float or_[2][4] = {}, oi[2][4] = {};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) cmma(or_[j], oi[j], hr, hi, f16[0][j], f16[2][j], f16[1][j]);
-        uint32_t qr[4] = {pack2(or_[0][0], or_[0][1]), pack2(or_[0][2], or_[0][3]), pack2(or_[1][0], or_[1][1]),
-                          pack2(or_[1][2], or_[1][3])};
-        uint32_t qi[4] = {pack2(oi[0][0], oi[0][1]), pack2(oi[0][2], oi[0][3]), pack2(oi[1][0], oi[1][1]),
-                          pack2(oi[1][2], oi[1][3])};
-        // conj twiddle W_M^{-q k_p}, q = 16 a + b
+            for (int j = 0; j < 2; ++j) cmma(or_[j], oi[j], hr, hi, f16[0][j], f16[2][j], f16[1][j]);
+            uint32_t qr[4] = {pack2(or_[0][0], or_[0][1]), pack2(or_[0][2], or_[0][3]), pack2(or_[1][0], or_[1][1]),
+                              pack2(or_[1][2], or_[1][3])};
+            uint32_t qi[4] = {pack2(oi[0][0], oi[0][1]), pack2(oi[0][2], oi[0][3]), pack2(oi[1][0], oi[1][1]),
+                              pack2(oi[1][2], oi[1][3])};
+            // conj twiddle W_M^{-q k_p}, q = 16 a + b
 #pragma unroll
-        for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]));
-        // back to row k_p (fragment [b][a] stored transposed: rows a, natural q)
-        {
-            const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
-            // registers: 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3 (b 8-15, a 8-15)
+            for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], tc3[i]);
+            // back to row k_p: registers 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3
             stsm_x4_t(plane_addr(sre, kp, chunk), qr[0], qr[1], qr[2], qr[3]);
             stsm_x4_t(plane_addr(sim, kp, chunk), qi[0], qi[1], qi[2], qi[3]);
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // ---- step 1': inverse outer DFT over k_p, outputs p < P/2, into rows p
-    for (int qt = warp; qt < 16; qt += NW) {
-        uint32_t ar[S::KS3][4], ai[S::KS3][4];
-#pragma unroll
-        for (int ks = 0; ks < S::KS3; ++ks) {
-            const uint32_t krow = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
-            ldsm_x4_t(ar[ks], plane_addr(sre, krow, chunk));
-            ldsm_x4_t(ai[ks], plane_addr(sim, krow, chunk));
-        }
-#pragma unroll
-        for (int j = 0; j < S::NT3; ++j) {
-            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- step 1': inverse outer DFT over k_p, outputs p < P/2, into rows p
+        for (int qt = warp; qt < 16; qt += NW) {
+            uint32_t ar[S::KS3][4], ai[S::KS3][4];
 #pragma unroll
             for (int ks = 0; ks < S::KS3; ++ks) {
-                const uint2* fb = tb.fpi + ((size_t)(ks * S::NT3 + j) * 3) * 32 + lane;
-                cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                const uint32_t krow = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+                ldsm_x4_t(ar[ks], plane_addr(sre, krow, chunk));
+                ldsm_x4_t(ai[ks], plane_addr(sim, krow, chunk));
             }
-            // rows q = 16 qt + g (+8), cols p = 8 j + 2t (+1) -> rows p, chunk 2 qt (+1)
-            const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
-            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk), pack2(yr[0], yr[1]), pack2(yr[2], yr[3]),
-                      pack2(yi[0], yi[1]), pack2(yi[2], yi[3]));
+#pragma unroll
+            for (int j = 0; j < S::NT3; ++j) {
+                float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < S::KS3; ++ks) {
+                    if (PRE3) {
+                        cmma(yr, yi, ar[ks], ai[ks], fpi[PRE3 ? ks : 0][PRE3 ? j : 0][0],
+                             fpi[PRE3 ? ks : 0][PRE3 ? j : 0][1], fpi[PRE3 ? ks : 0][PRE3 ? j : 0][2]);
+                    } else {
+                        const uint2* fb = tb.fpi + ((size_t)(ks * S::NT3 + j) * 3) * 32 + lane;
+                        cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                    }
+                }
+                const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+                stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk), pack2(yr[0], yr[1]), pack2(yr[2], yr[3]),
+                          pack2(yi[0], yi[1]), pack2(yi[2], yi[3]));
+            }
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
-    {
-        constexpr int CH = S::N / 8;
-        for (int i = tid; i < 2 * CH; i += NW * 32) {
-            const int plane = i / CH, ci = i % CH;
+        // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
+        for (int i = tid; i < 2 * CH; i += NT) {
+            const int plane = i / CH, n0 = (i % CH) * 8;
             if (plane == 1 && !has1) continue;
-            const int n0 = ci * 8;
             const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
             uint4 val;
             asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
@@ -346,13 +427,16 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
             }
             *reinterpret_cast<uint4*>(y + off) = val;
         }
+        // the next iteration's wait + barrier orders these reads before S is rewritten
     }
+    cp_async_wait_all();
 }
 
 // Spectrum in the kernel's fragment order: the SIMT transform of k[h]
-// (natural order, fp32, in shared memory), then per row k_p and lane the 8
-// values (j, e) at k = k_p + P (c + 16 d), c = g + 8 (e >> 1),
-// d = 8 j + 2 t + (e & 1), scaled by 1/M and rounded to bf16 (re, im).
+// (natural order, fp32, in shared memory), then per row k_p and lane 8 words:
+// for A-fragment register i of the [c][d] tile (c = g + 8 (i & 1),
+// d = 2t + 8 (i >> 1) + {0, 1}), the packed bf16 pair of real parts and the
+// packed pair of imaginary parts of Khat[k_p + P (c + 16 d)] = X / M.
 template <int LOG2M>
 __global__ void __launch_bounds__(Geometry<LOG2M, 1, false>::T)
 tc_spectrum(const float* __restrict__ k, int L, uint32_t* __restrict__ khat, const float2* __restrict__ tw) {
@@ -370,12 +454,14 @@ tc_spectrum(const float* __restrict__ k, int L, uint32_t* __restrict__ khat, con
     smem_stages<G, 1, NS, false>(smem2, tid, tw);
     uint32_t* out = khat + (size_t)h * M;
     for (int o = tid; o < M; o += G::T) {
-        const int kp = o / 256, rem = o % 256, lane = rem / 8, je = rem % 8;
-        const int j = je / 4, e = je % 4, g = lane >> 2, t = lane & 3;
-        const int c = g + 8 * (e >> 1), d = 8 * j + 2 * t + (e & 1);
-        const float2 z = cscale(smem2[Lay::at(kp + P * (c + 16 * d), 0)], 1.0f / M);
-        out[o] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.x)) |
-                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.y)) << 16);
+        const int kp = o / 256, rem = o % 256, lane = rem / 8, wd = rem % 8;
+        const int i = wd >> 1, part = wd & 1, g = lane >> 2, t = lane & 3;
+        const int c = g + 8 * (i & 1), d0 = 2 * t + 8 * (i >> 1);
+        const float2 z0 = cscale(smem2[Lay::at(kp + P * (c + 16 * d0), 0)], 1.0f / M);
+        const float2 z1 = cscale(smem2[Lay::at(kp + P * (c + 16 * (d0 + 1)), 0)], 1.0f / M);
+        const float lo = part ? z0.y : z0.x, hi = part ? z1.y : z1.x;
+        out[o] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
     }
 }
 
@@ -512,9 +598,19 @@ static cudaError_t tc_fwd_go(const fftconv_plan_s& p, const void* u, const void*
                              const void* khat, const float* D, void* y, cudaStream_t s) {
     constexpr int NW = 4;
     auto kern = tc::fused_fwd_tc<P, NW, GATED>;
-    const size_t smem = tc::TcShape<P>::kSmemPerPair;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dim3 grid((p.B + 1) / 2, p.H);
+    const size_t smem = tc::TcSmem<P, GATED>::kBytes;
+    // persistent grid: as many CTAs as are resident at once (computed once)
+    static int resident = 0;
+    if (resident == 0) {
+        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        int per_sm = 0, sms = 0, dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NW * 32, smem);
+        resident = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    }
+    const int items = ((p.B + 1) / 2) * p.H;
+    dim3 grid(items < resident ? items : resident);
     kern<<<grid, NW * 32, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
                                      (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.B, p.H);
     return cudaGetLastError();
