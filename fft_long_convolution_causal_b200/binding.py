@@ -38,6 +38,8 @@ _SIGS = {
     "fftconv_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv2d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
     "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv_fwd_static_workspace": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv_static_workspace_bytes": (ctypes.c_size_t, []),
     "fftconv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fftconv_version": (ctypes.c_int, []),
 }

@@ -148,6 +148,35 @@ FFTCONV_API fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t plan, const 
 FFTCONV_API fftconv_status fftconv2d_fwd(fftconv_plan_t plan, const void* u, const void* khat, void* y,
                              void* workspace, void* stream);
 
+/*
+ * Forward without a workspace argument: the same result as fftconv_fwd on a
+ * multi-pass plan (2N > 16384), with the scratch taken from a device array
+ * of FFTCONV_STATIC_WORKSPACE_BYTES built into the library instead of a
+ * caller buffer.  No counterpart on the pages: it exists for callers that
+ * cannot allocate device memory at the time they convolve (allocation is
+ * forbidden there, or would synchronise the device, or all memory belongs to
+ * someone else's pool).  It allocates nothing.
+ *   - Arguments and layouts as fftconv_fwd, minus the workspace.
+ *   - FFTCONV_ERR_UNSUPPORTED for a plan that is not multi-pass, or whose
+ *     scratch for one pair of rows (8 bytes per point of the length-2N
+ *     transform) is larger than the array; every N this library supports
+ *     (up to 2^20, 16 MiB per pair) fits.
+ *   - The array's device address is looked up on the first call on each
+ *     device, with that device current; make that first call before any
+ *     stream capture.
+ *   - Every call uses the same array: calls whose GPU work overlaps (other
+ *     streams, other threads) race on it and give wrong results; serialise
+ *     them.  Nothing in the array needs to be cleared between calls.
+ *   - The array occupies every GPU that loads the library until exit.
+ */
+#define FFTCONV_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+FFTCONV_API fftconv_status fftconv_fwd_static_workspace(fftconv_plan_t plan, const void* u, const void* v,
+                                                        const void* w, const void* khat, const float* D,
+                                                        void* y, void* stream);
+
+/* Size in bytes of the device array fftconv_fwd_static_workspace uses. */
+FFTCONV_API size_t fftconv_static_workspace_bytes(void);
+
 /* Human-readable name of a status code (static string). */
 FFTCONV_API const char* fftconv_status_string(fftconv_status status);
 
