@@ -55,14 +55,14 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--channels", type=int, default=0,
+                    help="override H (1-D) or C (2-D) for a smaller case, e.g. an ncu capture; 0 = as named")
     return ap.parse_args()
 
 
 def dist_env():
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return rank, world, local
+    from fft_long_convolution_causal_b200.dist import rank_env
+    return rank_env()
 
 
 def measured_peaks():
@@ -153,9 +153,17 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- workload
-def build_workload(name):
+def build_workload(name, channels=0):
     from fft_long_convolution_causal_b200 import workloads
-    return workloads.make_config(name)
+    if not channels:
+        return workloads.make_config(name)
+    c = dict(workloads.CONFIGS[name])
+    kind = c.pop("kind")
+    if kind == "1d":
+        c["H"] = channels
+        return workloads.make_1d(name=f"{name}_h{channels}", **c)
+    c["C"] = channels
+    return workloads.make_2d(name=f"{name}_c{channels}", **c)
 
 
 class Runner:
@@ -330,7 +338,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
         pg = dist
-    wl = build_workload(args.config)
+    wl = build_workload(args.config, args.channels)
     r = Runner(wl, torch)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     for _ in range(max(args.warmup, 3)):
@@ -354,22 +362,16 @@ def main():
     if pg:
         pg.barrier()
     clocks = sampler.stop() if sampler else None
-    total_ms = float(np.sum(per_step))
-    if pg:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    from fft_long_convolution_causal_b200.dist import job_throughput, max_over_ranks
+    total_ms = max_over_ranks(float(np.sum(per_step)), pg, device="cuda")
     ms_per_step = total_ms / args.steps
-    value = r.outputs * world / (ms_per_step * 1e-3)
+    value = job_throughput(r.outputs, world, ms_per_step * 1e-3)
 
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(r, max(3, min(args.steps, 20)), torch)
-        if pg:
-            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": r.outputs * world / (e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(e2e_ms, pg, device="cuda")
+        e2e = {"value": job_throughput(r.outputs, world, e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peak, peak_kind = measured_peaks()
@@ -394,7 +396,7 @@ def main():
         pg.destroy_process_group()
     if rank != 0:
         return 0
-    cfg = {"workload": args.config, "dtype_io": wl.dtype, "path": r.plan.path,
+    cfg = {"workload": wl.name, "dtype_io": wl.dtype, "path": r.plan.path,
            "l2": "flushed between timed steps (256 MiB write outside the events)",
            "parallelism": f"replicas x{world} (independent rows, no collective)"}
     if r.is2d:
@@ -415,7 +417,7 @@ def main_reference(args, rank, world):
     """The oracle as the reference arm: rank 0 times it on the host cores."""
     if rank != 0:
         return 0
-    wl = build_workload(args.config)
+    wl = build_workload(args.config, args.channels)
     s = OracleSampler(wl, seed=0)
     per_step = max(args.cpu_seconds / max(args.steps, 1), 0.25)
     n = s.calibrate(per_step)

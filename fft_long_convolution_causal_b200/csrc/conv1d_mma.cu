@@ -42,8 +42,10 @@ namespace fftc {
 namespace tc {
 
 // ------------------------------------------------------------ PTX wrappers
+// Register-only operations (mma, movmatrix) are not volatile, so the compiler
+// may interleave independent ones; shared-memory ones keep their order.
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -61,7 +63,7 @@ __device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r
 }
 __device__ __forceinline__ uint32_t movt(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
     return y;
 }
 // two fp32 -> packed bf16x2 (lo in the low half), round to nearest even
@@ -87,6 +89,24 @@ __device__ __forceinline__ void twiddle2(uint32_t& re, uint32_t& im, uint2 cs) {
     } else {
         re = as_u(__hfma2(r, c, __hneg2(__hmul2(i, s))));
         im = as_u(__hfma2(i, c, __hmul2(r, s)));
+    }
+}
+
+// Complex product of one 16x16 A tile with the two n-tiles of a 16x16 B:
+// the four products with Ar first, then the four with Ai, so each dependent
+// accumulation is four MMAs behind the one it waits for.
+__device__ __forceinline__ void cmma2(float (&yr)[2][4], float (&yi)[2][4], const uint32_t (&ar)[4],
+                                      const uint32_t (&ai)[4], const uint2 (&br)[2], const uint2 (&bi)[2],
+                                      const uint2 (&bni)[2]) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        mma16816(yr[j], ar, br[j].x, br[j].y);
+        mma16816(yi[j], ar, bi[j].x, bi[j].y);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        mma16816(yr[j], ai, bni[j].x, bni[j].y);
+        mma16816(yi[j], ai, br[j].x, br[j].y);
     }
 }
 
@@ -141,12 +161,130 @@ struct TcSmem {
     static constexpr int kBytes = kS + kX * (GATED ? 2 : 1);
 };
 
+// fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
+// registers of the 16x16 A fragment they form.
+__device__ __forceinline__ void pack_tile(uint32_t (&o)[4], const float (&t)[2][4]) {
+    o[0] = pack2(t[0][0], t[0][1]);
+    o[1] = pack2(t[0][2], t[0][3]);
+    o[2] = pack2(t[1][0], t[1][1]);
+    o[3] = pack2(t[1][2], t[1][3]);
+}
+// 16x16 transpose of an A fragment: block (r, c) -> (c, r), each 8x8 block transposed.
+__device__ __forceinline__ void transpose_tile(uint32_t (&o)[4], const uint32_t (&x)[4]) {
+    o[0] = movt(x[0]);
+    o[1] = movt(x[2]);
+    o[2] = movt(x[1]);
+    o[3] = movt(x[3]);
+}
+
+// Step 3 on RN rows k_p at once: the rows are independent, so the compiler
+// interleaves their dependency chains (MMA -> convert -> twiddle -> MMA).
+// kc0/kc1: the rows' Khat words, tw: their W_M^{-q k_p} twiddles.
+template <int RN>
+__device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int (&kp)[RN], int lane,
+                                           const uint2 (&f16)[3][2], const uint2 (&w256)[4], const uint4 (&kc0)[RN],
+                                           const uint4 (&kc1)[RN], const uint2 (&tw)[RN][4], __nv_bfloat162 dm2) {
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
+    uint32_t xr[RN][4], xi[RN][4];
+#pragma unroll
+    for (int r = 0; r < RN; ++r) {
+        ldsm_x4_t(xr[r], plane_addr(sre, kp[r], chunk));
+        ldsm_x4_t(xi[r], plane_addr(sim, kp[r], chunk));
+    }
+    // stage i: [b][a] x F16 -> [b][c]; twiddle W_256^{b c}; transpose -> [c][b]
+    float acr[RN][2][4], aci[RN][2][4];
+#pragma unroll
+    for (int r = 0; r < RN; ++r)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
+#pragma unroll
+    for (int r = 0; r < RN; ++r) {
+        uint32_t tr[4], ti[4];
+        pack_tile(tr, acr[r]);
+        pack_tile(ti, aci[r]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+        transpose_tile(xr[r], tr);
+        transpose_tile(xi[r], ti);
+    }
+    // stage ii: [c][b] x F16 -> [c][d] (spectrum at k = k_p + P (c + 16 d))
+#pragma unroll
+    for (int r = 0; r < RN; ++r)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
+    // pointwise product with (Khat + D/M) on packed pairs; Khat regs hold (re pair, im pair)
+#pragma unroll
+    for (int r = 0; r < RN; ++r) {
+        pack_tile(xr[r], acr[r]);
+        pack_tile(xi[r], aci[r]);
+        const uint32_t kre[4] = {kc0[r].x, kc0[r].z, kc1[r].x, kc1[r].z};
+        const uint32_t kim[4] = {kc0[r].y, kc0[r].w, kc1[r].y, kc1[r].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 zr = as_b2(xr[r][i]), zi = as_b2(xi[r][i]);
+            const __nv_bfloat162 kr = __hadd2(as_b2(kre[i]), dm2), ki = as_b2(kim[i]);
+            xr[r][i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
+            xi[r][i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
+        }
+    }
+    // inverse stage ii: [c][d] x conj(F16) -> [c][b]; conj parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
+#pragma unroll
+    for (int r = 0; r < RN; ++r)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
+    // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
+#pragma unroll
+    for (int r = 0; r < RN; ++r) {
+        uint32_t gr[4], gi[4];
+        pack_tile(gr, acr[r]);
+        pack_tile(gi, aci[r]);
+        transpose_tile(xr[r], gr);
+        transpose_tile(xi[r], gi);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<false>(xr[r][i], xi[r][i], w256[i]);
+    }
+    // inverse stage i: [b][c] x conj(F16) -> [b][a]
+#pragma unroll
+    for (int r = 0; r < RN; ++r)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
+    // conj twiddle W_M^{-q k_p} (q = 16 a + b), back to row k_p
+#pragma unroll
+    for (int r = 0; r < RN; ++r) {
+        uint32_t qr[4], qi[4];
+        pack_tile(qr, acr[r]);
+        pack_tile(qi, aci[r]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], tw[r][i]);
+        // registers 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3 (b 8-15, a 8-15)
+        stsm_x4_t(plane_addr(sre, kp[r], chunk), qr[0], qr[1], qr[2], qr[3]);
+        stsm_x4_t(plane_addr(sim, kp[r], chunk), qi[0], qi[1], qi[2], qi[3]);
+    }
+}
+
 // Persistent: each CTA walks work items (pair pp of channel h) with stride
 // gridDim.x; items of one channel are consecutive so concurrent CTAs share
 // Khat[h] in L2.  The next item's input is fetched with cp.async into the
 // staging planes while the current item runs its inner transforms.
 template <int P, int NW, bool GATED>
-__global__ void __launch_bounds__(NW * 32, P <= 32 ? 4 : 2)
+__global__ void __launch_bounds__(NW * 32, P <= 32 ? 3 : 2)
 fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
              const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
              __nv_bfloat16* __restrict__ y, TcTables tb, int B, int H) {
@@ -294,88 +432,40 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         // the staging planes are free: fetch the next item while this one runs
         if (item + (int)gridDim.x < items) stage_input(item + gridDim.x);
 
-        // ---- step 3: inner 256-point DFT, product with Khat, inverse, per row k_p
-        const float dmf = D ? D[h] * (1.0f / S::M) : 0.f;
-        const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
-        const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
-        uint4 kn0 = __ldg(&kh[(size_t)warp * 64 + lane * 2]), kn1 = __ldg(&kh[(size_t)warp * 64 + lane * 2 + 1]);
-        uint2 tn[4];
+        // ---- step 3: inner 256-point DFT, product with Khat, inverse; two rows k_p per iteration
+        {
+            constexpr int RN = 2;
+            static_assert((P / NW) % RN == 0, "rows per warp must split into pairs");
+            const float dmf = D ? D[h] * (1.0f / S::M) : 0.f;
+            const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
+            const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
+            uint4 kn0[RN], kn1[RN];
+            uint2 tn[RN][4];
+            auto fetch = [&](int kp0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tn[i] = __ldg(&tb.tw3[((size_t)warp * 4 + i) * 32 + lane]);
-        for (int kp = warp; kp < P; kp += NW) {
-            const uint4 kc0 = kn0, kc1 = kn1;
-            uint2 tc3[4];
+                for (int r = 0; r < RN; ++r) {
+                    const int kp = kp0 + r * NW;
+                    kn0[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
+                    kn1[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) tc3[i] = tn[i];
-            if (kp + NW < P) {
-                kn0 = __ldg(&kh[(size_t)(kp + NW) * 64 + lane * 2]);
-                kn1 = __ldg(&kh[(size_t)(kp + NW) * 64 + lane * 2 + 1]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) tn[i] = __ldg(&tb.tw3[((size_t)(kp + NW) * 4 + i) * 32 + lane]);
-            }
-            uint32_t xr[4], xi[4];
-            const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
-            ldsm_x4_t(xr, plane_addr(sre, kp, chunk));
-            ldsm_x4_t(xi, plane_addr(sim, kp, chunk));
-            // stage i: [b][a] x F16 -> [b][c]
-            float ur[2][4] = {}, ui[2][4] = {};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) cmma(ur[j], ui[j], xr, xi, f16[0][j], f16[1][j], f16[2][j]);
-            uint32_t tr[4] = {pack2(ur[0][0], ur[0][1]), pack2(ur[0][2], ur[0][3]), pack2(ur[1][0], ur[1][1]),
-                              pack2(ur[1][2], ur[1][3])};
-            uint32_t ti[4] = {pack2(ui[0][0], ui[0][1]), pack2(ui[0][2], ui[0][3]), pack2(ui[1][0], ui[1][1]),
-                              pack2(ui[1][2], ui[1][3])};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
-            // transpose [b][c] -> [c][b]
-            uint32_t cr[4] = {movt(tr[0]), movt(tr[2]), movt(tr[1]), movt(tr[3])};
-            uint32_t ci[4] = {movt(ti[0]), movt(ti[2]), movt(ti[1]), movt(ti[3])};
-            // stage ii: [c][b] x F16 -> [c][d]  (spectrum at k = k_p + P (c + 16 d))
-            float vr[2][4] = {}, vi[2][4] = {};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) cmma(vr[j], vi[j], cr, ci, f16[0][j], f16[1][j], f16[2][j]);
-            uint32_t zr4[4] = {pack2(vr[0][0], vr[0][1]), pack2(vr[0][2], vr[0][3]), pack2(vr[1][0], vr[1][1]),
-                               pack2(vr[1][2], vr[1][3])};
-            uint32_t zi4[4] = {pack2(vi[0][0], vi[0][1]), pack2(vi[0][2], vi[0][3]), pack2(vi[1][0], vi[1][1]),
-                               pack2(vi[1][2], vi[1][3])};
-            // pointwise product with (Khat + D/M), packed: Khat regs i hold (re pair, im pair)
-            {
-                const uint32_t kre[4] = {kc0.x, kc0.z, kc1.x, kc1.z}, kim[4] = {kc0.y, kc0.w, kc1.y, kc1.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __nv_bfloat162 zr = as_b2(zr4[i]), zi = as_b2(zi4[i]);
-                    const __nv_bfloat162 kr = __hadd2(as_b2(kre[i]), dm2), ki = as_b2(kim[i]);
-                    zr4[i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
-                    zi4[i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
+                    for (int i = 0; i < 4; ++i) tn[r][i] = __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]);
                 }
+            };
+            fetch(warp);
+            for (int kp0 = warp; kp0 < P; kp0 += RN * NW) {
+                uint4 kc0[RN], kc1[RN];
+                uint2 tc3[RN][4];
+#pragma unroll
+                for (int r = 0; r < RN; ++r) {
+                    kc0[r] = kn0[r];
+                    kc1[r] = kn1[r];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) tc3[r][i] = tn[r][i];
+                }
+                if (kp0 + RN * NW < P) fetch(kp0 + RN * NW);
+                const int kps[RN] = {kp0, kp0 + NW};
+                inner_rows<RN>(sre, sim, kps, lane, f16, w256, kc0, kc1, tc3, dm2);
             }
-            // inverse stage ii: [c][d] x conj(F16) -> [c][b]; conj parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
-            float sr[2][4] = {}, si[2][4] = {};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) cmma(sr[j], si[j], zr4, zi4, f16[0][j], f16[2][j], f16[1][j]);
-            uint32_t gr[4] = {pack2(sr[0][0], sr[0][1]), pack2(sr[0][2], sr[0][3]), pack2(sr[1][0], sr[1][1]),
-                              pack2(sr[1][2], sr[1][3])};
-            uint32_t gi[4] = {pack2(si[0][0], si[0][1]), pack2(si[0][2], si[0][3]), pack2(si[1][0], si[1][1]),
-                              pack2(si[1][2], si[1][3])};
-            // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
-            uint32_t hr[4] = {movt(gr[0]), movt(gr[2]), movt(gr[1]), movt(gr[3])};
-            uint32_t hi[4] = {movt(gi[0]), movt(gi[2]), movt(gi[1]), movt(gi[3])};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) twiddle2<false>(hr[i], hi[i], w256[i]);
-            // inverse stage i: [b][c] x conj(F16) -> [b][a]
-            float or_[2][4] = {}, oi[2][4] = {};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) cmma(or_[j], oi[j], hr, hi, f16[0][j], f16[2][j], f16[1][j]);
-            uint32_t qr[4] = {pack2(or_[0][0], or_[0][1]), pack2(or_[0][2], or_[0][3]), pack2(or_[1][0], or_[1][1]),
-                              pack2(or_[1][2], or_[1][3])};
-            uint32_t qi[4] = {pack2(oi[0][0], oi[0][1]), pack2(oi[0][2], oi[0][3]), pack2(oi[1][0], oi[1][1]),
-                              pack2(oi[1][2], oi[1][3])};
-            // conj twiddle W_M^{-q k_p}, q = 16 a + b
-#pragma unroll
-            for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], tc3[i]);
-            // back to row k_p: registers 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3
-            stsm_x4_t(plane_addr(sre, kp, chunk), qr[0], qr[1], qr[2], qr[3]);
-            stsm_x4_t(plane_addr(sim, kp, chunk), qi[0], qi[1], qi[2], qi[3]);
         }
         __syncthreads();
 
