@@ -215,8 +215,12 @@ constexpr int kColTile = 16;  // columns per CTA in the column passes (128 B of 
 
 template <int LOG2N1>
 using ColG = Geometry<LOG2N1, kColTile, true>;
+// Rows per CTA in the row pass: enough that one CTA holds 4096 points (at
+// most 16 rows), so short rows do not leave single-warp CTAs.
+constexpr int row_batch(int log2n2) { return log2n2 >= 12 ? 1 : ((4096 >> log2n2) > 16 ? 16 : (4096 >> log2n2)); }
+
 template <int LOG2N2>
-using RowG = Geometry<LOG2N2, 1, false>;
+using RowG = Geometry<LOG2N2, row_batch(LOG2N2), false>;
 
 // W_M^e from the two-level table, e reduced mod M.
 __device__ __forceinline__ float2 twiddle_M(const float2* __restrict__ lo, const float2* __restrict__ hi,
@@ -287,35 +291,37 @@ mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __r
     constexpr int NS = G::Plan::kStages, R0 = first_radix<G>(), RL = last_radix<G>();
     extern __shared__ float2 smem[];
     const int tid = threadIdx.x;
-    const int k1 = blockIdx.x;
+    constexpr int RC = G::C;                    // rows k1 of this CTA: k1_0 .. k1_0 + RC - 1
+    const int k1_0 = blockIdx.x * RC;
     const int64_t P = first + blockIdx.y;
-    float2* __restrict__ row = work + ((size_t)blockIdx.y * N1 + k1) * N2;
-    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
-    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
-    stage<G, 0, false, R0, R0, false>(tid, twR, [&](int n2, int) { return row[n2]; }, sts);
+    float2* __restrict__ rows = work + ((size_t)blockIdx.y * N1 + k1_0) * N2;
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    stage<G, 0, false, R0, R0, false>(tid, twR, [&](int n2, int c) { return rows[(size_t)c * N2 + n2]; }, sts);
     __syncthreads();
     if constexpr (MODE == 1) {
         smem_stages<G, 1, NS - 1, false>(smem, tid, twR);
-        float2* __restrict__ out = khat_out + ((size_t)P * N1 + k1) * N2;
-        stage<G, NS - 1, false, RL, RL, false>(tid, twR, lds,
-                                                [&](int k2, int, float2 z) { out[k2] = cscale(z, 1.0f / M); });
+        float2* __restrict__ out = khat_out + ((size_t)P * N1 + k1_0) * N2;
+        stage<G, NS - 1, false, RL, RL, false>(
+            tid, twR, lds, [&](int k2, int c, float2 z) { out[(size_t)c * N2 + k2] = cscale(z, 1.0f / M); });
     } else {
         smem_stages<G, 1, NS, false>(smem, tid, twR);
         const int h = (int)(P % H);
         const float dm = D ? D[h] * (1.0f / M) : 0.f;
-        const float2* __restrict__ kh = khat + ((size_t)h * N1 + k1) * N2;
+        const float2* __restrict__ kh = khat + ((size_t)h * N1 + k1_0) * N2;
         stage<G, 0, true, R0, R0, true>(
             tid, twR,
-            [&](int k2, int) {
-                float2 kk = __ldg(&kh[k2]);
+            [&](int k2, int c) {
+                float2 kk = __ldg(&kh[(size_t)c * N2 + k2]);
                 kk.x += dm;
-                return cmul(smem[Lay::at(k2, 0)], kk);
+                return cmul(smem[Lay::at(k2, c)], kk);
             },
             sts);
         __syncthreads();
         smem_stages<G, 1, NS - 1, true>(smem, tid, twR);
-        stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int n2, int, float2 z) {
-            row[n2] = cmulc(z, twiddle_M(lo, hi, (uint32_t)n2 * (uint32_t)k1, LOG2M, log2S));
+        stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int n2, int c, float2 z) {
+            const uint32_t k1 = (uint32_t)(k1_0 + c);
+            rows[(size_t)c * N2 + n2] = cmulc(z, twiddle_M(lo, hi, (uint32_t)n2 * k1, LOG2M, log2S));
         });
     }
 }
@@ -367,7 +373,7 @@ static cudaError_t mp_fwd_go(const fftconv_plan_s& p, const void* u, const void*
         k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
                                                                p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S, p.B,
                                                                p.H, first);
-        k2<<<dim3(N1, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
+        k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
                                                     p.log2S, p.H, first);
         k3<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
                                                                p.H, first);
@@ -399,7 +405,7 @@ static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L
         const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
         k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(nullptr, nullptr, k, (int)L, work, p.tw.wC,
                                                                p.tw.wLo, p.tw.wHi, p.log2S, p.B, p.H, first);
-        k2<<<dim3(N1, g), RowG<LOG2N2>::T, sr, s>>>(work, nullptr, khat, nullptr, p.tw.wL, p.tw.wLo, p.tw.wHi,
+        k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, nullptr, khat, nullptr, p.tw.wL, p.tw.wLo, p.tw.wHi,
                                                     p.log2S, p.H, first);
     }
     return cudaGetLastError();
