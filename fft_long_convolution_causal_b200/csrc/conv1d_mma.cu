@@ -158,7 +158,10 @@ template <int P, bool GATED>
 struct TcSmem {
     static constexpr int kS = 2 * P * 512;      // S: re and im planes, P rows of 256 q
     static constexpr int kX = P * 512;          // x staging: re and im planes, P/2 rows
-    static constexpr int kBytes = kS + kX * (GATED ? 2 : 1);
+    // The gate input w has its own staging planes, except for the largest
+    // transform, where it is staged in S's upper rows (free until step 1).
+    static constexpr bool kWInS = P >= 128;
+    static constexpr int kBytes = kS + kX * ((GATED && !kWInS) ? 2 : 1);
 };
 
 // fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
@@ -279,18 +282,112 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
     }
 }
 
+// Step 1: for each 16-q tile, the outer DFT over the P/2 nonzero p (rows of
+// the staging planes x, times w when gated), times W_M^{q k_p}, stored
+// transposed into S[k_p][q].  Shared by the forward kernel and the spectrum
+// kernel of the largest transforms.
+template <int P, int NW, bool GATED, bool PRE1, int F1, int F2>
+__device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t wre, uint32_t wim, uint32_t sre,
+                                            uint32_t sim, int lane, int warp, const uint2 (&fp)[F1][F2][3],
+                                            const TcTables& tb) {
+    using S = TcShape<P>;
+    constexpr bool TW_PREFETCH = S::NT1 <= 4;  // small tables: fetch the next tile's twiddles early
+    const int m8 = lane >> 3, r8 = lane & 7;
+    uint2 twn[TW_PREFETCH ? S::NT1 : 1][2];
+    if (TW_PREFETCH && warp < 16) {
+#pragma unroll
+        for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                twn[TW_PREFETCH ? j : 0][hh] = __ldg(&tb.tw1[((warp * S::NT1 + j) * 2 + hh) * 32 + lane]);
+    }
+    for (int qt = warp; qt < 16; qt += NW) {
+        uint2 twc[TW_PREFETCH ? S::NT1 : 1][2];
+        if (TW_PREFETCH) {
+#pragma unroll
+            for (int j = 0; j < S::NT1; ++j) {
+                twc[TW_PREFETCH ? j : 0][0] = twn[TW_PREFETCH ? j : 0][0];
+                twc[TW_PREFETCH ? j : 0][1] = twn[TW_PREFETCH ? j : 0][1];
+            }
+            if (qt + NW < 16) {
+#pragma unroll
+                for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        twn[TW_PREFETCH ? j : 0][hh] =
+                            __ldg(&tb.tw1[(((qt + NW) * S::NT1 + j) * 2 + hh) * 32 + lane]);
+            }
+        }
+        uint32_t ar[S::KS1][4], ai[S::KS1][4];
+#pragma unroll
+        for (int ks = 0; ks < S::KS1; ++ks) {
+            // A[q][p] from rows p, chunks 2 qt (+1).  Rows p >= P/2 are the
+            // zero padding: those lanes point at row 0 (a select -- ldmatrix
+            // must run warp-converged) and their registers are zeroed.
+            const uint32_t prow0 = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+            const uint32_t prow = prow0 < (uint32_t)(P / 2) ? prow0 : 0u;
+            ldsm_x4_t(ar[ks], plane_addr(xre, prow, chunk));
+            ldsm_x4_t(ai[ks], plane_addr(xim, prow, chunk));
+            if (GATED) {
+                uint32_t gr[4], gi[4];
+                ldsm_x4_t(gr, plane_addr(wre, prow, chunk));
+                ldsm_x4_t(gi, plane_addr(wim, prow, chunk));
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    ar[ks][r] = as_u(__hmul2(as_b2(ar[ks][r]), as_b2(gr[r])));
+                    ai[ks][r] = as_u(__hmul2(as_b2(ai[ks][r]), as_b2(gi[r])));
+                }
+            }
+            if (16 * ks + 8 >= P / 2) ar[ks][2] = ar[ks][3] = ai[ks][2] = ai[ks][3] = 0u;
+        }
+        // every A fragment of this tile is in registers before any store below,
+        // so S may alias the staging rows of this tile's columns
+#pragma unroll
+        for (int j = 0; j < S::NT1; ++j) {
+            uint2 tw0, tw1;
+            if (TW_PREFETCH) {
+                tw0 = twc[TW_PREFETCH ? j : 0][0];
+                tw1 = twc[TW_PREFETCH ? j : 0][1];
+            } else {
+                tw0 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 0) * 32 + lane]);
+                tw1 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 1) * 32 + lane]);
+            }
+            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < S::KS1; ++ks) {
+                if (PRE1) {
+                    cmma(yr, yi, ar[ks], ai[ks], fp[PRE1 ? ks : 0][PRE1 ? j : 0][0],
+                         fp[PRE1 ? ks : 0][PRE1 ? j : 0][1], fp[PRE1 ? ks : 0][PRE1 ? j : 0][2]);
+                } else {
+                    const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
+                    cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                }
+            }
+            // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
+            uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
+            uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
+            twiddle2<true>(pr[0], pi[0], tw0);
+            twiddle2<true>(pr[1], pi[1], tw1);
+            // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
+            const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
+        }
+    }
+}
+
 // Persistent: each CTA walks work items (pair pp of channel h) with stride
 // gridDim.x; items of one channel are consecutive so concurrent CTAs share
 // Khat[h] in L2.  The next item's input is fetched with cp.async into the
 // staging planes while the current item runs its inner transforms.
 template <int P, int NW, bool GATED>
-__global__ void __launch_bounds__(NW * 32, P <= 32 ? 3 : 2)
+__global__ void __launch_bounds__(NW * 32, P <= 32 ? 3 : (P <= 64 ? 2 : 1))
 fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
              const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
              __nv_bfloat16* __restrict__ y, TcTables tb, int B, int H) {
     using S = TcShape<P>;
     using SM = TcSmem<P, GATED>;
-    static_assert(P >= 16 && P <= 64, "outer factor");
+    static_assert(P >= 16 && P <= 128, "outer factor");
+    static_assert((P / NW) % 2 == 0, "step 3 takes rows in pairs");
     constexpr int NT = NW * 32;
     constexpr int CH = S::N / 8;                          // 16-byte chunks per row of u
     constexpr bool PRE1 = S::NT1 * S::KS1 <= 4;           // keep step-1 B fragments in registers
@@ -302,9 +399,12 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     const int items = npp * H;
     const uint32_t sre = smem_u32(smem), sim = sre + S::kPlaneBytes;
     const uint32_t xre = sre + SM::kS, xim = xre + SM::kX / 2;
-    const uint32_t wre = xre + SM::kX, wim = wre + SM::kX / 2;
+    // w planes: separate, or S rows P/2 .. P-1 (plane_addr(w, p) == plane_addr(S, p + P/2))
+    const uint32_t wre = SM::kWInS ? sre + (P / 2) * 512u : xre + SM::kX;
+    const uint32_t wim = SM::kWInS ? sim + (P / 2) * 512u : xre + SM::kX + SM::kX / 2;
 
-    auto stage_input = [&](int item) {
+    // cp.async the input rows of one item: which = 1 (u), 2 (w), 3 (both)
+    auto stage_input = [&](int item, int which) {
         const int hh = item / npp, b0 = 2 * (item % npp);
         const bool has1 = b0 + 1 < B;
         const size_t r0 = ((size_t)b0 * H + hh) * S::N;
@@ -314,8 +414,8 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
             const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
             const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing row
             const size_t off = (plane ? r1 : r0) + n0;
-            cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
-            if (GATED) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
+            if (which & 1) cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
+            if (GATED && (which & 2)) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
         }
         cp_async_commit();
     };
@@ -351,7 +451,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
                         __ldg(&tb.fpi[((ks * S::NT3 + j) * 3 + part) * 32 + lane]);
     }
 
-    if ((int)blockIdx.x < items) stage_input(blockIdx.x);
+    if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3);
 
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
         const int h = item / npp, b0 = 2 * (item % npp);
@@ -362,75 +462,10 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         __syncthreads();
 
         // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
-        uint2 twn[S::NT1][2];
-        if (warp < 16) {
-#pragma unroll
-            for (int j = 0; j < S::NT1; ++j)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) twn[j][hh] = __ldg(&tb.tw1[((warp * S::NT1 + j) * 2 + hh) * 32 + lane]);
-        }
-        for (int qt = warp; qt < 16; qt += NW) {
-            uint2 twc[S::NT1][2];
-#pragma unroll
-            for (int j = 0; j < S::NT1; ++j) {
-                twc[j][0] = twn[j][0];
-                twc[j][1] = twn[j][1];
-            }
-            if (qt + NW < 16) {
-#pragma unroll
-                for (int j = 0; j < S::NT1; ++j)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        twn[j][hh] = __ldg(&tb.tw1[(((qt + NW) * S::NT1 + j) * 2 + hh) * 32 + lane]);
-            }
-            uint32_t ar[S::KS1][4], ai[S::KS1][4];
-#pragma unroll
-            for (int ks = 0; ks < S::KS1; ++ks) {
-                // A[q][p] from rows p, chunks 2 qt (+1).  Rows p >= P/2 are the
-                // zero padding: those lanes point at row 0 (a select -- ldmatrix
-                // must run warp-converged) and their registers are zeroed.
-                const uint32_t prow0 = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
-                const uint32_t prow = prow0 < (uint32_t)(P / 2) ? prow0 : 0u;
-                ldsm_x4_t(ar[ks], plane_addr(xre, prow, chunk));
-                ldsm_x4_t(ai[ks], plane_addr(xim, prow, chunk));
-                if (GATED) {
-                    uint32_t gr[4], gi[4];
-                    ldsm_x4_t(gr, plane_addr(wre, prow, chunk));
-                    ldsm_x4_t(gi, plane_addr(wim, prow, chunk));
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        ar[ks][r] = as_u(__hmul2(as_b2(ar[ks][r]), as_b2(gr[r])));
-                        ai[ks][r] = as_u(__hmul2(as_b2(ai[ks][r]), as_b2(gi[r])));
-                    }
-                }
-                if (16 * ks + 8 >= P / 2) ar[ks][2] = ar[ks][3] = ai[ks][2] = ai[ks][3] = 0u;
-            }
-#pragma unroll
-            for (int j = 0; j < S::NT1; ++j) {
-                float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < S::KS1; ++ks) {
-                    if (PRE1) {
-                        cmma(yr, yi, ar[ks], ai[ks], fp[PRE1 ? ks : 0][PRE1 ? j : 0][0],
-                             fp[PRE1 ? ks : 0][PRE1 ? j : 0][1], fp[PRE1 ? ks : 0][PRE1 ? j : 0][2]);
-                    } else {
-                        const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
-                        cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
-                    }
-                }
-                // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
-                uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
-                uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
-                twiddle2<true>(pr[0], pi[0], twc[j][0]);
-                twiddle2<true>(pr[1], pi[1], twc[j][1]);
-                // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
-                const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
-                stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
-            }
-        }
+        outer_step1<P, NW, GATED, PRE1>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb);
         __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
-        if (item + (int)gridDim.x < items) stage_input(item + gridDim.x);
+        if (item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3);
 
         // ---- step 3: inner 256-point DFT, product with Khat, inverse; two rows k_p per iteration
         {
@@ -498,6 +533,9 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         }
         __syncthreads();
 
+        // S rows P/2 .. P-1 are free again: fetch the next item's w into them
+        if (GATED && SM::kWInS && item + (int)gridDim.x < items) stage_input(item + gridDim.x, 2);
+
         // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
         for (int i = tid; i < 2 * CH; i += NT) {
             const int plane = i / CH, n0 = (i % CH) * 8;
@@ -520,6 +558,92 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         // the next iteration's wait + barrier orders these reads before S is rewritten
     }
     cp_async_wait_all();
+}
+
+// Spectrum on the tensor cores, for transforms too long for one CTA's SIMT
+// transform: k[h] (rounded to bf16) goes through step 1 and the forward half
+// of step 3 exactly as x does in the forward kernel, and the [c][d]
+// accumulators, scaled by 1/M, are written in the fragment order the forward
+// kernel reads (per row k_p and lane: re pair, im pair of registers 0..3).
+template <int P, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
+tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, TcTables tb) {
+    using S = TcShape<P>;
+    constexpr int NT = NW * 32;
+    constexpr bool PRE1 = S::NT1 * S::KS1 <= 4;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const int h = blockIdx.x;
+    const uint32_t sre = smem_u32(smem), sim = sre + S::kPlaneBytes;
+    const uint32_t xre = sre + 2 * S::kPlaneBytes, xim = xre + S::kPlaneBytes / 2;
+    uint2 f16[3][2], w256[4];
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+    uint2 fp[PRE1 ? S::KS1 : 1][PRE1 ? S::NT1 : 1][3];
+    if (PRE1) {
+#pragma unroll
+        for (int ks = 0; ks < S::KS1; ++ks)
+#pragma unroll
+            for (int j = 0; j < S::NT1; ++j)
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+                    fp[PRE1 ? ks : 0][PRE1 ? j : 0][part] =
+                        __ldg(&tb.fp[((ks * S::NT1 + j) * 3 + part) * 32 + lane]);
+    }
+    // stage k[h] (taps n < L, zero after) as the real plane, zero imaginary plane
+    const float* __restrict__ kr = k + (size_t)h * L;
+    for (int i = tid; i < S::N / 8; i += NT) {
+        const int n0 = i * 8;
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = (n0 + e < L) ? kr[n0 + e] : 0.f;
+        const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(plane_addr(xre, p, chunk)),
+                     "r"(pack2(t[0], t[1])), "r"(pack2(t[2], t[3])), "r"(pack2(t[4], t[5])), "r"(pack2(t[6], t[7]))
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(plane_addr(xim, p, chunk)), "r"(0u), "r"(0u),
+                     "r"(0u), "r"(0u)
+                     : "memory");
+    }
+    __syncthreads();
+    outer_step1<P, NW, false, PRE1>(xre, xim, 0u, 0u, sre, sim, lane, warp, fp, tb);
+    __syncthreads();
+    const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
+    const float inv_m = 1.0f / (float)S::M;
+    for (int kp = warp; kp < P; kp += NW) {
+        uint32_t xr[4], xi[4];
+        ldsm_x4_t(xr, plane_addr(sre, kp, chunk));
+        ldsm_x4_t(xi, plane_addr(sim, kp, chunk));
+        float acr[2][4] = {}, aci[2][4] = {};
+        cmma2(acr, aci, xr, xi, f16[0], f16[1], f16[2]);
+        uint32_t tr[4], ti[4];
+        pack_tile(tr, acr);
+        pack_tile(ti, aci);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+        transpose_tile(xr, tr);
+        transpose_tile(xi, ti);
+        float vr[2][4] = {}, vi[2][4] = {};
+        cmma2(vr, vi, xr, xi, f16[0], f16[1], f16[2]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                vr[j][e] *= inv_m;
+                vi[j][e] *= inv_m;
+            }
+        uint32_t zr[4], zi[4];
+        pack_tile(zr, vr);
+        pack_tile(zi, vi);
+        uint4* out = khat + ((size_t)h * P + kp) * 64 + lane * 2;
+        out[0] = make_uint4(zr[0], zi[0], zr[1], zi[1]);
+        out[1] = make_uint4(zr[2], zi[2], zr[3], zi[3]);
+    }
 }
 
 // Spectrum in the kernel's fragment order: the SIMT transform of k[h]
@@ -607,7 +731,7 @@ void push_bfrags(std::vector<float2>& out, int ksteps, int ntiles, F value) {
 
 }  // namespace
 
-bool tc_supported(int log2M) { return log2M >= 12 && log2M <= 14; }
+bool tc_supported(int log2M) { return log2M >= 12 && log2M <= 15; }
 
 bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]) {
     if (!tc_supported(log2M)) return false;
@@ -686,7 +810,7 @@ bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]) {
 template <int P, bool GATED>
 static cudaError_t tc_fwd_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
                              const void* khat, const float* D, void* y, cudaStream_t s) {
-    constexpr int NW = 4;
+    constexpr int NW = P >= 128 ? 16 : 4;  // the largest transform runs one CTA per SM
     auto kern = tc::fused_fwd_tc<P, NW, GATED>;
     const size_t smem = tc::TcSmem<P, GATED>::kBytes;
     // persistent grid: as many CTAs as are resident at once (computed once)
@@ -718,6 +842,7 @@ cudaError_t launch_tc_fwd(const fftconv_plan_s& p, const void* u, const void* v,
         case 12: return tc_fwd_g<16>(p, u, v, w, khat, D, y, s);
         case 13: return tc_fwd_g<32>(p, u, v, w, khat, D, y, s);
         case 14: return tc_fwd_g<64>(p, u, v, w, khat, D, y, s);
+        case 15: return tc_fwd_g<128>(p, u, v, w, khat, D, y, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -737,6 +862,14 @@ cudaError_t launch_tc_spectrum(const fftconv_plan_s& p, const float* k, int64_t 
         case 12: return tc_spec_go<12>(p, k, L, khat, s);
         case 13: return tc_spec_go<13>(p, k, L, khat, s);
         case 14: return tc_spec_go<14>(p, k, L, khat, s);
+        case 15: {
+            constexpr int P = 128, NW = 16;
+            auto kern = tc::tc_spectrum_mma<P, NW>;
+            const size_t smem = 3 * tc::TcShape<P>::kPlaneBytes;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            kern<<<p.H, NW * 32, smem, s>>>(k, (int)L, (uint4*)khat, p.tc);
+            return cudaGetLastError();
+        }
         default: return cudaErrorInvalidValue;
     }
 }

@@ -221,10 +221,25 @@ __device__ __forceinline__ void stage(int tid, const float2* __restrict__ tw, Lo
         const int k = j & (NS - 1);
         if (LOG2NS > 0) {
             // W_{Ns R}^{r k} from the stage's table, laid out [r][k] so that the
-            // consecutive k of a warp read consecutive entries
+            // consecutive k of a warp read consecutive entries.  For R >= 16 only
+            // the powers r = 1, 2, 4, 8 (16) are loaded; every other power is the
+            // product of the loaded ones for the set bits of r (at most
+            // log2(R) - 1 fp32 complex products, error ~1e-7), which moves the
+            // stage from load throughput to FMA throughput.
             constexpr int OFF = StageTwiddles<G>::offset(S);
+            if constexpr (R >= 16) {
+                float2 wp[R];
 #pragma unroll
-            for (int r = 1; r < IN_R; ++r) v[q][r] = cmul_dir<INV>(v[q][r], __ldg(&tw[OFF + r * NS + k]));
+                for (int r = 1; r < R; r <<= 1) wp[r] = __ldg(&tw[OFF + r * NS + k]);
+#pragma unroll
+                for (int r = 3; r < R; ++r)
+                    if (r & (r - 1)) wp[r] = cmul(wp[r & (r - 1)], wp[r & -r]);
+#pragma unroll
+                for (int r = 1; r < IN_R; ++r) v[q][r] = cmul_dir<INV>(v[q][r], wp[r]);
+            } else {
+#pragma unroll
+                for (int r = 1; r < IN_R; ++r) v[q][r] = cmul_dir<INV>(v[q][r], __ldg(&tw[OFF + r * NS + k]));
+            }
         }
         dft<R, INV>(v[q]);
         const int base = ((j >> LOG2NS) << (LOG2NS + LOG2R)) + k;

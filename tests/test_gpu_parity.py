@@ -52,7 +52,7 @@ FUSED_N = [64, 128, 256, 512, 1024, 2048, 4096, 8192]
 def test_fused_full_compare(N, dtype):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
     y, path = run_1d(wl)
-    want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 8192) else "fused"
+    want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 16384) else "fused"
     assert path == want
     assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}", scale=row_scale_1d(wl))
 
@@ -81,7 +81,7 @@ def test_partial_kernel(N, L):
         assert_close(y[b, h, t], ref, "f32", f"partial N={N} L={L}", scale=row_scale_1d(wl, b, h))
 
 
-@pytest.mark.parametrize("N", [2048, 4096, 8192])
+@pytest.mark.parametrize("N", [2048, 4096, 8192, 16384])
 @pytest.mark.parametrize("B,gated,with_D,L", [(1, False, True, None), (5, True, True, None),
                                              (2, False, False, 333), (3, True, False, None)])
 def test_tensor_core_path(N, B, gated, with_D, L):
@@ -108,8 +108,8 @@ def test_no_skip_term_and_single_row():
     assert_close(y, oracle_full(wl), "f32", "B=1 no D", scale=row_scale_1d(wl))
 
 
-@pytest.mark.parametrize("N", [16384, 32768])
-@pytest.mark.parametrize("dtype,gated", [("f32", False), ("bf16", True), ("bf16", False)])
+@pytest.mark.parametrize("N,dtype,gated", [(16384, "f32", False), (32768, "f32", False), (16384, "f32", True),
+                                           (32768, "bf16", True), (32768, "bf16", False)])
 def test_multipass_full_compare(N, dtype, gated):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=gated, seed=N + gated, with_D=True)
     y, path = run_1d(wl)
