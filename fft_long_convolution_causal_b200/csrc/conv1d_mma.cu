@@ -51,6 +51,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// d = A B (zero accumulator: C is the zero register, no moves to clear d)
+__device__ __forceinline__ void mma16816z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
 __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -66,10 +73,23 @@ __device__ __forceinline__ uint32_t movt(uint32_t x) {
     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
     return y;
 }
-// two fp32 -> packed bf16x2 (lo in the low half), round to nearest even
+// two fp32 -> packed bf16x2 (lo in the low half).  IP = false: the
+// conversion instruction, round to nearest even.  IP = true: round to nearest
+// (ties away from zero) with integer arithmetic -- adding half an ulp of bf16
+// (0x8000) to the fp32 bit pattern carries into the kept upper 16 bits exactly
+// when the dropped bits are at least half, and a byte permute takes the two
+// upper halves.  The integer form runs on the ALU instead of the conversion
+// unit; which is faster depends on the kernel's mix (measured per size).
+// Inputs are finite and far below FLT_MAX, so the carry never overflows.
+template <bool IP = false>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    if (IP) {
+        const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
+        asm("prmt.b32 %0, %1, %2, 0x7632;\n" : "=r"(r) : "r"(a), "r"(b));
+    } else {
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    }
     return r;
 }
 __device__ __forceinline__ __nv_bfloat162 as_b2(uint32_t x) { return *reinterpret_cast<__nv_bfloat162*>(&x); }
@@ -108,6 +128,37 @@ __device__ __forceinline__ void cmma2(float (&yr)[2][4], float (&yi)[2][4], cons
         mma16816(yr[j], ai, bni[j].x, bni[j].y);
         mma16816(yi[j], ai, br[j].x, br[j].y);
     }
+}
+
+// As cmma2, overwriting yr, yi (products start from zero).
+__device__ __forceinline__ void cmma2z(float (&yr)[2][4], float (&yi)[2][4], const uint32_t (&ar)[4],
+                                       const uint32_t (&ai)[4], const uint2 (&br)[2], const uint2 (&bi)[2],
+                                       const uint2 (&bni)[2]) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        mma16816z(yr[j], ar, br[j].x, br[j].y);
+        mma16816z(yi[j], ar, bi[j].x, bi[j].y);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        mma16816(yr[j], ai, bni[j].x, bni[j].y);
+        mma16816(yi[j], ai, br[j].x, br[j].y);
+    }
+}
+
+// Complex product on one 16 x 8 tile; FIRST: overwrite instead of accumulate.
+template <bool FIRST>
+__device__ __forceinline__ void cmma_k(float (&yr)[4], float (&yi)[4], const uint32_t (&ar)[4],
+                                       const uint32_t (&ai)[4], uint2 br, uint2 bi, uint2 bni) {
+    if (FIRST) {
+        mma16816z(yr, ar, br.x, br.y);
+        mma16816z(yi, ar, bi.x, bi.y);
+    } else {
+        mma16816(yr, ar, br.x, br.y);
+        mma16816(yi, ar, bi.x, bi.y);
+    }
+    mma16816(yr, ai, bni.x, bni.y);
+    mma16816(yi, ai, br.x, br.y);
 }
 
 // Complex tile product on one 16 x 8 output tile:
@@ -166,11 +217,12 @@ struct TcSmem {
 
 // fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
 // registers of the 16x16 A fragment they form.
+template <bool IP = false>
 __device__ __forceinline__ void pack_tile(uint32_t (&o)[4], const float (&t)[2][4]) {
-    o[0] = pack2(t[0][0], t[0][1]);
-    o[1] = pack2(t[0][2], t[0][3]);
-    o[2] = pack2(t[1][0], t[1][1]);
-    o[3] = pack2(t[1][2], t[1][3]);
+    o[0] = pack2<IP>(t[0][0], t[0][1]);
+    o[1] = pack2<IP>(t[0][2], t[0][3]);
+    o[2] = pack2<IP>(t[1][0], t[1][1]);
+    o[3] = pack2<IP>(t[1][2], t[1][3]);
 }
 // 16x16 transpose of an A fragment: block (r, c) -> (c, r), each 8x8 block transposed.
 __device__ __forceinline__ void transpose_tile(uint32_t (&o)[4], const uint32_t (&x)[4]) {
@@ -183,7 +235,7 @@ __device__ __forceinline__ void transpose_tile(uint32_t (&o)[4], const uint32_t 
 // Step 3 on RN rows k_p at once: the rows are independent, so the compiler
 // interleaves their dependency chains (MMA -> convert -> twiddle -> MMA).
 // kc0/kc1: the rows' Khat words, tw: their W_M^{-q k_p} twiddles.
-template <int RN>
+template <int RN, bool IP>
 __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int (&kp)[RN], int lane,
                                            const uint2 (&f16)[3][2], const uint2 (&w256)[4], const uint4 (&kc0)[RN],
                                            const uint4 (&kc1)[RN], const uint2 (&tw)[RN][4], __nv_bfloat162 dm2) {
@@ -198,18 +250,12 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
     // stage i: [b][a] x F16 -> [b][c]; twiddle W_256^{b c}; transpose -> [c][b]
     float acr[RN][2][4], aci[RN][2][4];
 #pragma unroll
-    for (int r = 0; r < RN; ++r)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
-#pragma unroll
-    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
+    for (int r = 0; r < RN; ++r) cmma2z(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
 #pragma unroll
     for (int r = 0; r < RN; ++r) {
         uint32_t tr[4], ti[4];
-        pack_tile(tr, acr[r]);
-        pack_tile(ti, aci[r]);
+        pack_tile<IP>(tr, acr[r]);
+        pack_tile<IP>(ti, aci[r]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
         transpose_tile(xr[r], tr);
@@ -217,18 +263,12 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
     }
     // stage ii: [c][b] x F16 -> [c][d] (spectrum at k = k_p + P (c + 16 d))
 #pragma unroll
-    for (int r = 0; r < RN; ++r)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
-#pragma unroll
-    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
+    for (int r = 0; r < RN; ++r) cmma2z(acr[r], aci[r], xr[r], xi[r], f16[0], f16[1], f16[2]);
     // pointwise product with (Khat + D/M) on packed pairs; Khat regs hold (re pair, im pair)
 #pragma unroll
     for (int r = 0; r < RN; ++r) {
-        pack_tile(xr[r], acr[r]);
-        pack_tile(xi[r], aci[r]);
+        pack_tile<IP>(xr[r], acr[r]);
+        pack_tile<IP>(xi[r], aci[r]);
         const uint32_t kre[4] = {kc0[r].x, kc0[r].z, kc1[r].x, kc1[r].z};
         const uint32_t kim[4] = {kc0[r].y, kc0[r].w, kc1[r].y, kc1[r].w};
 #pragma unroll
@@ -241,19 +281,13 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
     }
     // inverse stage ii: [c][d] x conj(F16) -> [c][b]; conj parts (Re, Im, -Im) = (f16[0], f16[2], f16[1])
 #pragma unroll
-    for (int r = 0; r < RN; ++r)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
-#pragma unroll
-    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
+    for (int r = 0; r < RN; ++r) cmma2z(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
     // transpose [c][b] -> [b][c], conj twiddle W_256^{-b c}
 #pragma unroll
     for (int r = 0; r < RN; ++r) {
         uint32_t gr[4], gi[4];
-        pack_tile(gr, acr[r]);
-        pack_tile(gi, aci[r]);
+        pack_tile<IP>(gr, acr[r]);
+        pack_tile<IP>(gi, aci[r]);
         transpose_tile(xr[r], gr);
         transpose_tile(xi[r], gi);
 #pragma unroll
@@ -261,19 +295,13 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
     }
     // inverse stage i: [b][c] x conj(F16) -> [b][a]
 #pragma unroll
-    for (int r = 0; r < RN; ++r)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acr[r][j][e] = aci[r][j][e] = 0.f;
-#pragma unroll
-    for (int r = 0; r < RN; ++r) cmma2(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
+    for (int r = 0; r < RN; ++r) cmma2z(acr[r], aci[r], xr[r], xi[r], f16[0], f16[2], f16[1]);
     // conj twiddle W_M^{-q k_p} (q = 16 a + b), back to row k_p
 #pragma unroll
     for (int r = 0; r < RN; ++r) {
         uint32_t qr[4], qi[4];
-        pack_tile(qr, acr[r]);
-        pack_tile(qi, aci[r]);
+        pack_tile<IP>(qr, acr[r]);
+        pack_tile<IP>(qi, aci[r]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) twiddle2<false>(qr[i], qi[i], tw[r][i]);
         // registers 0 (b 0-7, a 0-7), 1 (b 8-15, a 0-7), 2 (b 0-7, a 8-15), 3 (b 8-15, a 8-15)
@@ -286,7 +314,7 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
 // the staging planes x, times w when gated), times W_M^{q k_p}, stored
 // transposed into S[k_p][q].  Shared by the forward kernel and the spectrum
 // kernel of the largest transforms.
-template <int P, int NW, bool GATED, bool PRE1, int F1, int F2>
+template <int P, int NW, bool GATED, bool PRE1, bool IP, int F1, int F2>
 __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t wre, uint32_t wim, uint32_t sre,
                                             uint32_t sim, int lane, int warp, const uint2 (&fp)[F1][F2][3],
                                             const TcTables& tb) {
@@ -352,20 +380,26 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
                 tw0 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 0) * 32 + lane]);
                 tw1 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 1) * 32 + lane]);
             }
-            float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+            float yr[4], yi[4];
 #pragma unroll
             for (int ks = 0; ks < S::KS1; ++ks) {
+                uint2 b0, b1, b2;
                 if (PRE1) {
-                    cmma(yr, yi, ar[ks], ai[ks], fp[PRE1 ? ks : 0][PRE1 ? j : 0][0],
-                         fp[PRE1 ? ks : 0][PRE1 ? j : 0][1], fp[PRE1 ? ks : 0][PRE1 ? j : 0][2]);
+                    b0 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][0];
+                    b1 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][1];
+                    b2 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][2];
                 } else {
                     const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
-                    cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                    b0 = __ldg(fb);
+                    b1 = __ldg(fb + 32);
+                    b2 = __ldg(fb + 64);
                 }
+                if (ks == 0) cmma_k<true>(yr, yi, ar[ks], ai[ks], b0, b1, b2);
+                else cmma_k<false>(yr, yi, ar[ks], ai[ks], b0, b1, b2);
             }
             // rows q = 16 qt + g (+8), cols k_p = 8 j + 2t (+1)
-            uint32_t pr[2] = {pack2(yr[0], yr[1]), pack2(yr[2], yr[3])};
-            uint32_t pi[2] = {pack2(yi[0], yi[1]), pack2(yi[2], yi[3])};
+            uint32_t pr[2] = {pack2<IP>(yr[0], yr[1]), pack2<IP>(yr[2], yr[3])};
+            uint32_t pi[2] = {pack2<IP>(yi[0], yi[1]), pack2<IP>(yi[2], yi[3])};
             twiddle2<true>(pr[0], pi[0], tw0);
             twiddle2<true>(pr[1], pi[1], tw1);
             // store transposed: rows k_p = 8 j + r, chunk 2 qt + hh
@@ -388,6 +422,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     using SM = TcSmem<P, GATED>;
     static_assert(P >= 16 && P <= 128, "outer factor");
     static_assert((P / NW) % 2 == 0, "step 3 takes rows in pairs");
+    constexpr bool IP = P >= 128;  // integer packing measured faster only for the largest transform
     constexpr int NT = NW * 32;
     constexpr int CH = S::N / 8;                          // 16-byte chunks per row of u
     constexpr bool PRE1 = S::NT1 * S::KS1 <= 4;           // keep step-1 B fragments in registers
@@ -462,7 +497,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         __syncthreads();
 
         // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
-        outer_step1<P, NW, GATED, PRE1>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb);
+        outer_step1<P, NW, GATED, PRE1, IP>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb);
         __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
         if (item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3);
@@ -499,7 +534,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
                 }
                 if (kp0 + RN * NW < P) fetch(kp0 + RN * NW);
                 const int kps[RN] = {kp0, kp0 + NW};
-                inner_rows<RN>(sre, sim, kps, lane, f16, w256, kc0, kc1, tc3, dm2);
+                inner_rows<RN, IP>(sre, sim, kps, lane, f16, w256, kc0, kc1, tc3, dm2);
             }
         }
         __syncthreads();
@@ -515,20 +550,26 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
             }
 #pragma unroll
             for (int j = 0; j < S::NT3; ++j) {
-                float yr[4] = {0.f, 0.f, 0.f, 0.f}, yi[4] = {0.f, 0.f, 0.f, 0.f};
+                float yr[4], yi[4];
 #pragma unroll
                 for (int ks = 0; ks < S::KS3; ++ks) {
+                    uint2 b0, b1, b2;
                     if (PRE3) {
-                        cmma(yr, yi, ar[ks], ai[ks], fpi[PRE3 ? ks : 0][PRE3 ? j : 0][0],
-                             fpi[PRE3 ? ks : 0][PRE3 ? j : 0][1], fpi[PRE3 ? ks : 0][PRE3 ? j : 0][2]);
+                        b0 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][0];
+                        b1 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][1];
+                        b2 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][2];
                     } else {
                         const uint2* fb = tb.fpi + ((size_t)(ks * S::NT3 + j) * 3) * 32 + lane;
-                        cmma(yr, yi, ar[ks], ai[ks], __ldg(fb), __ldg(fb + 32), __ldg(fb + 64));
+                        b0 = __ldg(fb);
+                        b1 = __ldg(fb + 32);
+                        b2 = __ldg(fb + 64);
                     }
+                    if (ks == 0) cmma_k<true>(yr, yi, ar[ks], ai[ks], b0, b1, b2);
+                    else cmma_k<false>(yr, yi, ar[ks], ai[ks], b0, b1, b2);
                 }
                 const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
-                stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk), pack2(yr[0], yr[1]), pack2(yr[2], yr[3]),
-                          pack2(yi[0], yi[1]), pack2(yi[2], yi[3]));
+                stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk), pack2<IP>(yr[0], yr[1]), pack2<IP>(yr[2], yr[3]),
+                          pack2<IP>(yi[0], yi[1]), pack2<IP>(yi[2], yi[3]));
             }
         }
         __syncthreads();
@@ -611,7 +652,7 @@ tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, Tc
                      : "memory");
     }
     __syncthreads();
-    outer_step1<P, NW, false, PRE1>(xre, xim, 0u, 0u, sre, sim, lane, warp, fp, tb);
+    outer_step1<P, NW, false, PRE1, true>(xre, xim, 0u, 0u, sre, sim, lane, warp, fp, tb);
     __syncthreads();
     const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
     const float inv_m = 1.0f / (float)S::M;
@@ -619,8 +660,8 @@ tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, Tc
         uint32_t xr[4], xi[4];
         ldsm_x4_t(xr, plane_addr(sre, kp, chunk));
         ldsm_x4_t(xi, plane_addr(sim, kp, chunk));
-        float acr[2][4] = {}, aci[2][4] = {};
-        cmma2(acr, aci, xr, xi, f16[0], f16[1], f16[2]);
+        float acr[2][4], aci[2][4];
+        cmma2z(acr, aci, xr, xi, f16[0], f16[1], f16[2]);
         uint32_t tr[4], ti[4];
         pack_tile(tr, acr);
         pack_tile(ti, aci);
@@ -628,8 +669,8 @@ tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, Tc
         for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
         transpose_tile(xr, tr);
         transpose_tile(xi, ti);
-        float vr[2][4] = {}, vi[2][4] = {};
-        cmma2(vr, vi, xr, xi, f16[0], f16[1], f16[2]);
+        float vr[2][4], vi[2][4];
+        cmma2z(vr, vi, xr, xi, f16[0], f16[1], f16[2]);
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
