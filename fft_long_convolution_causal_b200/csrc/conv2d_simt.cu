@@ -11,6 +11,8 @@
 //   pass 2: per 16-column tile: column DFT_{2Hs} over the Hs nonzero rows,
 //           times Khat[c][ky][kx], inverse column DFT keeping rows i < Hs -> work
 //   pass 3: inverse row DFT_{2Ws} of the Hs rows, keeping j < Ws -> y.
+#include <type_traits>
+
 #include "fft_simt.cuh"
 #include "plan.h"
 #include "tables.h"
@@ -52,7 +54,9 @@ c2_pass1(const IO* __restrict__ u, const float* __restrict__ k, int Kh, int Kw, 
     auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
     auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
     if constexpr (MODE == 0) {
-        const int ch = (int)(P % C), b0 = (int)(P / C) * 2;
+        // pairs are channel-major (P = ch * npp + pp): a channel's pairs run together
+        const int npp = (B + 1) / 2;
+        const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
         const bool has1 = b0 + 1 < B;
         const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
         stage<G, 0, false, R0 / 2, R0, false>(
@@ -82,10 +86,11 @@ c2_pass1(const IO* __restrict__ u, const float* __restrict__ k, int Kh, int Kw, 
 
 // Pass 2. MODE 0: column DFT, product, inverse column DFT (rows < Hs kept).
 //         MODE 1: column DFT only; Khat[c][ky][kx] = X / (LC LR).
-template <int LOG2LC, int LOG2LR, int MODE>
+// KB: the spectrum is stored as packed bf16 (re, im) words (bf16 plans), else fp32 complex.
+template <int LOG2LC, int LOG2LR, int MODE, bool KB>
 __global__ void __launch_bounds__(Col2G<LOG2LC>::T)
-c2_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __restrict__ khat_out,
-         const float2* __restrict__ twC, int C, int64_t first) {
+c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restrict__ khat_out,
+         const float2* __restrict__ twC, int npp, int64_t first) {
     using G = Col2G<LOG2LC>;
     using Lay = typename G::Lay;
     constexpr int LC = 1 << LOG2LC, LR = 1 << LOG2LR, Hs = LC / 2;
@@ -103,17 +108,34 @@ c2_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __r
     __syncthreads();
     if constexpr (MODE == 1) {
         smem_stages<G, 1, NS - 1, false>(smem, tid, twC);
-        float2* __restrict__ out = khat_out + (size_t)P * LC * LR;
+        const size_t base = (size_t)P * LC * LR;
         constexpr float scale = 1.0f / ((float)LC * (float)LR);
         stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int ky, int c, float2 z) {
-            out[(size_t)ky * LR + kx0 + c] = cscale(z, scale);
+            const size_t o = base + (size_t)ky * LR + kx0 + c;
+            z = cscale(z, scale);
+            if (KB)
+                static_cast<uint32_t*>(khat_out)[o] =
+                    (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.x)) |
+                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.y)) << 16);
+            else
+                static_cast<float2*>(khat_out)[o] = z;
         });
     } else {
         smem_stages<G, 1, NS, false>(smem, tid, twC);
-        const float2* __restrict__ kh = khat + (size_t)(P % C) * LC * LR;
+        const size_t kbase = (size_t)(P / npp) * LC * LR;
         stage<G, 0, true, R0, R0, true>(
             tid, twC,
-            [&](int ky, int c) { return cmul(smem[Lay::at(ky, c)], __ldg(&kh[(size_t)ky * LR + kx0 + c])); },
+            [&](int ky, int c) {
+                const size_t o = kbase + (size_t)ky * LR + kx0 + c;
+                float2 kk;
+                if (KB) {
+                    const uint32_t wv = __ldg(static_cast<const uint32_t*>(khat) + o);
+                    kk = make_float2(__uint_as_float(wv << 16), __uint_as_float(wv & 0xffff0000u));
+                } else {
+                    kk = __ldg(static_cast<const float2*>(khat) + o);
+                }
+                return cmul(smem[Lay::at(ky, c)], kk);
+            },
             sts);
         __syncthreads();
         smem_stages<G, 1, NS - 1, true>(smem, tid, twC);
@@ -144,7 +166,8 @@ c2_pass3(const float2* __restrict__ work, IO* __restrict__ y, const float2* __re
         tid, twR, [&](int kx, int r) { return in[(size_t)(i0 + r) * LR + kx]; }, sts);
     __syncthreads();
     smem_stages<G, 1, NS - 1, true>(smem, tid, twR);
-    const int ch = (int)(P % C), b0 = (int)(P / C) * 2;
+    const int npp = (B + 1) / 2;
+    const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
     const bool has1 = b0 + 1 < B;
     const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
     stage<G, NS - 1, true, RL, RL / 2, false>(tid, twR, lds, [&](int j, int r, float2 z) {
@@ -161,7 +184,7 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
     constexpr int RB = rows_per_cta<LOG2LR>(Hs);
     constexpr int LR = 1 << LOG2LR;
     auto k1 = c2_pass1<LOG2LR, RB, IO, 0>;
-    auto k2 = c2_pass2<LOG2LC, LOG2LR, 0>;
+    auto k2 = c2_pass2<LOG2LC, LOG2LR, 0, std::is_same<IO, __nv_bfloat16>::value>;
     auto k3 = c2_pass3<LOG2LR, RB, IO>;
     const size_t sr = Row2G<LOG2LR, RB>::Lay::kWords * sizeof(float2);
     const size_t sc = Col2G<LOG2LC>::Lay::kWords * sizeof(float2);
@@ -172,20 +195,21 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
         k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>((const IO*)u, nullptr, 0, 0, work, p.tw.wL, p.B,
                                                              p.H, Hs, first);
-        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, p.H, first);
+        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, (p.B + 1) / 2,
+                                                                first);
         k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first);
     }
     return cudaGetLastError();
 }
 
-template <int LOG2LC, int LOG2LR>
-static cudaError_t c2_spec_go(const fftconv_plan_s& p, const float* k, int Kh, int Kw, float2* khat,
-                              float2* work, cudaStream_t s) {
+template <int LOG2LC, int LOG2LR, bool KB>
+static cudaError_t c2_spec_go(const fftconv_plan_s& p, const float* k, int Kh, int Kw, void* khat, float2* work,
+                              cudaStream_t s) {
     constexpr int Hs = (1 << LOG2LC) / 2;
     constexpr int RB = rows_per_cta<LOG2LR>(Hs);
     constexpr int LR = 1 << LOG2LR;
     auto k1 = c2_pass1<LOG2LR, RB, float, 1>;
-    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1>;
+    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1, KB>;
     const size_t sr = Row2G<LOG2LR, RB>::Lay::kWords * sizeof(float2);
     const size_t sc = Col2G<LOG2LC>::Lay::kWords * sizeof(float2);
     ensure_smem2(k1, sr);
@@ -194,7 +218,7 @@ static cudaError_t c2_spec_go(const fftconv_plan_s& p, const float* k, int Kh, i
         const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
         k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(nullptr, k, Kh, Kw, work, p.tw.wL, p.B, p.H, Hs,
                                                              first);
-        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, nullptr, khat, p.tw.wC, p.H, first);
+        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, nullptr, khat, p.tw.wC, 1, first);
     }
     return cudaGetLastError();
 }
@@ -224,7 +248,8 @@ static cudaError_t c2_spec_w(const fftconv_plan_s& p, const float* k, int Kh, in
                              cudaStream_t s) {
     switch (ilog2_host(p.Ws)) {
 #define FFTC_C(LW) \
-    case LW: return c2_spec_go<LOG2LC, LW + 1>(p, k, Kh, Kw, khat, work, s);
+    case LW: return p.dtype == FFTCONV_BF16 ? c2_spec_go<LOG2LC, LW + 1, true>(p, k, Kh, Kw, khat, work, s) \
+                                            : c2_spec_go<LOG2LC, LW + 1, false>(p, k, Kh, Kw, khat, work, s);
         FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
 #undef FFTC_C
         default: return cudaErrorInvalidValue;

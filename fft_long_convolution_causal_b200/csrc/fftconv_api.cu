@@ -173,11 +173,16 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
     const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
     int64_t g = (int64_t)(kGroupBytes / per_pair);
+    // whole channels per group: a channel's pairs then run together and share
+    // the channel's spectrum in L2
+    const int64_t npp = (B + 1) / 2;
+    if (g >= npp) g -= g % npp;
     if (g < 1) g = 1;
     const int64_t most = p->pairs > C ? p->pairs : C;
     if (g > most) g = most;
     p->group = (int)g;
-    p->spectrum_bytes = (size_t)C * LC * LR * sizeof(float2);
+    // bf16 plans keep the spectrum as packed bf16 (re, im), fp32 plans as fp32 complex
+    p->spectrum_bytes = (size_t)C * LC * LR * (dtype == FFTCONV_BF16 ? sizeof(uint32_t) : sizeof(float2));
     p->workspace_bytes = (size_t)g * per_pair;
     fftconv_status st = upload_tables(p, host);
     if (st != FFTCONV_OK) {
