@@ -222,6 +222,11 @@ constexpr int row_batch(int log2n2) { return log2n2 >= 12 ? 1 : ((4096 >> log2n2
 template <int LOG2N2>
 using RowG = Geometry<LOG2N2, row_batch(LOG2N2), false>;
 
+// Outputs per exact twiddle lookup in the pass epilogues; in between the
+// twiddle is advanced by one fp32 complex product (at most kTwRun - 1 chained
+// products: relative error below 1e-6).
+constexpr int kTwRun = 8;
+
 // W_M^e from the two-level table, e reduced mod M.
 __device__ __forceinline__ float2 twiddle_M(const float2* __restrict__ lo, const float2* __restrict__ hi,
                                             uint32_t e, int log2M, int log2S) {
@@ -271,9 +276,14 @@ mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __rest
     __syncthreads();
     smem_stages<G, 1, NS - 1, false>(smem, tid, twC);
     float2* __restrict__ out = work + (size_t)blockIdx.y * ((size_t)N1 * N2);
-    stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int k1, int c, float2 z) {
-        const int n2 = n2_0 + c;
-        out[(size_t)k1 * N2 + n2] = cmul(z, twiddle_M(lo, hi, (uint32_t)n2 * (uint32_t)k1, LOG2M, log2S));
+    // W_M^{n2 k1} along the thread's outputs k1 = j + r N1/RL: looked up every
+    // kTwRun outputs, advanced by W_M^{n2 N1/RL} in between
+    float2 tw = make_float2(1.f, 0.f), step = make_float2(1.f, 0.f);
+    stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int k1, int c, float2 z, int r) {
+        const uint32_t n2 = (uint32_t)(n2_0 + c);
+        if (r == 0) step = twiddle_M(lo, hi, n2 * (uint32_t)(N1 / RL), LOG2M, log2S);
+        tw = (r % kTwRun == 0) ? twiddle_M(lo, hi, n2 * (uint32_t)k1, LOG2M, log2S) : cmul(tw, step);
+        out[(size_t)k1 * N2 + n2] = cmul(z, tw);
     });
 }
 
@@ -319,9 +329,13 @@ mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __r
             sts);
         __syncthreads();
         smem_stages<G, 1, NS - 1, true>(smem, tid, twR);
-        stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int n2, int c, float2 z) {
+        // W_M^{n2 k1} along the thread's outputs n2 = j + r N2/RL (see pass 1)
+        float2 tw = make_float2(1.f, 0.f), step = make_float2(1.f, 0.f);
+        stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int n2, int c, float2 z, int r) {
             const uint32_t k1 = (uint32_t)(k1_0 + c);
-            rows[(size_t)c * N2 + n2] = cmulc(z, twiddle_M(lo, hi, (uint32_t)n2 * k1, LOG2M, log2S));
+            if (r == 0) step = twiddle_M(lo, hi, k1 * (uint32_t)(N2 / RL), LOG2M, log2S);
+            tw = (r % kTwRun == 0) ? twiddle_M(lo, hi, (uint32_t)n2 * k1, LOG2M, log2S) : cmul(tw, step);
+            rows[(size_t)c * N2 + n2] = cmulc(z, tw);
         });
     }
 }

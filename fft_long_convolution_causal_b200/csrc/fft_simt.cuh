@@ -24,6 +24,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace fftc {
 
 // ---------------------------------------------------------------- complex ops
@@ -244,7 +246,13 @@ __device__ __forceinline__ void stage(int tid, const float2* __restrict__ tw, Lo
         dft<R, INV>(v[q]);
         const int base = ((j >> LOG2NS) << (LOG2NS + LOG2R)) + k;
 #pragma unroll
-        for (int r = 0; r < OUT_R; ++r) store(base + r * NS, c, v[q][r]);
+        for (int r = 0; r < OUT_R; ++r) {
+            // a store functor may also take r (a compile-time index after unrolling)
+            if constexpr (std::is_invocable_v<StoreF, int, int, float2, int>)
+                store(base + r * NS, c, v[q][r], r);
+            else
+                store(base + r * NS, c, v[q][r]);
+        }
     }
 }
 
