@@ -208,7 +208,7 @@ class Runner:
                           y=y, workspace=self.ws)
 
     def launches_per_step(self):
-        if self.plan.path in ("fused", "fused_tc"):
+        if self.plan.path in ("fused", "fused_tc", "fused_umma"):
             return 1
         pairs = ((self.wl.B + 1) // 2) * (self.wl.C if self.is2d else self.wl.H)
         group = max(1, self.plan.workspace_bytes // self._pair_bytes())
@@ -220,11 +220,12 @@ class Runner:
         return 2 * self.wl.N * 8
 
     def compute_dtype(self):
-        return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16"}.get(self.plan.path, "f32")
+        return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16",
+                "fused_umma": "bf16"}.get(self.plan.path, "f32")
 
     def dominant_kernel(self):
         return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2",
-                "fused_tc": "fused_fwd_tc"}.get(self.plan.path)
+                "fused_tc": "fused_fwd_tc", "fused_umma": "fused_fwd_umma"}.get(self.plan.path)
 
 
 def time_steps(r, steps, torch, flush):

@@ -40,6 +40,7 @@ _SIGS = {
     "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv_fwd_static_workspace": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv_static_workspace_bytes": (ctypes.c_size_t, []),
+    "fftconv_device_status": (ctypes.c_int, [_vp, _vp]),
     "fftconv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fftconv_version": (ctypes.c_int, []),
 }
@@ -129,6 +130,10 @@ class _PlanBase:
     @property
     def path(self) -> str:
         return self.lib.fftconv_plan_path(self._handle).decode()
+
+    def device_status(self, stream=None) -> int:
+        """Synchronise the stream; 0, or 6 (timed out) once after a launch whose device wait gave up."""
+        return int(self.lib.fftconv_device_status(self._handle, _stream(stream)))
 
     def new_spectrum(self, device=None) -> torch.Tensor:
         return torch.empty(self.spectrum_bytes, dtype=torch.uint8, device=device or "cuda")

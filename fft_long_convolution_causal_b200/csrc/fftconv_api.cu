@@ -49,6 +49,15 @@ fftconv_status upload_tables(fftconv_plan_s* p, const std::vector<float2>& host)
     return FFTCONV_OK;
 }
 
+// A zeroed 16-byte slot at the end of the tables for the device status word.
+size_t append_status_word(std::vector<float2>& host) {
+    if (host.size() % 2) host.push_back(make_float2(0.f, 0.f));
+    const size_t off = host.size();
+    host.push_back(make_float2(0.f, 0.f));
+    host.push_back(make_float2(0.f, 0.f));
+    return off;
+}
+
 fftconv_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return FFTCONV_OK;
     return FFTCONV_ERR_CUDA;
@@ -92,12 +101,18 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
     cudaGetDevice(&p->device);
     std::vector<float2> host;
     const int64_t M = int64_t(1) << p->log2M;
-    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[6] = {0, 0, 0, 0, 0, 0};
+    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[6] = {0, 0, 0, 0, 0, 0}, offU = 0;
     const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && !getenv("FFTCONV_NO_TC");
     if (use_tc) {
         p->path = fftc::PATH_FUSED_TC;
         fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the spectrum transform
         fftc::tc_tables(p->log2M, host, offTc);
+        // tcgen05 kernel: opt-in (FFTCONV_UMMA=1) until it is the faster one
+        const char* um = getenv("FFTCONV_UMMA");
+        if (fftc::umma_supported(p->log2M) && um && um[0] == '1') {
+            p->umma = true;
+            fftc::umma_bimages(p->log2M, host, &offU);
+        }
         p->spectrum_bytes = (size_t)H * M * sizeof(uint32_t);  // bf16 (re, im) in fragment order
         p->workspace_bytes = 0;
     } else if (p->log2M <= kFusedMaxLog2M) {
@@ -125,12 +140,15 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         p->spectrum_bytes = (size_t)H * M * sizeof(float2);
         p->workspace_bytes = (size_t)g * per_pair;
     }
+    const size_t offErr = append_status_word(host);
     fftconv_status st = upload_tables(p, host);
     if (st != FFTCONV_OK) {
         delete p;
         return st;
     }
     const float2* base = (const float2*)p->d_tables;
+    p->d_err = (int*)(base + offErr);
+    if (p->umma) p->umma_b = base + offU;
     p->tw.wL = base + offL;
     if (p->path == fftc::PATH_MULTIPASS) {
         p->tw.wC = base + offC;
@@ -171,6 +189,7 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     std::vector<float2> host;
     size_t offR = 0, offC = 0;
     fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
+    const size_t offErr = append_status_word(host);
     const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
     int64_t g = (int64_t)(kGroupBytes / per_pair);
     // whole channels per group: a channel's pairs then run together and share
@@ -191,6 +210,7 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     }
     p->tw.wL = (const float2*)p->d_tables + offR;
     p->tw.wC = (const float2*)p->d_tables + offC;
+    p->d_err = (int*)((const float2*)p->d_tables + offErr);
     *out = p;
     return FFTCONV_OK;
 }
@@ -210,7 +230,7 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
     if (!p) return "none";
     switch (p->path) {
         case fftc::PATH_FUSED: return "fused";
-        case fftc::PATH_FUSED_TC: return "fused_tc";
+        case fftc::PATH_FUSED_TC: return p->umma ? "fused_umma" : "fused_tc";
         case fftc::PATH_MULTIPASS: return "multipass";
         case fftc::PATH_2D: return "2d";
     }
@@ -247,7 +267,7 @@ fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if (p->path == fftc::PATH_FUSED_TC)
-        e = fftc::launch_tc_fwd(*p, u, v, w, khat, D, y, s);
+        e = p->umma ? fftc::launch_umma_fwd(*p, u, v, w, khat, D, y, s) : fftc::launch_tc_fwd(*p, u, v, w, khat, D, y, s);
     else if (p->path == fftc::PATH_FUSED)
         e = fftc::launch_fused_fwd(*p, u, v, w, (const float2*)khat, D, y, s);
     else
@@ -272,6 +292,17 @@ fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, 
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     return cuda_status(
         fftc::launch_conv2d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream));
+}
+
+fftconv_status fftconv_device_status(fftconv_plan_t p, void* stream) {
+    if (!p || !p->d_err) return FFTCONV_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FFTCONV_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, p->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FFTCONV_ERR_CUDA;
+    if (word == 0) return FFTCONV_OK;
+    const int zero = 0;
+    if (cudaMemcpy(p->d_err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FFTCONV_ERR_CUDA;
+    return FFTCONV_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -54,6 +54,9 @@ struct fftconv_plan_s {
     void* d_tables = nullptr;
     fftc::Tables tw;
     fftc::TcTablePtrs tc;
+    bool umma = false;              // fused tensor-core path on tcgen05 (else mma.sync)
+    const void* umma_b = nullptr;   // tcgen05 path: B operand images of the DFT matrices
+    int* d_err = nullptr;           // device status word: nonzero after a timed-out device wait
     bool spectrum_ready = false;
     int device = 0;
 };
@@ -72,6 +75,13 @@ bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]);
 cudaError_t launch_tc_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s);
 cudaError_t launch_tc_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
                           const float* D, void* y, cudaStream_t s);
+
+// 1-D bf16 fused path on tcgen05 (2N in {4096, 8192}); shares the spectrum
+// layout and twiddle tables of the mma.sync path.
+bool umma_supported(int log2M);
+bool umma_bimages(int log2M, std::vector<float2>& out, size_t* off);
+cudaError_t launch_umma_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
+                            const float* D, void* y, cudaStream_t s);
 
 // 1-D fused path (one CTA per (pair of batch rows, channel)).
 cudaError_t launch_fused_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,

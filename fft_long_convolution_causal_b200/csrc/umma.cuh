@@ -1,0 +1,129 @@
+// umma.cuh -- thin wrappers over the sm_100a fifth-generation tensor-core
+// instructions (tcgen05: tensor-memory allocation, MMA, commit, TMEM loads and
+// stores) and the shared-memory mbarrier that MMA completion arrives on.
+//
+// Conventions used by the kernels (checked on B200 against exact integer
+// products before use):
+// * kind::f16 MMA, bf16 operands, fp32 accumulator, M = 128 (cta_group::1):
+//   D row m lives in TMEM lane m, column n in TMEM column (D address + n).
+// * A from TMEM: row m in lane m; 32-bit column c holds the K elements 2c (low
+//   half) and 2c + 1 (high half); one K = 16 step spans 8 columns.
+// * B from shared memory, K-major, no swizzle: core matrices of 8 rows (N) x
+//   16 bytes (8 K elements), the two K halves 128 bytes apart (LBO) and
+//   consecutive 8-row groups 256 bytes apart (SBO).
+// * tcgen05.ld / st with shape 16x256b: register i of thread (g = lane / 4,
+//   t = lane % 4) is TMEM lane g + 8 (i / 2), column 2 t + (i % 2) of an
+//   8-column block (the mma.sync m16n8 accumulator layout); .xR repeats the
+//   block over R consecutive 8-column blocks, registers 4r .. 4r + 3 for block r.
+#pragma once
+
+#include <stdint.h>
+
+namespace fftc {
+namespace um {
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// order tcgen05 operations against thread barriers
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// make generic-proxy shared-memory writes visible to the tensor core
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M x N
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// shared-memory matrix descriptor, K-major, no swizzle, LBO 128 B, SBO 256 B
+__device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(256u >> 4) << 32) |
+           (1ull << 46);
+}
+// byte offset of element (row n, k) of a K = 16 B tile in that layout
+__host__ __device__ constexpr uint32_t kmajor_off(int n, int k) {
+    return (uint32_t)((n / 8) * 256 + (k / 8) * 128 + (n % 8) * 16 + (k % 8) * 2);
+}
+
+// D[tmem] (+)= A[tmem] x B[smem]; issued by one thread
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// arrive on the mbarrier once every MMA issued so far by this thread is complete
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// One bounded probe: the thread may sleep up to ~20 us waiting for the phase.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity to complete: false when
+// the limit (2^16 probes, on the order of a second) is reached first; the
+// caller then reports a timeout instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity) {
+    for (int i = 0; i < (1 << 16); ++i)
+        if (mbar_try_wait(addr, parity)) return true;
+    return false;
+}
+
+// TMEM loads: the wait is tied to the destination registers so no use of them
+// is scheduled before it.
+__device__ __forceinline__ void ld16x256_x1(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void ld16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+template <int R>
+__device__ __forceinline__ void wait_ld(uint32_t (&r)[R]) {
+#pragma unroll
+    for (int i = 0; i < R; ++i) asm volatile("" : "+r"(r[i]));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < R; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+// one 16x16 bf16 A tile (re) and its partner (im) into 16 TMEM columns: the
+// A fragment registers (0: rows 0-7 k 0-7, 1: rows 8-15 k 0-7, 2: rows 0-7
+// k 8-15, 3: rows 8-15 k 8-15) go to columns so that column c holds
+// k = 2 (c / 2) + 8 (c % 2) + {0, 1}; the B images list K in that order.
+__device__ __forceinline__ void st_afrag2(uint32_t taddr, const uint32_t (&re)[4], const uint32_t (&im)[4]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(re[0]),
+        "r"(re[2]), "r"(re[1]), "r"(re[3]), "r"(im[0]), "r"(im[2]), "r"(im[1]), "r"(im[3])
+        : "memory");
+}
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// the input index k held at position kappa of a K = 16 step in TMEM column order
+__host__ __device__ constexpr int kperm(int kappa) { return 2 * (kappa / 4) + 8 * ((kappa / 2) % 2) + (kappa % 2); }
+
+}  // namespace um
+}  // namespace fftc

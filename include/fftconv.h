@@ -67,7 +67,7 @@ typedef enum {
     FFTCONV_ERR_NOT_READY = 3,   /* fftconv_fwd before any fftconv_kernel_spectrum on this plan   */
     FFTCONV_ERR_OOM = 4,         /* the plan's small tables could not be allocated               */
     FFTCONV_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed                  */
-    FFTCONV_ERR_TIMEOUT = 6      /* reserved: a bounded device-side wait gave up                 */
+    FFTCONV_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (fftconv_device_status)   */
 } fftconv_status;
 
 typedef enum {
@@ -111,7 +111,11 @@ FFTCONV_API size_t fftconv_spectrum_bytes(fftconv_plan_t plan);
  * need; 0 when the plan's path needs none (then workspace may be NULL). */
 FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
 
-/* Name of the execution path the plan chose ("fused", "multipass", "2d"). */
+/* Name of the execution path the plan chose: "fused" (fp32 on-chip),
+ * "fused_tc" (bf16 on-chip, 2N <= 32768, warp-level mma.sync tensor cores),
+ * "fused_umma" (the same on tcgen05 tensor cores, 2N = 4096 or 8192, chosen
+ * when the environment variable FFTCONV_UMMA=1 is set at plan creation),
+ * "multipass", "2d". */
 FFTCONV_API const char* fftconv_plan_path(fftconv_plan_t plan);
 
 /*
@@ -176,6 +180,16 @@ FFTCONV_API fftconv_status fftconv_fwd_static_workspace(fftconv_plan_t plan, con
 
 /* Size in bytes of the device array fftconv_fwd_static_workspace uses. */
 FFTCONV_API size_t fftconv_static_workspace_bytes(void);
+
+/*
+ * Device status of a plan: synchronises the stream, then reads and clears the
+ * plan's device status word.  Kernels that wait on the tensor cores bound
+ * every wait; a wait that gives up (the hardware never signalled) abandons
+ * the launch, leaves y incomplete and sets the word.  Returns FFTCONV_OK, or
+ * FFTCONV_ERR_TIMEOUT once after such a launch; FFTCONV_ERR_CUDA if the
+ * synchronisation or the read fails.  No counterpart on the pages.
+ */
+FFTCONV_API fftconv_status fftconv_device_status(fftconv_plan_t plan, void* stream);
 
 /* Human-readable name of a status code (static string). */
 FFTCONV_API const char* fftconv_status_string(fftconv_status status);

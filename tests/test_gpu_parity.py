@@ -93,6 +93,23 @@ def test_tensor_core_path(N, B, gated, with_D, L):
                  gate=wl.v if gated else None, scale=row_scale_1d(wl))
 
 
+@pytest.mark.parametrize("N", [2048, 4096])
+@pytest.mark.parametrize("B,gated,with_D,L", [(1, False, True, None), (5, True, True, None),
+                                             (2, False, False, 333), (3, True, False, None), (8, False, True, None)])
+def test_umma_path(N, B, gated, with_D, L, monkeypatch):
+    """bf16 fused kernel on tcgen05 (opt-in at plan creation): same cases as the mma.sync kernel."""
+    monkeypatch.setenv("FFTCONV_UMMA", "1")
+    wl = wlmod.make_1d(B, 5, N, dtype="bf16", gated=gated, seed=3 * N + B, with_D=with_D, L=L)
+    y, path = run_1d(wl)
+    assert path == "fused_umma"
+    assert_close(y, oracle_full(wl), "bf16", f"umma N={N} B={B} gated={gated} D={with_D} L={L}",
+                 gate=wl.v if gated else None, scale=row_scale_1d(wl))
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan(B, 5, N, "bf16", gated=gated)
+    assert plan.path == "fused_umma"
+    assert plan.device_status() == 0
+
+
 def test_tensor_core_large_dynamic_range():
     """Inputs far from unit scale: the bf16 path keeps fp32's exponent range."""
     wl = wlmod.make_1d(2, 2, 4096, dtype="bf16", seed=11)
