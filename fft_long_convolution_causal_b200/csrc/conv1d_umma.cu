@@ -27,6 +27,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <type_traits>
 #include <vector>
 
 #include "plan.h"
@@ -47,25 +48,23 @@ struct UShape {
     static constexpr int N3 = 2 * PH;                    // S1' accumulator columns (Re p | Im p)
     static constexpr int NT3 = PH / 8;
     static constexpr int T3 = P / 8;                     // step-3 tiles of 8 rows k_p
-    static constexpr int kCols = P <= 32 ? 128 : 256;    // TMEM columns per CTA
-    // S1: R1 tiles per MMA batch; A columns 16 KS1 per tile, then the accumulators
+    static constexpr int TS = T3 / 2;                    // step-3 tiles per slot (two slots)
+    static constexpr int kCols = 256;                    // TMEM columns per CTA
+    // S1: both 128-row tiles in one batch: A (16 KS1 columns each), then the accumulators
     static constexpr int kA1 = 16 * KS1;
-    static constexpr int R1 = 2 * (kA1 + N1) <= 96 ? 2 : 1;
-    static constexpr int kD1 = N1;                       // first S1 accumulator column (aligned to N1)
-    // step 3: R3 tiles per batch, A (16 columns) then the accumulators (32 columns)
-    static constexpr int R3 = (T3 < (kCols - 32) / 48) ? T3 : ((kCols - 32) / 48 >= 4 ? 4 : 2);
-    static constexpr int kD3 = ((16 * R3 + 31) / 32) * 32;
-    // S1': both 128-row tiles in one batch
+    static constexpr int kD1 = ((2 * kA1 + N1 - 1) / N1) * N1;
+    // step 3: slot s at column 128 s: A of tile u at 16 u, accumulator at 32 + 32 u
+    // S1': both tiles in one batch
     static constexpr int kA3 = 16 * KS3;
     static constexpr int kD3p = ((2 * kA3 + N3 - 1) / N3) * N3;
     // B images (bf16, K-major core-matrix layout), bytes
     static constexpr int kB1 = N1 * 32, kBF = 32 * 32, kB3 = N3 * 32;
-    static constexpr int kOffB1 = 0;                     // [ks][2]
+    static constexpr int kOffB1 = 0;                       // [ks][2]
     static constexpr int kOffBF = kOffB1 + KS1 * 2 * kB1;  // fwd 1, fwd 2, inv 1, inv 2
     static constexpr int kOffB3 = kOffBF + 4 * kBF;        // [ks][2]
     static constexpr int kBBytes = kOffB3 + KS3 * 2 * kB3;
-    static_assert(R1 * kA1 <= kD1 && kD1 + R1 * N1 <= kCols, "S1 columns");
-    static_assert(kD3 + 32 * R3 <= kCols && T3 % R3 == 0, "step-3 columns");
+    static_assert(kD1 + 2 * N1 <= kCols, "S1 columns");
+    static_assert(TS >= 1 && 32 + 32 * TS <= 128 && 16 * TS <= 32, "step-3 columns");
     static_assert(kD3p + 2 * N3 <= kCols, "S1' columns");
 };
 
@@ -74,15 +73,29 @@ struct USmem {
     static constexpr int kS = 2 * P * 512;                       // S planes (re, im), P rows of 256 q
     static constexpr int kX = P * 512;                           // staging planes of x (P/2 rows each)
     static constexpr int kW = GATED ? kX : 0;                    // staging planes of w
+    static constexpr int kStage = kX + kW;                       // one staging buffer (two, alternating by item)
     static constexpr int kB = UShape<P>::kBBytes;
-    static constexpr int kOffX = kS, kOffW = kS + kX, kOffB = kS + kX + kW;
+    static constexpr int kOffX = kS, kOffB = kS + 2 * kStage;
     static constexpr int kBytes = kOffB + kB;
 };
 
 __device__ __forceinline__ uint32_t lane_off(int lane0) { return (uint32_t)lane0 << 16; }
 
+// warps 0-7 compute (warp w: TMEM lane quarter w % 4, row half w / 4 of every 16-row group), warp 8 issues the MMAs
+constexpr int kUmmaCompute = 256;
+constexpr int kUmmaThreads = kUmmaCompute + 32;
+
+// Barriers in shared memory: afull[i] (8 arrivals: every compute warp has
+// stored its A rows for batch slot i), dfull[i] (one arrival: the MMAs of the
+// slot's batch are complete).  Slots 0 and 1 alternate in step 3; slot 2 is
+// S1 and S1'.
+struct UBars {
+    uint64_t afull[3];
+    uint64_t dfull[3];
+};
+
 template <int P, bool GATED>
-__global__ void __launch_bounds__(128, (P <= 32 && !GATED) ? 3 : 2)
+__global__ void __launch_bounds__(kUmmaThreads, 2)
 fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
                const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
                __nv_bfloat16* __restrict__ y, TcTables tb, const uint4* __restrict__ bimg, int* __restrict__ err,
@@ -90,39 +103,22 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
     using S = TcShape<P>;
     using U = UShape<P>;
     using SM = USmem<P, GATED>;
-    constexpr int NT = 128;
+    constexpr int NT = kUmmaCompute;  // compute threads
     constexpr int CH = S::N / 8;  // 16-byte chunks per row of u
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ __align__(8) UBars s_bar;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m8 = lane >> 3, r8 = lane & 7;
     const int npp = (B + 1) / 2;
     const int items = npp * H;
     const uint32_t sre = tc::smem_u32(smem), sim = sre + S::kPlaneBytes;
-    const uint32_t xre = sre + SM::kOffX, xim = xre + SM::kX / 2;
-    const uint32_t wre = sre + SM::kOffW, wim = wre + SM::kX / 2;
+    const uint32_t xbase = sre + SM::kOffX;  // staging buffer of the item k-th in this CTA: xbase + (k & 1) kStage
     const uint32_t bsm = sre + SM::kOffB;
-    const uint32_t mbar = tc::smem_u32(&s_mbar);
+    const uint32_t afull = tc::smem_u32(&s_bar.afull[0]), dfull = tc::smem_u32(&s_bar.dfull[0]);
 
-    auto stage_input = [&](int item) {
-        const int hh = item / npp, b0 = 2 * (item % npp);
-        const bool has1 = b0 + 1 < B;
-        const size_t r0 = ((size_t)b0 * H + hh) * S::N;
-        const size_t r1 = has1 ? ((size_t)(b0 + 1) * H + hh) * S::N : r0;
-        for (int i = tid; i < 2 * CH; i += NT) {
-            const int plane = i / CH, n0 = (i % CH) * 8;
-            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
-            const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing row
-            const size_t off = (plane ? r1 : r0) + n0;
-            cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
-            if (GATED) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
-        }
-        cp_async_commit();
-    };
-
-    // B images into shared memory, visible to the tensor core
-    for (int i = tid; i < U::kBBytes / 16; i += NT) {
+    // ---- set-up: B images into shared memory (visible to the tensor core), TMEM, barriers
+    for (int i = tid; i < U::kBBytes / 16; i += kUmmaThreads) {
         const uint4 val = __ldg(&bimg[i]);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(bsm + 16u * i), "r"(val.x), "r"(val.y),
                      "r"(val.z), "r"(val.w)
@@ -133,62 +129,151 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
         um::tmem_alloc(tc::smem_u32(&s_tmem), U::kCols);
         um::tmem_relinquish();
     }
-    if (tid == 0) um::mbar_init(mbar, 1);
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            um::mbar_init(afull + 8 * i, kUmmaCompute / 32);
+            um::mbar_init(dfull + 8 * i, 1);
+        }
+    }
     um::fence_before();
     __syncthreads();
     um::fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t tl = tmem + lane_off(32 * warp);  // this warp's TMEM lane quarter
 
-    uint2 w256[4];
+    if (warp == kUmmaCompute / 32) {
+        // ================= MMA issuer: one lane walks the same batch sequence as the compute warps
+        if (lane == 0) {
+            const uint32_t id1 = um::idesc_bf16(128, U::N1), id16 = um::idesc_bf16(128, 32),
+                           id3 = um::idesc_bf16(128, U::N3);
+            uint32_t pa[3] = {0u, 0u, 0u};
+            auto wait_a = [&](int i) {
+                const bool ok = um::mbar_wait(afull + 8 * i, pa[i]);
+                pa[i] ^= 1u;
+                um::fence_after();
+                return ok;
+            };
+            bool ok = true;
+            for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+                // S1: rows q, K = p < P/2, both tiles
+                if (!(ok = wait_a(2))) break;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
-
-    const uint32_t id1 = um::idesc_bf16(128, U::N1), id16 = um::idesc_bf16(128, 32), id3 = um::idesc_bf16(128, U::N3);
-    uint32_t phase = 0;
-    bool dead = false;
-    // All threads: finish TMEM stores, then one thread issues the batch and commits.
-    auto issue = [&](auto&& body) {
-        um::wait_st();
-        um::fence_before();
-        __syncthreads();
-        if (tid == 0) {
+                for (int t = 0; t < 2; ++t) {
+                    const uint32_t d = tmem + U::kD1 + t * U::N1, a = tmem + t * U::kA1;
+#pragma unroll
+                    for (int ks = 0; ks < U::KS1; ++ks) {
+                        um::mma_ts(d, a + 16 * ks, um::sdesc_kmajor(bsm + U::kOffB1 + (2 * ks) * U::kB1), id1, ks > 0);
+                        um::mma_ts(d, a + 16 * ks + 8, um::sdesc_kmajor(bsm + U::kOffB1 + (2 * ks + 1) * U::kB1), id1, 1);
+                    }
+                }
+                um::mma_commit(dfull + 16);
+                // step 3: four stages, the two slots alternating
+#pragma unroll 1
+                for (int st = 0; st < 4 && ok; ++st)
+#pragma unroll
+                    for (int sl = 0; sl < 2; ++sl) {
+                        if (!(ok = wait_a(sl))) break;
+                        const uint32_t bf = bsm + U::kOffBF + (st < 2 ? 0 : 2) * U::kBF;
+#pragma unroll
+                        for (int uu = 0; uu < U::TS; ++uu) {
+                            const uint32_t d = tmem + 128 * sl + 32 + 32 * uu, a = tmem + 128 * sl + 16 * uu;
+                            um::mma_ts(d, a, um::sdesc_kmajor(bf), id16, 0);
+                            um::mma_ts(d, a + 8, um::sdesc_kmajor(bf + U::kBF), id16, 1);
+                        }
+                        um::mma_commit(dfull + 8 * sl);
+                    }
+                if (!ok) break;
+                // S1': rows q, K = k_p, N = p < P/2, both tiles
+                if (!(ok = wait_a(2))) break;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint32_t d = tmem + U::kD3p + t * U::N3, a = tmem + t * U::kA3;
+#pragma unroll
+                    for (int ks = 0; ks < U::KS3; ++ks) {
+                        um::mma_ts(d, a + 16 * ks, um::sdesc_kmajor(bsm + U::kOffB3 + (2 * ks) * U::kB3), id3, ks > 0);
+                        um::mma_ts(d, a + 16 * ks + 8, um::sdesc_kmajor(bsm + U::kOffB3 + (2 * ks + 1) * U::kB3), id3, 1);
+                    }
+                }
+                um::mma_commit(dfull + 16);
+            }
+            if (!ok) atomicExch(err, 1);
+        }
+    } else {
+        // ================= compute warps: TMEM lanes 32 q + 16 r .. + 15 of every 128-lane tile
+        const int q = warp & 3, r = warp >> 2;
+        const uint32_t tl = tmem + lane_off(32 * q + 16 * r);
+        uint2 w256[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+        uint32_t pd[3] = {0u, 0u, 0u};
+        bool dead = false;
+        // this warp's A rows of slot i are in TMEM: tell the issuer
+        auto signal = [&](int i) {
+            um::wait_st();
+            um::fence_before();
+            __syncwarp();
+            if (lane == 0) um::mbar_arrive(afull + 8 * i);
+        };
+        // wait for slot i's products (bounded); a timeout marks the CTA dead at the next named barrier
+        auto wait_d = [&](int i) {
+            const bool ok = um::mbar_wait(dfull + 8 * i, pd[i]);
+            pd[i] ^= 1u;
             um::fence_after();
-            body();
-            um::mma_commit(mbar);
-        }
-        // reconverge warp 0 before any of its lanes waits on the barrier the
-        // issuing lane has yet to arm
-        __syncwarp();
-    };
-    // All threads: wait for the batch (bounded); a timeout marks the CTA dead.
-    auto await = [&]() {
-        const bool ok = um::mbar_wait(mbar, phase);
-        phase ^= 1u;
-        um::fence_after();
-        if (__syncthreads_or(!ok)) {
-            dead = true;
-            if (tid == 0) atomicExch(err, 1);
-        }
-    };
+            dead |= !ok;
+        };
+        auto stage_input = [&](int item, int buf) {
+            const uint32_t xre = xbase + buf * SM::kStage, xim = xre + SM::kX / 2;
+            const uint32_t wre = xre + SM::kX, wim = wre + SM::kX / 2;
+            const int hh = item / npp, b0 = 2 * (item % npp);
+            const bool has1 = b0 + 1 < B;
+            const size_t r0 = ((size_t)b0 * H + hh) * S::N;
+            const size_t r1 = has1 ? ((size_t)(b0 + 1) * H + hh) * S::N : r0;
+            for (int i = tid; i < 2 * CH; i += NT) {
+                const int plane = i / CH, n0 = (i % CH) * 8;
+                const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+                const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing row
+                const size_t off = (plane ? r1 : r0) + n0;
+                cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
+                if (GATED) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
+            }
+            cp_async_commit();
+        };
+        const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);  // step-3 ldmatrix / stmatrix chunk
 
-    if ((int)blockIdx.x < items) stage_input(blockIdx.x);
+        if ((int)blockIdx.x < items) stage_input(blockIdx.x, 0);
+        int k = 0;  // items done by this CTA
+        for (int item = blockIdx.x; item < items; item += gridDim.x, ++k) {
+            const int h = item / npp, b0 = 2 * (item % npp);
+            const bool has1 = b0 + 1 < B;
+            const size_t row0 = ((size_t)b0 * H + h) * S::N;
+            const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
+            // the next item's rows go to the other buffer (free: its last reader was the
+            // previous item's S1, and the barrier below the previous S1 has passed)
+            if (item + (int)gridDim.x < items) {
+                stage_input(item + gridDim.x, (k + 1) & 1);
+                asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+            } else {
+                cp_async_wait_all();
+            }
+            if (um::bar_or(1, NT, dead)) break;
+            const uint32_t xre = xbase + (k & 1) * SM::kStage, xim = xre + SM::kX / 2;
+            const uint32_t wre = xre + SM::kX, wim = wre + SM::kX / 2;
 
-    for (int item = blockIdx.x; item < items && !dead; item += gridDim.x) {
-        const int h = item / npp, b0 = 2 * (item % npp);
-        const bool has1 = b0 + 1 < B;
-        const size_t row0 = ((size_t)b0 * H + h) * S::N;
-        const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
-        cp_async_wait_all();
-        __syncthreads();
-
-        // ---------------- S1: outer DFT over p < P/2, rows q, R1 tiles of 128 q per batch
-        for (int t0 = 0; t0 < 2 && !dead; t0 += U::R1) {
+            // ---------------- S1: A = x rows q of both tiles (K = p < P/2)
+            uint2 tw[2][U::NT1][2];  // W_M^{q k_p} of this warp's rows, fetched ahead of use
 #pragma unroll
-            for (int uu = 0; uu < U::R1; ++uu)
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int qt = 8 * (t0 + uu) + 2 * warp + r;
+                for (int j = 0; j < U::NT1; ++j)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int qt = 8 * t + 2 * q + r;
+                        tw[t][j][hh] = __ldg(&tb.tw1[((qt * U::NT1 + j) * 2 + hh) * 32 + lane]);
+                    }
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+                {
+                    const int qt = 8 * t + 2 * q + r;
 #pragma unroll
                     for (int ks = 0; ks < U::KS1; ++ks) {
                         uint32_t ar[4], ai[4];
@@ -207,254 +292,233 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
                             }
                         }
                         if (16 * ks + 8 >= P / 2) ar[2] = ar[3] = ai[2] = ai[3] = 0u;
-                        um::st_afrag2(tl + lane_off(16 * r) + uu * U::kA1 + 16 * ks, ar, ai);
+                        um::st_afrag2(tl + t * U::kA1 + 16 * ks, ar, ai);
                     }
                 }
-            issue([&] {
-#pragma unroll
-                for (int uu = 0; uu < U::R1; ++uu) {
-                    const uint32_t d = tmem + U::kD1 + uu * U::N1, a = tmem + uu * U::kA1;
-#pragma unroll
-                    for (int ks = 0; ks < U::KS1; ++ks) {
-                        um::mma_ts(d, a + 16 * ks, um::sdesc_kmajor(bsm + U::kOffB1 + (2 * ks) * U::kB1), id1, ks > 0);
-                        um::mma_ts(d, a + 16 * ks + 8, um::sdesc_kmajor(bsm + U::kOffB1 + (2 * ks + 1) * U::kB1), id1, 1);
-                    }
-                }
-            });
-            await();
-            if (dead) break;
+            signal(2);
+            wait_d(2);
             // x W_M^{q k_p}, stored transposed into S[k_p][q]
 #pragma unroll
-            for (int uu = 0; uu < U::R1; ++uu)
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int qt = 8 * (t0 + uu) + 2 * warp + r;
-                    const uint32_t dl = tl + lane_off(16 * r) + U::kD1 + uu * U::N1;
+            for (int t = 0; t < 2; ++t) {
+                uint32_t yv[8 * U::NT1];  // Re blocks then Im blocks
+                {
+                    const uint32_t dl = tl + U::kD1 + t * U::N1;
+                    um::ld16x256<U::NT1>(dl, yv);
+                    um::ld16x256<U::NT1>(dl + P, yv + 4 * U::NT1);
+                }
+                um::wait_ld<8 * U::NT1>(yv);
+                {
+                    const int qt = 8 * t + 2 * q + r;
 #pragma unroll
                     for (int j = 0; j < U::NT1; ++j) {
-                        uint32_t yr[4], yi[4];
-                        um::ld16x256_x1(dl + 8 * j, yr);
-                        um::ld16x256_x1(dl + P + 8 * j, yi);
-                        const uint2 tw0 = __ldg(&tb.tw1[((qt * U::NT1 + j) * 2 + 0) * 32 + lane]);
-                        const uint2 tw1 = __ldg(&tb.tw1[((qt * U::NT1 + j) * 2 + 1) * 32 + lane]);
-                        um::wait_ld(yr);
-                        um::wait_ld(yi);
+                        const uint32_t* yr = yv + 4 * j;
+                        const uint32_t* yi = yr + 4 * U::NT1;
                         uint32_t pr[2] = {pack2(__uint_as_float(yr[0]), __uint_as_float(yr[1])),
                                           pack2(__uint_as_float(yr[2]), __uint_as_float(yr[3]))};
                         uint32_t pi[2] = {pack2(__uint_as_float(yi[0]), __uint_as_float(yi[1])),
                                           pack2(__uint_as_float(yi[2]), __uint_as_float(yi[3]))};
-                        twiddle2<true>(pr[0], pi[0], tw0);
-                        twiddle2<true>(pr[1], pi[1], tw1);
+                        twiddle2<true>(pr[0], pi[0], tw[t][j][0]);
+                        twiddle2<true>(pr[1], pi[1], tw[t][j][1]);
                         const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
                         stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
                     }
                 }
-        }
-        if (dead) break;
-        __syncthreads();
-        // the staging planes are free: fetch the next item while this one runs
-        if (item + (int)gridDim.x < items) stage_input(item + gridDim.x);
+            }
+            if (um::bar_or(1, NT, dead)) break;  // S complete
 
-        // ---------------- step 3: inner 256-point DFT, product with Khat, inverse
-        {
+            // ---------------- step 3: inner 256-point DFT, product with Khat, inverse
             const float dmf = D ? D[h] * (1.0f / S::M) : 0.f;
             const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
             const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
-            const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
-            for (int T0 = 0; T0 < U::T3 && !dead; T0 += U::R3) {
-                // stage-0 A tiles: rows b, K = a, from S rows k_p
+            // stage-0 A tiles of both slots: rows b, K = a, from S rows k_p
 #pragma unroll
-                for (int uu = 0; uu < U::R3; ++uu)
+            for (int sl = 0; sl < 2; ++sl) {
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int kp = 8 * (T0 + uu) + 2 * warp + r;
+                for (int uu = 0; uu < U::TS; ++uu)
+                    {
+                        const int kp = 8 * (sl * U::TS + uu) + 2 * q + r;
                         uint32_t xr[4], xi[4];
                         ldsm_x4_t(xr, plane_addr(sre, kp, ichunk));
                         ldsm_x4_t(xi, plane_addr(sim, kp, ichunk));
-                        um::st_afrag2(tl + lane_off(16 * r) + 16 * uu, xr, xi);
+                        um::st_afrag2(tl + 128 * sl + 16 * uu, xr, xi);
                     }
-#pragma unroll 1
-                for (int s = 0; s < 4 && !dead; ++s) {
-                    const uint32_t bf1 = bsm + U::kOffBF + (s < 2 ? 0 : 2) * U::kBF;
-                    issue([&] {
+                signal(sl);
+            }
+            // spectrum words of this warp's rows (both slots), fetched two epilogues ahead of use
+            uint4 kc0[2][U::TS], kc1[2][U::TS];
 #pragma unroll
-                        for (int uu = 0; uu < U::R3; ++uu) {
-                            const uint32_t d = tmem + U::kD3 + 32 * uu, a = tmem + 16 * uu;
-                            um::mma_ts(d, a, um::sdesc_kmajor(bf1), id16, 0);
-                            um::mma_ts(d, a + 8, um::sdesc_kmajor(bf1 + U::kBF), id16, 1);
-                        }
-                    });
-                    // fetch what this stage's epilogue needs while the products run
-                    uint4 kc0[U::R3][2], kc1[U::R3][2];
-                    uint2 tc3[U::R3][2][4];
-                    if (s == 1) {
+            for (int sl = 0; sl < 2; ++sl)
 #pragma unroll
-                        for (int uu = 0; uu < U::R3; ++uu)
+                for (int uu = 0; uu < U::TS; ++uu) {
+                    const int kp = 8 * (sl * U::TS + uu) + 2 * q + r;
+                    kc0[sl][uu] = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
+                    kc1[sl][uu] = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
+                }
+            uint2 tc3[2][U::TS][4];  // W_M^{-q k_p}, fetched at the start of stage 2
+            auto epilogue = [&](auto st_c, auto sl_c) {
+                constexpr int ST = decltype(st_c)::value;
+                constexpr int sl = decltype(sl_c)::value;
+                if (ST == 2 && sl == 0) {
 #pragma unroll
-                            for (int r = 0; r < 2; ++r) {
-                                const int kp = 8 * (T0 + uu) + 2 * warp + r;
-                                kc0[uu][r] = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
-                                kc1[uu][r] = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
-                            }
-                    }
-                    if (s == 3) {
+                    for (int s2 = 0; s2 < 2; ++s2)
 #pragma unroll
-                        for (int uu = 0; uu < U::R3; ++uu)
+                        for (int uu = 0; uu < U::TS; ++uu) {
+                            const int kp = 8 * (s2 * U::TS + uu) + 2 * q + r;
 #pragma unroll
-                            for (int r = 0; r < 2; ++r) {
-                                const int kp = 8 * (T0 + uu) + 2 * warp + r;
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    tc3[uu][r][i] = __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]);
-                            }
-                    }
-                    await();
-                    if (dead) break;
-#pragma unroll
-                    for (int uu = 0; uu < U::R3; ++uu)
-#pragma unroll
-                        for (int r = 0; r < 2; ++r) {
-                            const uint32_t dl = tl + lane_off(16 * r) + U::kD3 + 32 * uu;
-                            const uint32_t al = tl + lane_off(16 * r) + 16 * uu;
-                            uint32_t acc[16];
-                            um::ld16x256_x4(dl, acc);
-                            um::wait_ld(acc);
-                            float acr[2][4], aci[2][4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                acr[0][e] = __uint_as_float(acc[e]);
-                                acr[1][e] = __uint_as_float(acc[4 + e]);
-                                aci[0][e] = __uint_as_float(acc[8 + e]);
-                                aci[1][e] = __uint_as_float(acc[12 + e]);
-                            }
-                            uint32_t xr[4], xi[4];
-                            if (s == 0) {
-                                // [b][c]: x W_256^{b c}, transpose -> [c][b]
-                                uint32_t tr[4], ti[4];
-                                pack_tile(tr, acr);
-                                pack_tile(ti, aci);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
-                                transpose_tile(xr, tr);
-                                transpose_tile(xi, ti);
-                                um::st_afrag2(al, xr, xi);
-                            } else if (s == 1) {
-                                // [c][d]: spectrum at k = k_p + P (c + 16 d); x (Khat + D/M)
-                                pack_tile(xr, acr);
-                                pack_tile(xi, aci);
-                                const uint32_t kre[4] = {kc0[uu][r].x, kc0[uu][r].z, kc1[uu][r].x, kc1[uu][r].z};
-                                const uint32_t kim[4] = {kc0[uu][r].y, kc0[uu][r].w, kc1[uu][r].y, kc1[uu][r].w};
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const __nv_bfloat162 zr = as_b2(xr[i]), zi = as_b2(xi[i]);
-                                    const __nv_bfloat162 kr = __hadd2(as_b2(kre[i]), dm2), ki = as_b2(kim[i]);
-                                    xr[i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
-                                    xi[i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
-                                }
-                                um::st_afrag2(al, xr, xi);
-                            } else if (s == 2) {
-                                // [c][b]: transpose -> [b][c], x W_256^{-b c}
-                                uint32_t gr[4], gi[4];
-                                pack_tile(gr, acr);
-                                pack_tile(gi, aci);
-                                transpose_tile(xr, gr);
-                                transpose_tile(xi, gi);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) twiddle2<false>(xr[i], xi[i], w256[i]);
-                                um::st_afrag2(al, xr, xi);
-                            } else {
-                                // [b][a]: x W_M^{-q k_p}, back to S row k_p
-                                const int kp = 8 * (T0 + uu) + 2 * warp + r;
-                                pack_tile(xr, acr);
-                                pack_tile(xi, aci);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) twiddle2<false>(xr[i], xi[i], tc3[uu][r][i]);
-                                stsm_x4_t(plane_addr(sre, kp, ichunk), xr[0], xr[1], xr[2], xr[3]);
-                                stsm_x4_t(plane_addr(sim, kp, ichunk), xi[0], xi[1], xi[2], xi[3]);
-                            }
+                            for (int i = 0; i < 4; ++i)
+                                tc3[s2][uu][i] = __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]);
                         }
                 }
-            }
-        }
-        if (dead) break;
-        __syncthreads();
+                wait_d(sl);
+                uint32_t accs[U::TS * 16];
+#pragma unroll
+                for (int uu = 0; uu < U::TS; ++uu)
+                        um::ld16x256<4>(tl + 128 * sl + 32 + 32 * uu, accs + uu * 16);
+                um::wait_ld<U::TS * 16>(accs);
+#pragma unroll
+                for (int uu = 0; uu < U::TS; ++uu)
+                    {
+                        const uint32_t al = tl + 128 * sl + 16 * uu;
+                        const uint32_t* acc = accs + uu * 16;
+                        float acr[2][4], aci[2][4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            acr[0][e] = __uint_as_float(acc[e]);
+                            acr[1][e] = __uint_as_float(acc[4 + e]);
+                            aci[0][e] = __uint_as_float(acc[8 + e]);
+                            aci[1][e] = __uint_as_float(acc[12 + e]);
+                        }
+                        uint32_t xr[4], xi[4];
+                        if (ST == 0) {
+                            // [b][c]: x W_256^{b c}, transpose -> [c][b]
+                            uint32_t tr[4], ti[4];
+                            pack_tile(tr, acr);
+                            pack_tile(ti, aci);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+                            transpose_tile(xr, tr);
+                            transpose_tile(xi, ti);
+                            um::st_afrag2(al, xr, xi);
+                        } else if (ST == 1) {
+                            // [c][d]: spectrum at k = k_p + P (c + 16 d); x (Khat + D/M)
+                            pack_tile(xr, acr);
+                            pack_tile(xi, aci);
+                            const uint32_t kre[4] = {kc0[sl][uu].x, kc0[sl][uu].z, kc1[sl][uu].x, kc1[sl][uu].z};
+                            const uint32_t kim[4] = {kc0[sl][uu].y, kc0[sl][uu].w, kc1[sl][uu].y, kc1[sl][uu].w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const __nv_bfloat162 zr = as_b2(xr[i]), zi = as_b2(xi[i]);
+                                const __nv_bfloat162 kr = __hadd2(as_b2(kre[i]), dm2), ki = as_b2(kim[i]);
+                                xr[i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
+                                xi[i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
+                            }
+                            um::st_afrag2(al, xr, xi);
+                        } else if (ST == 2) {
+                            // [c][b]: transpose -> [b][c], x W_256^{-b c}
+                            uint32_t gr[4], gi[4];
+                            pack_tile(gr, acr);
+                            pack_tile(gi, aci);
+                            transpose_tile(xr, gr);
+                            transpose_tile(xi, gi);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) twiddle2<false>(xr[i], xi[i], w256[i]);
+                            um::st_afrag2(al, xr, xi);
+                        } else {
+                            // [b][a]: x W_M^{-q k_p}, back to S row k_p
+                            const int kp = 8 * (sl * U::TS + uu) + 2 * q + r;
+                            pack_tile(xr, acr);
+                            pack_tile(xi, aci);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) twiddle2<false>(xr[i], xi[i], tc3[sl][uu][i]);
+                            stsm_x4_t(plane_addr(sre, kp, ichunk), xr[0], xr[1], xr[2], xr[3]);
+                            stsm_x4_t(plane_addr(sim, kp, ichunk), xi[0], xi[1], xi[2], xi[3]);
+                        }
+                    }
+                if (ST < 3) signal(sl);
+            };
+            using I0 = std::integral_constant<int, 0>;
+            using I1 = std::integral_constant<int, 1>;
+            using I2 = std::integral_constant<int, 2>;
+            using I3 = std::integral_constant<int, 3>;
+            epilogue(I0{}, I0{});
+            epilogue(I0{}, I1{});
+            epilogue(I1{}, I0{});
+            epilogue(I1{}, I1{});
+            epilogue(I2{}, I0{});
+            epilogue(I2{}, I1{});
+            epilogue(I3{}, I0{});
+            epilogue(I3{}, I1{});
+            if (um::bar_or(1, NT, dead)) break;  // S complete
 
-        // ---------------- S1': inverse outer DFT over k_p, outputs p < P/2 into S rows p
+            // ---------------- S1': inverse outer DFT over k_p, outputs p < P/2 into S rows p
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < 2; ++t)
+                {
+                    const int qt = 8 * t + 2 * q + r;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int qt = 8 * t + 2 * warp + r;
-#pragma unroll
-                for (int ks = 0; ks < U::KS3; ++ks) {
-                    uint32_t ar[4], ai[4];
-                    const uint32_t krow = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
-                    ldsm_x4_t(ar, plane_addr(sre, krow, chunk));
-                    ldsm_x4_t(ai, plane_addr(sim, krow, chunk));
-                    um::st_afrag2(tl + lane_off(16 * r) + t * U::kA3 + 16 * ks, ar, ai);
+                    for (int ks = 0; ks < U::KS3; ++ks) {
+                        uint32_t ar[4], ai[4];
+                        const uint32_t krow = 16 * ks + r8 + 8 * (m8 >> 1), chunk = 2 * qt + (m8 & 1);
+                        ldsm_x4_t(ar, plane_addr(sre, krow, chunk));
+                        ldsm_x4_t(ai, plane_addr(sim, krow, chunk));
+                        um::st_afrag2(tl + t * U::kA3 + 16 * ks, ar, ai);
+                    }
                 }
-            }
-        issue([&] {
+            signal(2);
+            // every warp has read its S1' operands: S rows p may be rewritten below
+            if (um::bar_or(1, NT, dead)) break;
+            wait_d(2);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const uint32_t d = tmem + U::kD3p + t * U::N3, a = tmem + t * U::kA3;
+                uint32_t zv[8 * U::NT3];  // Re blocks then Im blocks
+                {
+                    const uint32_t dl = tl + U::kD3p + t * U::N3;
+                    um::ld16x256<U::NT3>(dl, zv);
+                    um::ld16x256<U::NT3>(dl + U::PH, zv + 4 * U::NT3);
+                }
+                um::wait_ld<8 * U::NT3>(zv);
+                {
+                    const int qt = 8 * t + 2 * q + r;
 #pragma unroll
-                for (int ks = 0; ks < U::KS3; ++ks) {
-                    um::mma_ts(d, a + 16 * ks, um::sdesc_kmajor(bsm + U::kOffB3 + (2 * ks) * U::kB3), id3, ks > 0);
-                    um::mma_ts(d, a + 16 * ks + 8, um::sdesc_kmajor(bsm + U::kOffB3 + (2 * ks + 1) * U::kB3), id3, 1);
+                    for (int j = 0; j < U::NT3; ++j) {
+                        const uint32_t* yr = zv + 4 * j;
+                        const uint32_t* yi = yr + 4 * U::NT3;
+                        const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+                        stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk),
+                                  pack2(__uint_as_float(yr[0]), __uint_as_float(yr[1])),
+                                  pack2(__uint_as_float(yr[2]), __uint_as_float(yr[3])),
+                                  pack2(__uint_as_float(yi[0]), __uint_as_float(yi[1])),
+                                  pack2(__uint_as_float(yi[2]), __uint_as_float(yi[3])));
+                    }
                 }
             }
-        });
-        await();
-        if (dead) break;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int qt = 8 * t + 2 * warp + r;
-                const uint32_t dl = tl + lane_off(16 * r) + U::kD3p + t * U::N3;
-#pragma unroll
-                for (int j = 0; j < U::NT3; ++j) {
-                    uint32_t yr[4], yi[4];
-                    um::ld16x256_x1(dl + 8 * j, yr);
-                    um::ld16x256_x1(dl + U::PH + 8 * j, yi);
-                    um::wait_ld(yr);
-                    um::wait_ld(yi);
-                    const uint32_t prow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
-                    stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, prow, chunk),
-                              pack2(__uint_as_float(yr[0]), __uint_as_float(yr[1])),
-                              pack2(__uint_as_float(yr[2]), __uint_as_float(yr[3])),
-                              pack2(__uint_as_float(yi[0]), __uint_as_float(yi[1])),
-                              pack2(__uint_as_float(yi[2]), __uint_as_float(yi[3])));
-                }
-            }
-        __syncthreads();
+            if (um::bar_or(1, NT, dead)) break;  // output rows complete
 
-        // ---------------- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
-        for (int i = tid; i < 2 * CH; i += NT) {
-            const int plane = i / CH, n0 = (i % CH) * 8;
-            if (plane == 1 && !has1) continue;
-            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
-            uint4 val;
-            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
-                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                         : "r"(plane_addr(plane ? sim : sre, p, chunk)));
-            const size_t off = (plane ? row1 : row0) + n0;
-            if (GATED) {
-                const uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + off));
-                val.x = as_u(__hmul2(as_b2(val.x), as_b2(vv.x)));
-                val.y = as_u(__hmul2(as_b2(val.y), as_b2(vv.y)));
-                val.z = as_u(__hmul2(as_b2(val.z), as_b2(vv.z)));
-                val.w = as_u(__hmul2(as_b2(val.w), as_b2(vv.w)));
+            // ---------------- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
+            for (int i = tid; i < 2 * CH; i += NT) {
+                const int plane = i / CH, n0 = (i % CH) * 8;
+                if (plane == 1 && !has1) continue;
+                const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+                uint4 val;
+                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                             : "r"(plane_addr(plane ? sim : sre, p, chunk)));
+                const size_t off = (plane ? row1 : row0) + n0;
+                if (GATED) {
+                    const uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + off));
+                    val.x = as_u(__hmul2(as_b2(val.x), as_b2(vv.x)));
+                    val.y = as_u(__hmul2(as_b2(val.y), as_b2(vv.y)));
+                    val.z = as_u(__hmul2(as_b2(val.z), as_b2(vv.z)));
+                    val.w = as_u(__hmul2(as_b2(val.w), as_b2(vv.w)));
+                }
+                *reinterpret_cast<uint4*>(y + off) = val;
             }
-            *reinterpret_cast<uint4*>(y + off) = val;
+            // the next iteration's wait + barrier orders these reads before S is rewritten
         }
-        // the next iteration's wait + barrier orders these reads before S is rewritten
+        cp_async_wait_all();
+        if (dead && tid == 0) atomicExch(err, 1);
     }
-    cp_async_wait_all();
-    // a timed-out batch may still be running (its phase is the one before
-    // `phase`): wait for it, bounded, before freeing TMEM
-    if (dead) um::mbar_wait(mbar, phase ^ 1u);
+    // every wait above is bounded; in normal operation all MMAs are complete here
     um::fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -578,7 +642,7 @@ static cudaError_t umma_fwd_go(const fftconv_plan_s& p, const void* u, const voi
         cudaFuncAttributes fa;
         int per_sm = 512 / tc::UShape<P>::kCols;
         if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess) {
-            const int regs = ((fa.numRegs + 7) / 8) * 8 * 128;
+            const int regs = ((fa.numRegs + 7) / 8) * 8 * tc::kUmmaThreads;
             const int by_regs = regs > 0 ? regs_sm / regs : 1;
             const int by_smem = smem_sm / (int)(smem + fa.sharedSizeBytes + 1024);
             per_sm = per_sm < by_regs ? per_sm : by_regs;
@@ -589,7 +653,7 @@ static cudaError_t umma_fwd_go(const fftconv_plan_s& p, const void* u, const voi
     }
     const int items = ((p.B + 1) / 2) * p.H;
     dim3 grid(items < resident ? items : resident);
-    kern<<<grid, 128, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
+    kern<<<grid, tc::kUmmaThreads, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
                                  (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, (const uint4*)p.umma_b, p.d_err,
                                  p.B, p.H);
     return cudaGetLastError();
