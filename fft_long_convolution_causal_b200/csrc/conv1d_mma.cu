@@ -242,13 +242,14 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     const int npp = (B + 1) / 2;
     const int items = npp * H;
     const uint32_t sre = smem_u32(smem), sim = sre + S::kPlaneBytes;
-    const uint32_t xre = sre + SM::kS, xim = xre + SM::kX / 2;
+    const uint32_t xre0 = sre + SM::kS;  // staging buffer 0 (buffer 1 follows when kNBuf = 2, ungated only)
     // w planes: separate, or S rows P/2 .. P-1 (plane_addr(w, p) == plane_addr(S, p + P/2))
-    const uint32_t wre = SM::kWInS ? sre + (P / 2) * 512u : xre + SM::kX;
-    const uint32_t wim = SM::kWInS ? sim + (P / 2) * 512u : xre + SM::kX + SM::kX / 2;
+    const uint32_t wre = SM::kWInS ? sre + (P / 2) * 512u : xre0 + SM::kX;
+    const uint32_t wim = SM::kWInS ? sim + (P / 2) * 512u : xre0 + SM::kX + SM::kX / 2;
 
-    // cp.async the input rows of one item: which = 1 (u), 2 (w), 3 (both)
-    auto stage_input = [&](int item, int which) {
+    // cp.async the input rows of one item into staging buffer buf: which = 1 (u), 2 (w), 3 (both)
+    auto stage_input = [&](int item, int which, int buf) {
+        const uint32_t xre = xre0 + buf * SM::kX, xim = xre + SM::kX / 2;
         const int hh = item / npp, b0 = 2 * (item % npp);
         const bool has1 = b0 + 1 < B;
         const size_t r0 = ((size_t)b0 * H + hh) * S::N;
@@ -295,21 +296,30 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
                         __ldg(&tb.fpi[((ks * S::NT3 + j) * 3 + part) * 32 + lane]);
     }
 
-    if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3);
+    if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3, 0);
 
-    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    int k = 0;  // items done by this CTA
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++k) {
         const int h = item / npp, b0 = 2 * (item % npp);
         const bool has1 = b0 + 1 < B;
         const size_t row0 = ((size_t)b0 * H + h) * S::N;
         const size_t row1 = ((size_t)(b0 + 1) * H + h) * S::N;
-        cp_async_wait_all();
+        const int buf = SM::kNBuf == 2 ? (k & 1) : 0;
+        if (SM::kNBuf == 2 && item + (int)gridDim.x < items) {
+            // the other buffer was last read by the previous item's step 1 (a barrier ago)
+            stage_input(item + gridDim.x, 3, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            cp_async_wait_all();
+        }
         __syncthreads();
+        const uint32_t xre = xre0 + buf * SM::kX, xim = xre + SM::kX / 2;
 
         // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
         outer_step1<P, NW, GATED, PRE1, IP>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb);
         __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
-        if (item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3);
+        if (SM::kNBuf == 1 && item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3, 0);
 
         // ---- step 3: inner 256-point DFT, product with Khat, inverse; two rows k_p per iteration
         {
@@ -384,7 +394,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         __syncthreads();
 
         // S rows P/2 .. P-1 are free again: fetch the next item's w into them
-        if (GATED && SM::kWInS && item + (int)gridDim.x < items) stage_input(item + gridDim.x, 2);
+        if (GATED && SM::kWInS && item + (int)gridDim.x < items) stage_input(item + gridDim.x, 2, 0);
 
         // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
         for (int i = tid; i < 2 * CH; i += NT) {

@@ -184,7 +184,10 @@ struct TcSmem {
     // The gate input w has its own staging planes, except for the largest
     // transform, where it is staged in S's upper rows (free until step 1).
     static constexpr bool kWInS = P >= 128;
-    static constexpr int kBytes = kS + kX * ((GATED && !kWInS) ? 2 : 1);
+    // Ungated transforms up to 2N = 8192 keep two staging buffers, used by
+    // alternate items, so the next item's rows are requested one item earlier.
+    static constexpr int kNBuf = (!GATED && P <= 32) ? 2 : 1;
+    static constexpr int kBytes = kS + kNBuf * kX * ((GATED && !kWInS) ? 2 : 1);
 };
 
 // fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
