@@ -102,27 +102,6 @@ __device__ __forceinline__ bool bar_or(int id, int n, bool pred) {
     return r != 0;
 }
 
-// 1-D bulk copies (TMA, no multicast): global -> shared completing on an
-// mbarrier's transaction count, and shared -> global in bulk groups.
-// Addresses 16-byte aligned, sizes multiples of 16 bytes.
-__device__ __forceinline__ void mbar_expect_tx(uint32_t addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(mbar)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until the shared-memory sources of all committed bulk stores have been read
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// wait until all committed bulk stores are complete
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 // TMEM loads: the wait is tied to the destination registers so no use of them
 // is scheduled before it.
 // R consecutive 8-column blocks (R = 1, 2, 4, 8) of 16 lanes: registers 4r .. 4r + 3 hold block r
