@@ -397,23 +397,41 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         if (GATED && SM::kWInS && item + (int)gridDim.x < items) stage_input(item + gridDim.x, 2, 0);
 
         // ---- store y (gate by v), coalesced 16-byte chunks of rows b and b+1
-        for (int i = tid; i < 2 * CH; i += NT) {
-            const int plane = i / CH, n0 = (i % CH) * 8;
-            if (plane == 1 && !has1) continue;
-            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
-            uint4 val;
-            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
-                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                         : "r"(plane_addr(plane ? sim : sre, p, chunk)));
-            const size_t off = (plane ? row1 : row0) + n0;
-            if (GATED) {
+        if constexpr (!GATED) {
+            // unrolled: every chunk's shared-memory read and global store issue back to back
+            constexpr int ITER = 2 * CH / NT;
+            static_assert(ITER * NT == 2 * CH, "store loop");
+#pragma unroll
+            for (int e = 0; e < ITER; ++e) {
+                const int i = tid + e * NT;
+                const int plane = i / CH, n0 = (i % CH) * 8;
+                if (plane == 1 && !has1) continue;
+                const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+                uint4 val;
+                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                             : "r"(plane_addr(plane ? sim : sre, p, chunk)));
+                *reinterpret_cast<uint4*>(y + (plane ? row1 : row0) + n0) = val;
+            }
+        } else {
+            // gated: the loop as written (unrolling with the gate's loads hoisted
+            // spills at this kernel's register budget and was measured slower)
+            for (int i = tid; i < 2 * CH; i += NT) {
+                const int plane = i / CH, n0 = (i % CH) * 8;
+                if (plane == 1 && !has1) continue;
+                const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+                uint4 val;
+                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                             : "r"(plane_addr(plane ? sim : sre, p, chunk)));
+                const size_t off = (plane ? row1 : row0) + n0;
                 const uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + off));
                 val.x = as_u(__hmul2(as_b2(val.x), as_b2(vv.x)));
                 val.y = as_u(__hmul2(as_b2(val.y), as_b2(vv.y)));
                 val.z = as_u(__hmul2(as_b2(val.z), as_b2(vv.z)));
                 val.w = as_u(__hmul2(as_b2(val.w), as_b2(vv.w)));
+                *reinterpret_cast<uint4*>(y + off) = val;
             }
-            *reinterpret_cast<uint4*>(y + off) = val;
         }
         // the next iteration's wait + barrier orders these reads before S is rewritten
     }
