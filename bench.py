@@ -221,11 +221,11 @@ class Runner:
 
     def compute_dtype(self):
         return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16",
-                "fused_umma": "bf16"}.get(self.plan.path, "f32")
+                "fused_umma": "bf16", "2d_tc": "f32+bf16"}.get(self.plan.path, "f32")
 
     def dominant_kernel(self):
         return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2",
-                "fused_tc": "fused_fwd_tc", "fused_umma": "fused_fwd_umma"}.get(self.plan.path)
+                "fused_tc": "fused_fwd_tc", "fused_umma": "fused_fwd_umma", "2d_tc": "c2tc_cols"}.get(self.plan.path)
 
 
 def time_steps(r, steps, torch, flush):

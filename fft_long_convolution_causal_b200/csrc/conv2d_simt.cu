@@ -87,7 +87,11 @@ c2_pass1(const IO* __restrict__ u, const float* __restrict__ k, int Kh, int Kw, 
 // Pass 2. MODE 0: column DFT, product, inverse column DFT (rows < Hs kept).
 //         MODE 1: column DFT only; Khat[c][ky][kx] = X / (LC LR).
 // KB: the spectrum is stored as packed bf16 (re, im) words (bf16 plans), else fp32 complex.
-template <int LOG2LC, int LOG2LR, int MODE, bool KB>
+// KTC (MODE 1, bf16, 2 Hs = 512): stored in the order the tensor-core column
+// pass reads -- per channel, column kx and parity of ky, per lane the packed
+// (re pair, im pair) of the four A-fragment registers of the [c][d] tile,
+// ky = parity + 2 (c + 16 d).
+template <int LOG2LC, int LOG2LR, int MODE, bool KB, bool KTC = false>
 __global__ void __launch_bounds__(Col2G<LOG2LC>::T)
 c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restrict__ khat_out,
          const float2* __restrict__ twC, int npp, int64_t first) {
@@ -113,7 +117,15 @@ c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restr
         stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int ky, int c, float2 z) {
             const size_t o = base + (size_t)ky * LR + kx0 + c;
             z = cscale(z, scale);
-            if (KB)
+            if constexpr (KTC) {
+                static_assert(LC == 512 && KB, "fragment order: bf16, 512-point columns");
+                const int kq = ky >> 1, cc = kq & 15, d = kq >> 4;
+                const int ln = 4 * (cc & 7) + ((d >> 1) & 3), reg = (cc >> 3) + 2 * (d >> 3);
+                const size_t word = (((size_t)P * LR + kx0 + c) * 2 + (ky & 1)) * 256 + ln * 8 + 2 * reg;
+                uint16_t* h = static_cast<uint16_t*>(khat_out);
+                h[word * 2 + (d & 1)] = __bfloat16_as_ushort(__float2bfloat16_rn(z.x));
+                h[(word + 1) * 2 + (d & 1)] = __bfloat16_as_ushort(__float2bfloat16_rn(z.y));
+            } else if (KB)
                 static_cast<uint32_t*>(khat_out)[o] =
                     (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.x)) |
                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(z.y)) << 16);
@@ -195,21 +207,29 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
         k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>((const IO*)u, nullptr, 0, 0, work, p.tw.wL, p.B,
                                                              p.H, Hs, first);
-        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, (p.B + 1) / 2,
-                                                                first);
+        if (p.tc2d) {
+            const cudaError_t e = launch_c2tc_cols(p, work, khat, g, first, s);
+            if (e != cudaSuccess) return e;
+        } else {
+            k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, (p.B + 1) / 2,
+                                                                    first);
+        }
         k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first);
     }
     return cudaGetLastError();
 }
 
-template <int LOG2LC, int LOG2LR, bool KB>
+template <int LOG2LC, int LOG2LR, bool KB, bool KTC = false>
 static cudaError_t c2_spec_go(const fftconv_plan_s& p, const float* k, int Kh, int Kw, void* khat, float2* work,
                               cudaStream_t s) {
+    if constexpr (KB && !KTC && LOG2LC == 9) {
+        if (p.tc2d) return c2_spec_go<LOG2LC, LOG2LR, true, true>(p, k, Kh, Kw, khat, work, s);
+    }
     constexpr int Hs = (1 << LOG2LC) / 2;
     constexpr int RB = rows_per_cta<LOG2LR>(Hs);
     constexpr int LR = 1 << LOG2LR;
     auto k1 = c2_pass1<LOG2LR, RB, float, 1>;
-    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1, KB>;
+    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1, KB, KTC>;
     const size_t sr = Row2G<LOG2LR, RB>::Lay::kWords * sizeof(float2);
     const size_t sc = Col2G<LOG2LC>::Lay::kWords * sizeof(float2);
     ensure_smem2(k1, sr);

@@ -1,0 +1,268 @@
+// conv2d_tc.cu -- the column pass of the 2-D causal FFT convolution on the
+// bf16 tensor cores, for images of 256 rows (columns of 2 Hs = 512 points).
+//
+// After the row pass the workspace holds, per pair of images (real +
+// imaginary part) and for every row i < 256 and column kx < 2 Ws, the row
+// spectrum W[i][kx] (fp32 complex).  The column pass of "Native
+// Multi-Dimensional Subquadratic Operators via Input Dependent Long
+// Convolutions" (abstract: the multi-dimensional FFT convolution) is, per
+// column, a 512-point DFT over the 256 nonzero rows, a product with the
+// channel's spectrum column, and the inverse keeping rows i < 256.  With the
+// upper half zero, the 512-point DFT splits into two 256-point DFTs (ky even:
+// of x; ky odd: of x W_512^i), each the 16 x 16 Monarch product of
+// "FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores"
+// (abstract) on mma.sync: over a (i = 16 a + b), times W_256^{b c}, transpose,
+// over b.  The inverse runs the conjugate products in reverse order and
+// recombines the halves: z[i] = Z_even[i] + W_512^{-i} Z_odd[i].
+// Per CTA: 16 consecutive columns of one pair; per warp: 4 columns, two
+// units (even, odd) at a time.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "plan.h"
+#include "tables.h"
+#include "tc_common.cuh"
+
+namespace fftc {
+namespace tc {
+
+constexpr int kC2Cols = 16;  // columns per CTA
+
+// Column pass.  work: [pair][256][LR] fp32 complex; khat: [channel][LR][2 (ky parity)][32 lanes][8 words]
+// Output tile: row i, 16 columns of fp32 complex; column c of row i at
+// position c ^ s(i), s(i) = (i & 7) | (((i >> 5) & 1) << 3), so the 32 lanes
+// of one accumulator store (one column, rows g + 32 t + const) hit every
+// position twice (two wavefronts, the minimum for 8-byte stores).
+__device__ __forceinline__ int c2_outpos(int i, int c) { return i * kC2Cols + (c ^ ((i & 7) | (((i >> 5) & 1) << 3))); }
+
+template <int LOG2LR>
+__global__ void __launch_bounds__(128, 4)
+c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables tb, int npp, int64_t first) {
+    constexpr int LR = 1 << LOG2LR, Hs = 256;
+    __shared__ __align__(128) uint8_t smem[2 * kC2Cols * 512];  // re, im planes: row = column, 256 i
+    __shared__ __align__(16) float2 otile[Hs * kC2Cols];        // results, rows i, before the coalesced store
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const int64_t P = first + blockIdx.y;
+    const int kx0 = blockIdx.x * kC2Cols;
+    const int ch = (int)(P / npp);
+    float2* __restrict__ img = work + (size_t)blockIdx.y * Hs * LR;
+    const uint32_t pre = smem_u32(smem), pim = pre + kC2Cols * 512;
+
+    // ---- tile of 256 rows x 16 columns -> bf16 planes (row = column, two rows i per 32-bit word)
+#pragma unroll 4
+    for (int it = 0; it < (Hs / 2) * (kC2Cols / 2) / 128; ++it) {
+        const int idx = tid + it * 128;
+        const int i = 2 * (idx / (kC2Cols / 2)), c = 2 * (idx % (kC2Cols / 2));
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(img + (size_t)i * LR + kx0 + c));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(img + (size_t)(i + 1) * LR + kx0 + c));
+        const uint32_t o = (uint32_t)(i & 7) * 2u;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(pre, c, i >> 3) + o), "r"(pack2(a.x, b.x)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(pim, c, i >> 3) + o), "r"(pack2(a.y, b.y)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(pre, c + 1, i >> 3) + o), "r"(pack2(a.z, b.z))
+                     : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(pim, c + 1, i >> 3) + o), "r"(pack2(a.w, b.w))
+                     : "memory");
+    }
+    uint2 f16[3][2], w256[4], t512[4];
+    float2 tz[2][4];  // W_512^{i} in accumulator order, fp32
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+        t512[i] = __ldg(&tb.t512[i * 32 + lane]);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tz[j][e] = __ldg(&tb.t512f[(j * 4 + e) * 32 + lane]);
+    __syncthreads();
+
+    const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
+    const uint4* __restrict__ kh = khat + ((size_t)ch * LR + kx0) * 2 * 64;
+    // i = 16 a + b of accumulator element (j, e): a = 8 j + 2 t + (e & 1), b = g + 8 (e >> 1)
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+        const int col = 4 * warp + cc;
+        uint4 k0[2], k1[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            k0[u] = __ldg(&kh[((size_t)col * 2 + u) * 64 + lane * 2]);
+            k1[u] = __ldg(&kh[((size_t)col * 2 + u) * 64 + lane * 2 + 1]);
+        }
+        uint32_t xr[2][4], xi[2][4];
+        ldsm_x4_t(xr[0], plane_addr(pre, col, ichunk));
+        ldsm_x4_t(xi[0], plane_addr(pim, col, ichunk));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xr[1][i] = xr[0][i];
+            xi[1][i] = xi[0][i];
+            twiddle2<true>(xr[1][i], xi[1][i], t512[i]);  // odd ky: x W_512^{i}
+        }
+        float acr[2][2][4], aci[2][2][4];
+        // forward: [b][a] x F16 -> [b][c]; x W_256^{b c}; transpose -> [c][b]; x F16 -> [c][d]
+#pragma unroll
+        for (int u = 0; u < 2; ++u) cmma2z(acr[u], aci[u], xr[u], xi[u], f16[0], f16[1], f16[2]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            uint32_t tr[4], ti[4];
+            pack_tile(tr, acr[u]);
+            pack_tile(ti, aci[u]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+            transpose_tile(xr[u], tr);
+            transpose_tile(xi[u], ti);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) cmma2z(acr[u], aci[u], xr[u], xi[u], f16[0], f16[1], f16[2]);
+        // spectrum at ky = u + 2 (c + 16 d): product with Khat
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            pack_tile(xr[u], acr[u]);
+            pack_tile(xi[u], aci[u]);
+            const uint32_t kre[4] = {k0[u].x, k0[u].z, k1[u].x, k1[u].z};
+            const uint32_t kim[4] = {k0[u].y, k0[u].w, k1[u].y, k1[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __nv_bfloat162 zr = as_b2(xr[u][i]), zi = as_b2(xi[u][i]);
+                const __nv_bfloat162 kr = as_b2(kre[i]), ki = as_b2(kim[i]);
+                xr[u][i] = as_u(__hfma2(zr, kr, __hneg2(__hmul2(zi, ki))));
+                xi[u][i] = as_u(__hfma2(zr, ki, __hmul2(zi, kr)));
+            }
+        }
+        // inverse: [c][d] x conj(F16) -> [c][b]; transpose -> [b][c]; x W_256^{-b c}; x conj(F16) -> [b][a]
+#pragma unroll
+        for (int u = 0; u < 2; ++u) cmma2z(acr[u], aci[u], xr[u], xi[u], f16[0], f16[2], f16[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            uint32_t gr[4], gi[4];
+            pack_tile(gr, acr[u]);
+            pack_tile(gi, aci[u]);
+            transpose_tile(xr[u], gr);
+            transpose_tile(xi[u], gi);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) twiddle2<false>(xr[u][i], xi[u][i], w256[i]);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) cmma2z(acr[u], aci[u], xr[u], xi[u], f16[0], f16[2], f16[1]);
+        // z[i] = Z_even[i] + W_512^{-i} Z_odd[i] (fp32) into the output tile
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 w = tz[j][e];
+                const float orr = acr[1][j][e], oi = aci[1][j][e];
+                // W_512^{-i} = cos + i sin of 2 pi i / 512
+                const float zr = acr[0][j][e] + fmaf(orr, w.x, -oi * w.y);
+                const float zi = aci[0][j][e] + fmaf(oi, w.x, orr * w.y);
+                const int i = 16 * (8 * j + 2 * t + (e & 1)) + g + 8 * (e >> 1);
+                otile[c2_outpos(i, col)] = make_float2(zr, zi);
+            }
+    }
+    __syncthreads();
+    // ---- rows i < 256 of the 16 columns back to the workspace, 128 bytes per row
+#pragma unroll 4
+    for (int it = 0; it < Hs * (kC2Cols / 2) / 128; ++it) {
+        const int idx = tid + it * 128;
+        const int i = idx / (kC2Cols / 2), c = 2 * (idx % (kC2Cols / 2));
+        // columns c, c + 1 sit in adjacent positions (their order flips when s(i) is odd)
+        const int p0 = c2_outpos(i, c);
+        const float4 v = *reinterpret_cast<const float4*>(&otile[p0 & ~1]);
+        const float4 o = (p0 & 1) ? make_float4(v.z, v.w, v.x, v.y) : v;
+        __stcg(reinterpret_cast<float4*>(img + (size_t)i * LR + kx0 + c), o);
+    }
+}
+
+}  // namespace tc
+
+// ================================================================== host side
+namespace {
+
+uint16_t bf16_bits_c2(double x) {
+    const float f = (float)x;
+    uint32_t b;
+    memcpy(&b, &f, 4);
+    b += 0x7fffu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+uint32_t pack_c2(double lo, double hi) { return (uint32_t)bf16_bits_c2(lo) | ((uint32_t)bf16_bits_c2(hi) << 16); }
+void cs_c2(int64_t e, int64_t L, double* c, double* s) {
+    int64_t r = e % L;
+    if (r < 0) r += L;
+    const double a = 2.0 * M_PI * (double)r / (double)L;
+    *c = cos(a);
+    *s = sin(a);
+}
+void push_u2_c2(std::vector<float2>& out, uint32_t x, uint32_t y) {
+    float2 f;
+    memcpy(&f.x, &x, 4);
+    memcpy(&f.y, &y, 4);
+    out.push_back(f);
+}
+
+}  // namespace
+
+bool c2tc_supported(int Hs, int Ws, int dtype) { return dtype == FFTCONV_BF16 && Hs == 256 && Ws >= 16; }
+
+// Tables of the tensor-core column pass: DFT_16 fragments and W_256^{b c}
+// (shared with the 1-D kernel's tables), W_512^{i} as packed bf16 pairs in
+// A-fragment order and as fp32 in accumulator order.
+bool c2tc_tables(std::vector<float2>& out, size_t off[4]) {
+    size_t o1[6];
+    if (!tc_tables(12, out, o1)) return false;
+    off[0] = o1[0];
+    off[1] = o1[1];
+    // t512: A fragment [b][a], register r: b = g + 8 (r & 1), a = 2 t + 8 (r >> 1) + {0, 1}; (cos, sin) of W_512^{16 a + b}
+    off[2] = out.size();
+    for (int r = 0; r < 4; ++r)
+        for (int lane = 0; lane < 32; ++lane) {
+            const int g = lane >> 2, t = lane & 3, b = g + 8 * (r & 1), a0 = 2 * t + 8 * (r >> 1);
+            double ca, sa, cb, sb;
+            cs_c2(16 * a0 + b, 512, &ca, &sa);
+            cs_c2(16 * (a0 + 1) + b, 512, &cb, &sb);
+            push_u2_c2(out, pack_c2(ca, cb), pack_c2(sa, sb));
+        }
+    // t512f: accumulator (j, e): a = 8 j + 2 t + (e & 1), b = g + 8 (e >> 1); (cos, sin) of W_512^{16 a + b}, fp32
+    off[3] = out.size();
+    for (int j = 0; j < 2; ++j)
+        for (int e = 0; e < 4; ++e)
+            for (int lane = 0; lane < 32; ++lane) {
+                const int g = lane >> 2, t = lane & 3;
+                const int a = 8 * j + 2 * t + (e & 1), b = g + 8 * (e >> 1);
+                double c, s;
+                cs_c2(16 * a + b, 512, &c, &s);
+                out.push_back(make_float2((float)c, (float)s));
+            }
+    return true;
+}
+
+template <int LOG2LR>
+static cudaError_t c2tc_go(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
+                           cudaStream_t s) {
+    constexpr int LR = 1 << LOG2LR;
+    tc::c2tc_cols<LOG2LR><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc, (p.B + 1) / 2,
+                                                                     first);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_c2tc_cols(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
+                             cudaStream_t s) {
+    switch (p.Ws) {
+        case 16: return c2tc_go<5>(p, work, khat, g, first, s);
+        case 32: return c2tc_go<6>(p, work, khat, g, first, s);
+        case 64: return c2tc_go<7>(p, work, khat, g, first, s);
+        case 128: return c2tc_go<8>(p, work, khat, g, first, s);
+        case 256: return c2tc_go<9>(p, work, khat, g, first, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace fftc

@@ -187,8 +187,12 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     cudaGetDevice(&p->device);
     const int64_t LR = 2 * (int64_t)Ws, LC = 2 * (int64_t)Hs;
     std::vector<float2> host;
-    size_t offR = 0, offC = 0;
+    size_t offR = 0, offC = 0, offT[4] = {0, 0, 0, 0};
     fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
+    if (fftc::c2tc_supported(Hs, Ws, dtype) && !getenv("FFTCONV_NO_TC")) {
+        p->tc2d = true;
+        fftc::c2tc_tables(host, offT);
+    }
     const size_t offErr = append_status_word(host);
     const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
     int64_t g = (int64_t)(kGroupBytes / per_pair);
@@ -211,6 +215,13 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     p->tw.wL = (const float2*)p->d_tables + offR;
     p->tw.wC = (const float2*)p->d_tables + offC;
     p->d_err = (int*)((const float2*)p->d_tables + offErr);
+    if (p->tc2d) {
+        const float2* base = (const float2*)p->d_tables;
+        p->c2tc.f16 = (const uint2*)(base + offT[0]);
+        p->c2tc.w256 = (const uint2*)(base + offT[1]);
+        p->c2tc.t512 = (const uint2*)(base + offT[2]);
+        p->c2tc.t512f = base + offT[3];
+    }
     *out = p;
     return FFTCONV_OK;
 }
@@ -232,7 +243,7 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
         case fftc::PATH_FUSED: return "fused";
         case fftc::PATH_FUSED_TC: return p->umma ? "fused_umma" : "fused_tc";
         case fftc::PATH_MULTIPASS: return "multipass";
-        case fftc::PATH_2D: return "2d";
+        case fftc::PATH_2D: return p->tc2d ? "2d_tc" : "2d";
     }
     return "unknown";
 }

@@ -33,6 +33,14 @@ struct TcTablePtrs {
     const uint2* tw3 = nullptr;   // [k_p][reg 4][lane]             (cos, sin) of W_M^{q k_p}, q = 16 a + b
 };
 
+// Constant tables of the 2-D tensor-core column pass.
+struct C2TcTables {
+    const uint2* f16 = nullptr;     // DFT_16 B fragments (as TcTablePtrs::f16)
+    const uint2* w256 = nullptr;    // W_256^{b c} pairs (as TcTablePtrs::w256)
+    const uint2* t512 = nullptr;    // [reg 4][lane] (cos, sin) pairs of W_512^{i}, A-fragment order
+    const float2* t512f = nullptr;  // [j 2][e 4][lane] (cos, sin) of W_512^{i}, accumulator order, fp32
+};
+
 }  // namespace fftc
 
 struct fftconv_plan_s {
@@ -57,6 +65,8 @@ struct fftconv_plan_s {
     bool umma = false;              // fused tensor-core path on tcgen05 (else mma.sync)
     const void* umma_b = nullptr;   // tcgen05 path: B operand images of the DFT matrices
     int* d_err = nullptr;           // device status word: nonzero after a timed-out device wait
+    bool tc2d = false;              // 2-D: column pass on the tensor cores (bf16, Hs = 256)
+    fftc::C2TcTables c2tc;
     bool spectrum_ready = false;
     int device = 0;
 };
@@ -95,6 +105,13 @@ cudaError_t launch_multipass_spectrum(const fftconv_plan_s& p, const float* k, i
 cudaError_t launch_multipass_fwd(const fftconv_plan_s& p, const void* u, const void* v,
                                  const void* w, const float2* khat, const float* D, void* y,
                                  float2* work, cudaStream_t s);
+
+// 2-D column pass on the bf16 tensor cores (images of 256 rows); its spectrum
+// is stored in per-lane fragment order.
+bool c2tc_supported(int Hs, int Ws, int dtype);
+bool c2tc_tables(std::vector<float2>& out, size_t off[4]);
+cudaError_t launch_c2tc_cols(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
+                             cudaStream_t s);
 
 // 2-D path (row DFT -> column DFT, product, inverse column DFT -> row iDFT).
 cudaError_t launch_conv2d_spectrum(const fftconv_plan_s& p, const float* k, int Kh, int Kw,

@@ -228,6 +228,16 @@ def test_conv2d_small_kernel():
     assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel", scale=row_scale_2d(wl))
 
 
+@pytest.mark.parametrize("Ws,Kh,Kw", [(256, 24, 24), (64, 256, 9)])
+def test_conv2d_tensor_core_columns(Ws, Kh, Kw):
+    """bf16 images of 256 rows: the column pass runs on the tensor cores (every output compared)."""
+    from fft_long_convolution_causal_b200 import binding
+    wl = wlmod.make_2d(3, 2, 256, Ws, dtype="bf16", seed=Ws + Kh, Kh=Kh, Kw=Kw, sigma=64.0)
+    assert binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, "bf16").path == "2d_tc"
+    y = run_2d(wl)
+    assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "bf16", f"2d tc 256x{Ws} k{Kh}x{Kw}", scale=row_scale_2d(wl))
+
+
 def test_conv2d_named_sampled():
     wl = _named("conv2d_b4_c256_256x256_bf16")
     y = run_2d(wl)
