@@ -205,8 +205,14 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
     ensure_smem2(k3, sr);
     for (int64_t first = 0; first < p.pairs; first += p.group) {
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
-        k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>((const IO*)u, nullptr, 0, 0, work, p.tw.wL, p.B,
-                                                             p.H, Hs, first);
+        const bool tc_rows = c2tc_rows_supported(p);
+        if (tc_rows) {
+            const cudaError_t e = launch_c2tc_rows_fwd(p, u, work, g, first, s);
+            if (e != cudaSuccess) return e;
+        } else {
+            k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>((const IO*)u, nullptr, 0, 0, work, p.tw.wL, p.B,
+                                                                 p.H, Hs, first);
+        }
         if (p.tc2d) {
             const cudaError_t e = launch_c2tc_cols(p, work, khat, g, first, s);
             if (e != cudaSuccess) return e;
@@ -214,7 +220,12 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
             k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, (p.B + 1) / 2,
                                                                     first);
         }
-        k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first);
+        if (tc_rows) {
+            const cudaError_t e = launch_c2tc_rows_inv(p, work, y, g, first, s);
+            if (e != cudaSuccess) return e;
+        } else {
+            k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first);
+        }
     }
     return cudaGetLastError();
 }

@@ -181,6 +181,210 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
     }
 }
 
+
+// Row tile of the forward row pass: row r, LR = 512 columns of fp32 complex;
+// column kx of row r at kx ^ ((kx >> 6) & 3), which spreads one accumulator
+// store (kx = parity + 2 g + 64 t + const over the lanes) over every
+// position twice; columns kx, kx + 1 (kx even) stay adjacent.
+__device__ __forceinline__ int c2_rowpos(int r, int kx) { return r * 512 + (kx ^ ((kx >> 6) & 3)); }
+
+// Forward row pass (images of 256 x 256): rows i of the pair's two images
+// (real, imaginary part), 512-point DFT over j < 256 as two 256-point
+// Monarch DFTs (kx even: of x; kx odd: of x W_512^j) -> work[pair][i][kx].
+constexpr int kC2RowsF = 8;  // rows per CTA
+__global__ void __launch_bounds__(128, 4)
+c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2TcTables tb, int B, int C,
+              int64_t first) {
+    constexpr int Hs = 256, Ws = 256, LR = 512;
+    __shared__ __align__(128) uint8_t smem[2 * kC2RowsF * 512];   // re, im planes: row r, 256 j
+    __shared__ __align__(16) float2 otile[kC2RowsF * LR];          // row spectra before the coalesced store
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const int64_t P = first + blockIdx.y;
+    const int i0 = blockIdx.x * kC2RowsF;
+    const int npp = (B + 1) / 2;
+    const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
+    const bool has1 = b0 + 1 < B;
+    const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
+    const uint32_t pre = smem_u32(smem), pim = pre + kC2RowsF * 512;
+    // ---- rows i0 .. i0 + 7 of both images -> planes (16-byte chunks)
+    for (int idx = tid; idx < 2 * kC2RowsF * 32; idx += 128) {
+        const int plane = idx / (kC2RowsF * 32), r = (idx / 32) % kC2RowsF, chunk = idx % 32;
+        const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing image
+        const size_t off = (plane ? (has1 ? img1 : img0) : img0) + (size_t)(i0 + r) * Ws + chunk * 8;
+        cp_async16(plane_addr(plane ? pim : pre, r, chunk), u + off, bytes);
+    }
+    cp_async_commit();
+    uint2 f16[3][2], w256[4], t512[4];
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+        t512[i] = __ldg(&tb.t512[i * 32 + lane]);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+    for (int rr = 0; rr < kC2RowsF / 4; ++rr) {
+        const int r = 2 * warp + rr;
+        uint32_t xr[2][4], xi[2][4];
+        ldsm_x4_t(xr[0], plane_addr(pre, r, ichunk));
+        ldsm_x4_t(xi[0], plane_addr(pim, r, ichunk));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xr[1][i] = xr[0][i];
+            xi[1][i] = xi[0][i];
+            twiddle2<true>(xr[1][i], xi[1][i], t512[i]);  // odd kx: x W_512^{j}
+        }
+        float acr[2][2][4], aci[2][2][4];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            uint32_t tr[4], ti[4];
+            pack_tile(tr, acr[v]);
+            pack_tile(ti, aci[v]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+            transpose_tile(xr[v], tr);
+            transpose_tile(xi[v], ti);
+        }
+#pragma unroll
+        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
+        // accumulator (n, e) of unit v: c = g + 8 (e >> 1), d = 8 n + 2 t + (e & 1); kx = v + 2 (c + 16 d)
+#pragma unroll
+        for (int v = 0; v < 2; ++v)
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = g + 8 * (e >> 1), d = 8 * n + 2 * t + (e & 1);
+                    otile[c2_rowpos(r, v + 2 * (c + 16 * d))] = make_float2(acr[v][n][e], aci[v][n][e]);
+                }
+    }
+    __syncthreads();
+    float2* __restrict__ out = work + (size_t)blockIdx.y * Hs * LR + (size_t)i0 * LR;
+#pragma unroll 4
+    for (int it = 0; it < kC2RowsF * (LR / 2) / 128; ++it) {
+        const int idx = tid + it * 128;
+        const int r = idx / (LR / 2), kx = 2 * (idx % (LR / 2));
+        const int p0 = c2_rowpos(r, kx);
+        const float4 val = *reinterpret_cast<const float4*>(&otile[p0 & ~1]);
+        __stcg(reinterpret_cast<float4*>(out + (size_t)r * LR + kx),
+               (p0 & 1) ? make_float4(val.z, val.w, val.x, val.y) : val);
+    }
+}
+
+// Inverse row pass (images of 256 x 256): work[pair][i][kx] -> 512-point
+// inverse DFT over kx keeping j < 256, as two 256-point Monarch inverses
+// (kx even, kx odd) recombined with W_512^{-j} -> y rows of both images.
+constexpr int kC2RowsI = 16;  // rows per CTA
+__global__ void __launch_bounds__(128, 4)
+c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2TcTables tb, int B, int C,
+              int64_t first) {
+    constexpr int Hs = 256, Ws = 256, LR = 512;
+    // planes (row r, 256 k'): [parity][re, im]; then y planes (row r, 256 j) [image]
+    __shared__ __align__(128) uint8_t smem[4 * kC2RowsI * 512 + 2 * kC2RowsI * 512];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    const int64_t P = first + blockIdx.y;
+    const int i0 = blockIdx.x * kC2RowsI;
+    const int npp = (B + 1) / 2;
+    const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
+    const bool has1 = b0 + 1 < B;
+    const uint32_t base = smem_u32(smem);
+    auto plane = [&](int par, int im) { return base + (uint32_t)((2 * par + im) * kC2RowsI * 512); };
+    const uint32_t y0p = base + 4 * kC2RowsI * 512, y1p = y0p + kC2RowsI * 512;
+    const float2* __restrict__ in = work + (size_t)blockIdx.y * Hs * LR + (size_t)i0 * LR;
+    // ---- rows -> bf16 planes split by the parity of kx: k' = kx / 2, two k' per 32-bit word
+#pragma unroll 4
+    for (int it = 0; it < kC2RowsI * (LR / 4) / 128; ++it) {
+        const int idx = tid + it * 128;
+        const int r = idx / (LR / 4), kx = 4 * (idx % (LR / 4)), k2 = kx / 2;
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(in + (size_t)r * LR + kx));      // kx, kx + 1
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(in + (size_t)r * LR + kx + 2));  // kx + 2, kx + 3
+        const uint32_t o = (uint32_t)(k2 & 7) * 2u, chunk = (uint32_t)(k2 >> 3);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(0, 0), r, chunk) + o), "r"(pack2(a.x, b.x)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(0, 1), r, chunk) + o), "r"(pack2(a.y, b.y)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(1, 0), r, chunk) + o), "r"(pack2(a.z, b.z)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(1, 1), r, chunk) + o), "r"(pack2(a.w, b.w)) : "memory");
+    }
+    uint2 f16[3][2], w256[4];
+    float2 tz[2][4];
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tz[j][e] = __ldg(&tb.t512f[(j * 4 + e) * 32 + lane]);
+    __syncthreads();
+    const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
+#pragma unroll 1
+    for (int rr = 0; rr < kC2RowsI / 4; ++rr) {
+        const int r = 4 * warp + rr;
+        // A = [c][d], k' = c + 16 d, of the even and odd columns
+        uint32_t xr[2][4], xi[2][4];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            ldsm_x4_t(xr[v], plane_addr(plane(v, 0), r, ichunk));
+            ldsm_x4_t(xi[v], plane_addr(plane(v, 1), r, ichunk));
+        }
+        float acr[2][2][4], aci[2][2][4];
+        // [c][d] x conj(F16) -> [c][b]; transpose -> [b][c]; x W_256^{-b c}; x conj(F16) -> [b][a]
+#pragma unroll
+        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            uint32_t gr[4], gi[4];
+            pack_tile(gr, acr[v]);
+            pack_tile(gi, aci[v]);
+            transpose_tile(xr[v], gr);
+            transpose_tile(xi[v], gi);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) twiddle2<false>(xr[v][i], xi[v][i], w256[i]);
+        }
+#pragma unroll
+        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
+        // z[j] = Z_even[j] + W_512^{-j} Z_odd[j]: re -> image b0, im -> image b0 + 1
+        float zr[2][4], zi[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 w = tz[n][e];
+                const float orr = acr[1][n][e], oi = aci[1][n][e];
+                zr[n][e] = acr[0][n][e] + fmaf(orr, w.x, -oi * w.y);
+                zi[n][e] = aci[0][n][e] + fmaf(oi, w.x, orr * w.y);
+            }
+        uint32_t pr[4], pi[4];
+        pack_tile(pr, zr);
+        pack_tile(pi, zi);
+        stsm_x4_t(plane_addr(y0p, r, ichunk), pr[0], pr[1], pr[2], pr[3]);
+        stsm_x4_t(plane_addr(y1p, r, ichunk), pi[0], pi[1], pi[2], pi[3]);
+    }
+    __syncthreads();
+    // ---- y rows i0 .. i0 + 15 of both images, 16-byte chunks
+    const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
+    for (int idx = tid; idx < 2 * kC2RowsI * 32; idx += 128) {
+        const int im = idx / (kC2RowsI * 32), r = (idx / 32) % kC2RowsI, chunk = idx % 32;
+        if (im == 1 && !has1) continue;
+        uint4 val;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                     : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                     : "r"(plane_addr(im ? y1p : y0p, r, chunk)));
+        *reinterpret_cast<uint4*>(y + (im ? img1 : img0) + (size_t)(i0 + r) * Ws + chunk * 8) = val;
+    }
+}
+
 }  // namespace tc
 
 // ================================================================== host side
@@ -211,6 +415,7 @@ void push_u2_c2(std::vector<float2>& out, uint32_t x, uint32_t y) {
 }  // namespace
 
 bool c2tc_supported(int Hs, int Ws, int dtype) { return dtype == FFTCONV_BF16 && Hs == 256 && Ws >= 16; }
+bool c2tc_rows_supported(const fftconv_plan_s& p) { return p.tc2d && p.Ws == 256; }
 
 // Tables of the tensor-core column pass: DFT_16 fragments and W_256^{b c}
 // (shared with the 1-D kernel's tables), W_512^{i} as packed bf16 pairs in
@@ -250,6 +455,19 @@ static cudaError_t c2tc_go(const fftconv_plan_s& p, float2* work, const void* kh
     constexpr int LR = 1 << LOG2LR;
     tc::c2tc_cols<LOG2LR><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc, (p.B + 1) / 2,
                                                                      first);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_c2tc_rows_fwd(const fftconv_plan_s& p, const void* u, float2* work, int g, int64_t first,
+                                 cudaStream_t s) {
+    tc::c2tc_rows_fwd<<<dim3(256 / tc::kC2RowsF, g), 128, 0, s>>>((const __nv_bfloat16*)u, work, p.c2tc, p.B, p.H,
+                                                                  first);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_c2tc_rows_inv(const fftconv_plan_s& p, const float2* work, void* y, int g, int64_t first,
+                                 cudaStream_t s) {
+    tc::c2tc_rows_inv<<<dim3(256 / tc::kC2RowsI, g), 128, 0, s>>>(work, (__nv_bfloat16*)y, p.c2tc, p.B, p.H, first);
     return cudaGetLastError();
 }
 
