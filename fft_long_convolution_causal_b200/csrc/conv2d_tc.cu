@@ -54,7 +54,7 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
     const uint32_t pre = smem_u32(smem), pim = pre + kC2Cols * 512;
 
     // ---- tile of 256 rows x 16 columns -> bf16 planes (row = column, two rows i per 32-bit word)
-#pragma unroll 4
+#pragma unroll
     for (int it = 0; it < (Hs / 2) * (kC2Cols / 2) / 128; ++it) {
         const int idx = tid + it * 128;
         const int i = 2 * (idx / (kC2Cols / 2)), c = 2 * (idx % (kC2Cols / 2));
@@ -302,7 +302,7 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
     const uint32_t y0p = base + 4 * kC2RowsI * 512, y1p = y0p + kC2RowsI * 512;
     const float2* __restrict__ in = work + (size_t)blockIdx.y * Hs * LR + (size_t)i0 * LR;
     // ---- rows -> bf16 planes split by the parity of kx: k' = kx / 2, two k' per 32-bit word
-#pragma unroll 4
+#pragma unroll 8
     for (int it = 0; it < kC2RowsI * (LR / 4) / 128; ++it) {
         const int idx = tid + it * 128;
         const int r = idx / (LR / 4), kx = 4 * (idx % (LR / 4)), k2 = kx / 2;
