@@ -40,7 +40,8 @@ METRIC = "FFT-conv output elems/s and % of HBM roofline (1 B200), N=1K–1M and 
 DEFAULT_CONFIG = "hyena_b8_h768_n4096_bf16"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ["fft_simt.cuh", "conv1d_simt.cu", "conv2d_simt.cu", "conv1d_mma.cu"]
+KERNEL_SOURCES = ["fft_simt.cuh", "conv1d_simt.cu", "conv2d_simt.cu", "tc_common.cuh", "conv1d_mma.cu", "umma.cuh",
+                  "conv1d_umma.cu", "conv2d_tc.cu"]
 
 
 def parse():
