@@ -146,8 +146,9 @@ def test_multipass_sampled(log2N):
     assert_close(y[b, h, t], ref, "f32", f"multipass N=2^{log2N}", scale=row_scale_1d(wl, b, h))
 
 
-def test_multipass_ragged_groups():
+def test_multipass_ragged_groups(monkeypatch):
     """More pairs than one workspace group holds, with a short last group."""
+    monkeypatch.setenv("FFTCONV_GROUP_MB", "64")  # 4 pairs of 16 MiB per group: groups of 4, 4, 2
     N = 1 << 20
     wl = wlmod.make_1d(3, 5, N, dtype="bf16", seed=99, alpha=1e-5)
     y, _ = run_1d(wl)
@@ -226,6 +227,16 @@ def test_conv2d_small_kernel():
     wl = wlmod.make_2d(2, 3, 64, 64, dtype="f32", seed=2, Kh=5, Kw=17)
     y = run_2d(wl)
     assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel", scale=row_scale_2d(wl))
+
+
+def test_conv2d_tensor_core_groups(monkeypatch):
+    """2-D on the tensor cores with several workspace groups (the last one short)."""
+    monkeypatch.setenv("FFTCONV_GROUP_MB", "4")  # 4 pairs of 1 MiB per group: groups of 4, 2 (6 pairs)
+    wl = wlmod.make_2d(4, 3, 256, 256, dtype="bf16", seed=31, Kh=12, Kw=20, sigma=64.0)
+    y = run_2d(wl)
+    idx = wlmod.sample_points_2d(wl.B, wl.C, wl.Hs, wl.Ws, 2048, seed=31)
+    ref = oracle.causal_conv2d_points(wl.u, wl.k, *idx)
+    assert_close(y[idx], ref, "bf16", "2d tc groups", scale=row_scale_2d(wl, idx[0], idx[1]))
 
 
 @pytest.mark.parametrize("Ws,Kh,Kw", [(256, 24, 24), (64, 256, 9)])
