@@ -21,8 +21,8 @@
 //   pass 2: per row k1, DFT_N2 over n2, times Khat[k1][k2] (+ D/M), inverse
 //           DFT_N2, times W_M^{-n2 k1}, back into the workspace;
 //   pass 3: per column n2, inverse DFT_N1, only n1 < N1/2 (n < N) kept.
-// Pairs are processed in groups so the workspace of one group stays small
-// (L2-sized) and is reused group after group.
+// Pairs are processed in groups (the plan sizes them, up to 1 GiB of
+// workspace) and the workspace is reused group after group.
 #include "fft_simt.cuh"
 #include "plan.h"
 #include "tables.h"
