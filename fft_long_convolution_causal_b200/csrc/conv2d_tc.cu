@@ -39,7 +39,16 @@ constexpr int kC2Cols = 16;  // columns per CTA
 // position twice (two wavefronts, the minimum for 8-byte stores).
 __device__ __forceinline__ int c2_outpos(int i, int c) { return i * kC2Cols + (c ^ ((i & 7) | (((i >> 5) & 1) << 3))); }
 
-template <int LOG2LR>
+// bf16 workspace of the all-tensor-core 2-D path (256 x 256 images), per
+// pair 512 KiB each:
+//   rows -> columns  W1[kx 512][row tile 32][re, im][8 rows]
+//   columns -> rows  W2[i 256][column tile 32][kx parity][re, im][8 k' = kx / 2]
+// Every pass rounds to bf16 where it reads its operands, so storing bf16
+// changes no result; each write is a whole 32- or 64-byte segment and each
+// read a 16-byte copy into the reader's swizzled planes.
+constexpr size_t kW1Bytes = 512 * 1024;
+
+template <int LOG2LR, bool BW>
 __global__ void __launch_bounds__(128, 4)
 c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables tb, int npp, int64_t first) {
     constexpr int LR = 1 << LOG2LR, Hs = 256;
@@ -53,9 +62,19 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
     float2* __restrict__ img = work + (size_t)blockIdx.y * Hs * LR;
     const uint32_t pre = smem_u32(smem), pim = pre + kC2Cols * 512;
 
-    // ---- tile of 256 rows x 16 columns -> bf16 planes (row = column, two rows i per 32-bit word)
+    uint8_t* __restrict__ w1 = reinterpret_cast<uint8_t*>(img);  // bf16 workspace (BW)
+    if constexpr (BW) {
+        // ---- W1 columns kx0 .. kx0 + 15 (1 KiB each) -> planes, 16-byte copies
+        const uint8_t* src = w1 + (size_t)kx0 * 1024;
+        for (int q = tid; q < kC2Cols * 64; q += 128) {
+            const int col = q >> 6, tile = (q >> 1) & 31, pl = q & 1;
+            cp_async16(plane_addr(pl ? pim : pre, col, tile), src + (size_t)q * 16, 16);
+        }
+        cp_async_commit();
+    }
+    // ---- fp32 workspace: tile of 256 rows x 16 columns -> bf16 planes (row = column, two rows i per 32-bit word)
 #pragma unroll
-    for (int it = 0; it < (Hs / 2) * (kC2Cols / 2) / 128; ++it) {
+    for (int it = 0; it < (BW ? 0 : (Hs / 2) * (kC2Cols / 2) / 128); ++it) {
         const int idx = tid + it * 128;
         const int i = 2 * (idx / (kC2Cols / 2)), c = 2 * (idx % (kC2Cols / 2));
         const float4 a = __ldcg(reinterpret_cast<const float4*>(img + (size_t)i * LR + kx0 + c));
@@ -83,6 +102,7 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
     for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tz[j][e] = __ldg(&tb.t512f[(j * 4 + e) * 32 + lane]);
+    if (BW) cp_async_wait_all();
     __syncthreads();
 
     const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
@@ -168,7 +188,26 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
             }
     }
     __syncthreads();
-    // ---- rows i < 256 of the 16 columns back to the workspace, 128 bytes per row
+    if constexpr (BW) {
+        // ---- W2 rows i: this tile's 64 bytes ([parity][re, im][8 k']); lane m of an
+        // 8-lane group writes 8 bytes: segment m / 2 (parity, re/im), k' = 4 (m & 1) .. + 3
+        uint8_t* __restrict__ w2 = w1 + kW1Bytes + (size_t)(kx0 / kC2Cols) * 64;
+#pragma unroll 4
+        for (int q = tid; q < Hs * 8; q += 128) {
+            const int i = q >> 3, m = q & 7, seg = m >> 1, h = m & 1;
+            const int parity = seg >> 1, im = seg & 1;
+            float v[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const float2 z = otile[c2_outpos(i, 8 * h + 2 * jj + parity)];
+                v[jj] = im ? z.y : z.x;
+            }
+            const uint2 o = make_uint2(pack2(v[0], v[1]), pack2(v[2], v[3]));
+            *reinterpret_cast<uint2*>(w2 + (size_t)i * 2048 + seg * 16 + h * 8) = o;
+        }
+        return;
+    }
+    // ---- fp32 workspace: rows i < 256 of the 16 columns back, 128 bytes per row
 #pragma unroll 4
     for (int it = 0; it < Hs * (kC2Cols / 2) / 128; ++it) {
         const int idx = tid + it * 128;
@@ -268,15 +307,21 @@ c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2
                 }
     }
     __syncthreads();
-    float2* __restrict__ out = work + (size_t)blockIdx.y * Hs * LR + (size_t)i0 * LR;
-#pragma unroll 4
-    for (int it = 0; it < kC2RowsF * (LR / 2) / 128; ++it) {
-        const int idx = tid + it * 128;
-        const int r = idx / (LR / 2), kx = 2 * (idx % (LR / 2));
-        const int p0 = c2_rowpos(r, kx);
-        const float4 val = *reinterpret_cast<const float4*>(&otile[p0 & ~1]);
-        __stcg(reinterpret_cast<float4*>(out + (size_t)r * LR + kx),
-               (p0 & 1) ? make_float4(val.z, val.w, val.x, val.y) : val);
+    // ---- W1[kx][row tile i0 / 8][re, im][8 rows]: 32 bytes per column kx
+    static_assert(kC2RowsF == 8, "one row tile of W1 per CTA");
+    uint8_t* __restrict__ w1 = reinterpret_cast<uint8_t*>(work + (size_t)blockIdx.y * Hs * LR) + (size_t)(i0 / 8) * 32;
+#pragma unroll
+    for (int kx = tid; kx < LR; kx += 128) {
+        float re[8], im[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const float2 z = otile[c2_rowpos(r, kx)];
+            re[r] = z.x;
+            im[r] = z.y;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(w1 + (size_t)kx * 1024);
+        dst[0] = make_uint4(pack2(re[0], re[1]), pack2(re[2], re[3]), pack2(re[4], re[5]), pack2(re[6], re[7]));
+        dst[1] = make_uint4(pack2(im[0], im[1]), pack2(im[2], im[3]), pack2(im[4], im[5]), pack2(im[6], im[7]));
     }
 }
 
@@ -300,20 +345,14 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
     const uint32_t base = smem_u32(smem);
     auto plane = [&](int par, int im) { return base + (uint32_t)((2 * par + im) * kC2RowsI * 512); };
     const uint32_t y0p = base + 4 * kC2RowsI * 512, y1p = y0p + kC2RowsI * 512;
-    const float2* __restrict__ in = work + (size_t)blockIdx.y * Hs * LR + (size_t)i0 * LR;
-    // ---- rows -> bf16 planes split by the parity of kx: k' = kx / 2, two k' per 32-bit word
-#pragma unroll 8
-    for (int it = 0; it < kC2RowsI * (LR / 4) / 128; ++it) {
-        const int idx = tid + it * 128;
-        const int r = idx / (LR / 4), kx = 4 * (idx % (LR / 4)), k2 = kx / 2;
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(in + (size_t)r * LR + kx));      // kx, kx + 1
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(in + (size_t)r * LR + kx + 2));  // kx + 2, kx + 3
-        const uint32_t o = (uint32_t)(k2 & 7) * 2u, chunk = (uint32_t)(k2 >> 3);
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(0, 0), r, chunk) + o), "r"(pack2(a.x, b.x)) : "memory");
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(0, 1), r, chunk) + o), "r"(pack2(a.y, b.y)) : "memory");
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(1, 0), r, chunk) + o), "r"(pack2(a.z, b.z)) : "memory");
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(plane_addr(plane(1, 1), r, chunk) + o), "r"(pack2(a.w, b.w)) : "memory");
+    // ---- W2 rows i0 .. i0 + 15 (2 KiB each: [column tile][parity][re, im][8 k']) -> planes
+    const uint8_t* __restrict__ w2 =
+        reinterpret_cast<const uint8_t*>(work + (size_t)blockIdx.y * Hs * LR) + kW1Bytes + (size_t)i0 * 2048;
+    for (int q = tid; q < kC2RowsI * 128; q += 128) {
+        const int r = q >> 7, tile = (q >> 2) & 31, par = (q >> 1) & 1, pl = q & 1;
+        cp_async16(plane_addr(plane(par, pl), r, tile), w2 + (size_t)q * 16, 16);
     }
+    cp_async_commit();
     uint2 f16[3][2], w256[4];
     float2 tz[2][4];
 #pragma unroll
@@ -326,6 +365,7 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
     for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tz[j][e] = __ldg(&tb.t512f[(j * 4 + e) * 32 + lane]);
+    cp_async_wait_all();
     __syncthreads();
     const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
 #pragma unroll 1
@@ -453,7 +493,15 @@ template <int LOG2LR>
 static cudaError_t c2tc_go(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
                            cudaStream_t s) {
     constexpr int LR = 1 << LOG2LR;
-    tc::c2tc_cols<LOG2LR><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc, (p.B + 1) / 2,
+    if constexpr (LOG2LR == 9) {
+        // all passes on the tensor cores: the bf16 workspace
+        if (c2tc_rows_supported(p)) {
+            tc::c2tc_cols<LOG2LR, true><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc,
+                                                                                 (p.B + 1) / 2, first);
+            return cudaGetLastError();
+        }
+    }
+    tc::c2tc_cols<LOG2LR, false><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc, (p.B + 1) / 2,
                                                                      first);
     return cudaGetLastError();
 }
