@@ -46,7 +46,8 @@ namespace tc {
 // kc0/kc1: the rows' Khat words, tw: their W_M^{-q k_p} twiddles.
 template <int RN, bool IP>
 __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int (&kp)[RN], int lane,
-                                           const uint2 (&f16)[3][2], const uint2 (&w256)[4], const uint4 (&kc0)[RN],
+                                           const uint2 (&f16)[3][2], const uint2 (&w256)[4],
+                                           const uint32_t (&w256n)[4], const uint4 (&kc0)[RN],
                                            const uint4 (&kc1)[RN], const uint2 (&tw)[RN][4], __nv_bfloat162 dm2) {
     const int m8 = lane >> 3, r8 = lane & 7;
     const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
@@ -66,7 +67,7 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
         pack_tile<IP>(tr, acr[r]);
         pack_tile<IP>(ti, aci[r]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+        for (int i = 0; i < 4; ++i) twiddle2n<true>(tr[i], ti[i], w256[i], w256n[i]);
         transpose_tile(xr[r], tr);
         transpose_tile(xi[r], ti);
     }
@@ -100,7 +101,7 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
         transpose_tile(xr[r], gr);
         transpose_tile(xi[r], gi);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) twiddle2<false>(xr[r][i], xi[r][i], w256[i]);
+        for (int i = 0; i < 4; ++i) twiddle2n<false>(xr[r][i], xi[r][i], w256[i], w256n[i]);
     }
     // inverse stage i: [b][c] x conj(F16) -> [b][a]
 #pragma unroll
@@ -273,6 +274,9 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+    uint32_t w256n[4];  // the negated sines
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w256n[i] = as_u(__hneg2(as_b2(w256[i].y)));
     uint2 fp[PRE1 ? S::KS1 : 1][PRE1 ? S::NT1 : 1][3];
     if (PRE1) {
 #pragma unroll
@@ -328,32 +332,30 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
             const float dmf = D ? D[h] * (1.0f / S::M) : 0.f;
             const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
             const uint4* __restrict__ kh = khat + (size_t)h * P * 64;  // 32 lanes x 2 uint4 per row
-            uint4 kn0[RN], kn1[RN];
-            uint2 tn[RN][4];
-            auto fetch = [&](int kp0) {
+            // two sets of the rows' Khat words and twiddles, filled alternately one
+            // iteration ahead (a ping-pong instead of copying the prefetched set)
+            uint4 ka0[RN], ka1[RN], kb0[RN], kb1[RN];
+            uint2 ta[RN][4], tq[RN][4];
+            auto fetch = [&](int kp0, uint4(&k0)[RN], uint4(&k1)[RN], uint2(&t)[RN][4]) {
 #pragma unroll
                 for (int r = 0; r < RN; ++r) {
                     const int kp = kp0 + r * NW;
-                    kn0[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
-                    kn1[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
+                    k0[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2]);
+                    k1[r] = __ldg(&kh[(size_t)kp * 64 + lane * 2 + 1]);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) tn[r][i] = __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]);
+                    for (int i = 0; i < 4; ++i) t[r][i] = __ldg(&tb.tw3[((size_t)kp * 4 + i) * 32 + lane]);
                 }
             };
-            fetch(warp);
-            for (int kp0 = warp; kp0 < P; kp0 += RN * NW) {
-                uint4 kc0[RN], kc1[RN];
-                uint2 tc3[RN][4];
-#pragma unroll
-                for (int r = 0; r < RN; ++r) {
-                    kc0[r] = kn0[r];
-                    kc1[r] = kn1[r];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) tc3[r][i] = tn[r][i];
-                }
-                if (kp0 + RN * NW < P) fetch(kp0 + RN * NW);
+            static_assert((P / NW) % (2 * RN) == 0, "row pairs per warp come in twos");
+            fetch(warp, ka0, ka1, ta);
+            for (int kp0 = warp; kp0 < P; kp0 += 2 * RN * NW) {
+                const int kq = kp0 + RN * NW;
+                fetch(kq, kb0, kb1, tq);
                 const int kps[RN] = {kp0, kp0 + NW};
-                inner_rows<RN, IP>(sre, sim, kps, lane, f16, w256, kc0, kc1, tc3, dm2);
+                inner_rows<RN, IP>(sre, sim, kps, lane, f16, w256, w256n, ka0, ka1, ta, dm2);
+                if (kq + RN * NW < P) fetch(kq + RN * NW, ka0, ka1, ta);
+                const int kqs[RN] = {kq, kq + NW};
+                inner_rows<RN, IP>(sre, sim, kqs, lane, f16, w256, w256n, kb0, kb1, tq, dm2);
             }
         }
         __syncthreads();
@@ -462,6 +464,9 @@ tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, Tc
         for (int j = 0; j < 2; ++j) f16[part][j] = __ldg(&tb.f16[(j * 3 + part) * 32 + lane]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) w256[i] = __ldg(&tb.w256[i * 32 + lane]);
+    uint32_t w256n[4];  // the negated sines
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w256n[i] = as_u(__hneg2(as_b2(w256[i].y)));
     uint2 fp[PRE1 ? S::KS1 : 1][PRE1 ? S::NT1 : 1][3];
     if (PRE1) {
 #pragma unroll

@@ -84,6 +84,20 @@ __device__ __forceinline__ void twiddle2(uint32_t& re, uint32_t& im, uint2 cs) {
     }
 }
 
+// As twiddle2 with the negated sine ns = -s at hand: two products and two
+// fused multiply-adds, no negation.
+template <bool FWD>
+__device__ __forceinline__ void twiddle2n(uint32_t& re, uint32_t& im, uint2 cs, uint32_t ns) {
+    const __nv_bfloat162 r = as_b2(re), i = as_b2(im), c = as_b2(cs.x), s = as_b2(cs.y), n = as_b2(ns);
+    if (FWD) {
+        re = as_u(__hfma2(r, c, __hmul2(i, s)));
+        im = as_u(__hfma2(i, c, __hmul2(r, n)));
+    } else {
+        re = as_u(__hfma2(r, c, __hmul2(i, n)));
+        im = as_u(__hfma2(i, c, __hmul2(r, s)));
+    }
+}
+
 // Complex product of one 16x16 A tile with the two n-tiles of a 16x16 B:
 // the four products with Ar first, then the four with Ai, so each dependent
 // accumulation is four MMAs behind the one it waits for.
