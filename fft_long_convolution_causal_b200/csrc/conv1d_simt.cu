@@ -211,10 +211,14 @@ cudaError_t launch_fused_spectrum(const fftconv_plan_s& p, const float* k, int64
 }
 
 // ========================================================== multi-pass path
-constexpr int kColTile = 16;  // columns per CTA in the column passes (128 B of fp32 complex)
+// Columns per CTA in the column passes: as many as one CTA's 16384 points
+// allow, at most 32 (rows of 256 B of fp32 complex in the workspace, 128 B of
+// fp32 input and output).
+template <int LOG2N1>
+constexpr int kColTile = (16384 >> LOG2N1) < 32 ? (16384 >> LOG2N1) : 32;
 
 template <int LOG2N1>
-using ColG = Geometry<LOG2N1, kColTile, true>;
+using ColG = Geometry<LOG2N1, kColTile<LOG2N1>, true>;
 // Rows per CTA in the row pass: enough that one CTA holds 4096 points (at
 // most 16 rows), so short rows do not leave single-warp CTAs.
 constexpr int row_batch(int log2n2) { return log2n2 >= 12 ? 1 : ((4096 >> log2n2) > 16 ? 16 : (4096 >> log2n2)); }
@@ -249,7 +253,7 @@ mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __rest
     extern __shared__ float2 smem[];
     const int tid = threadIdx.x;
     const int64_t P = first + blockIdx.y;
-    const int n2_0 = blockIdx.x * kColTile;
+    const int n2_0 = blockIdx.x * kColTile<LOG2N1>;
     auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
     auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
     if constexpr (MODE == 0) {
@@ -353,7 +357,7 @@ mp_pass3(const float2* __restrict__ work, const IO* __restrict__ v, IO* __restri
     extern __shared__ float2 smem[];
     const int tid = threadIdx.x;
     const int64_t P = first + blockIdx.y;
-    const int n2_0 = blockIdx.x * kColTile;
+    const int n2_0 = blockIdx.x * kColTile<LOG2N1>;
     const float2* __restrict__ in = work + (size_t)blockIdx.y * ((size_t)N1 * N2);
     auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
     auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
@@ -384,12 +388,12 @@ static cudaError_t mp_fwd_go(const fftconv_plan_s& p, const void* u, const void*
     ensure_smem(k3, sc);
     for (int64_t first = 0; first < p.pairs; first += p.group) {
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
-        k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
+        k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
                                                                p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S, p.B,
                                                                p.H, first);
         k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
                                                     p.log2S, p.H, first);
-        k3<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
+        k3<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
                                                                p.H, first);
     }
     return cudaGetLastError();
@@ -417,7 +421,7 @@ static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L
     ensure_smem(k2, sr);
     for (int64_t first = 0; first < p.H; first += p.group) {
         const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
-        k1<<<dim3(N2 / kColTile, g), ColG<LOG2N1>::T, sc, s>>>(nullptr, nullptr, k, (int)L, work, p.tw.wC,
+        k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>(nullptr, nullptr, k, (int)L, work, p.tw.wC,
                                                                p.tw.wLo, p.tw.wHi, p.log2S, p.B, p.H, first);
         k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, nullptr, khat, nullptr, p.tw.wL, p.tw.wLo, p.tw.wHi,
                                                     p.log2S, p.H, first);
@@ -432,8 +436,8 @@ static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L
         case 17: return CALL(8, 9);      \
         case 18: return CALL(9, 9);      \
         case 19: return CALL(9, 10);     \
-        case 20: return CALL(10, 10);    \
-        case 21: return CALL(10, 11);    \
+        case 20: return CALL(9, 11);     \
+        case 21: return CALL(9, 12);     \
         default: return cudaErrorInvalidValue; \
     }
 
@@ -453,8 +457,8 @@ bool multipass_tables(int log2M, std::vector<float2>& out, size_t* offC, size_t*
         case 17: return mp_tables_go<8, 9>(out, offC, offR);
         case 18: return mp_tables_go<9, 9>(out, offC, offR);
         case 19: return mp_tables_go<9, 10>(out, offC, offR);
-        case 20: return mp_tables_go<10, 10>(out, offC, offR);
-        case 21: return mp_tables_go<10, 11>(out, offC, offR);
+        case 20: return mp_tables_go<9, 11>(out, offC, offR);
+        case 21: return mp_tables_go<9, 12>(out, offC, offR);
         default: return false;
     }
 }

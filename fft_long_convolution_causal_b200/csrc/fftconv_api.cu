@@ -130,7 +130,7 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         p->workspace_bytes = 0;
     } else {
         p->path = fftc::PATH_MULTIPASS;
-        p->log2N1 = p->log2M / 2;
+        p->log2N1 = p->log2M / 2 < 9 ? p->log2M / 2 : 9;  // columns of at most 512 points (32 per CTA)
         p->log2N2 = p->log2M - p->log2N1;
         p->log2S = (p->log2M + 1) / 2;
         const int64_t S = int64_t(1) << p->log2S;
