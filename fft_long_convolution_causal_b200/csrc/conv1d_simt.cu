@@ -293,8 +293,9 @@ mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __rest
 
 // Pass 2.  MODE 0: forward row DFT, product with Khat (+D/M), inverse, conj
 // twiddle, in place.  MODE 1: forward row DFT only, Khat[k1][k2] = X / M.
+// Three CTAs of up to 256 threads per SM (at most 85 registers; no spills).
 template <int LOG2N1, int LOG2N2, int MODE>
-__global__ void __launch_bounds__(RowG<LOG2N2>::T)
+__global__ void __launch_bounds__(RowG<LOG2N2>::T, RowG<LOG2N2>::T <= 256 ? 3 : 1)
 mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __restrict__ khat_out,
          const float* __restrict__ D, const float2* __restrict__ twR, const float2* __restrict__ lo,
          const float2* __restrict__ hi, int log2S, int H, int64_t first) {
