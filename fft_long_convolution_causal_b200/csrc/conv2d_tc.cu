@@ -190,11 +190,14 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
     __syncthreads();
     if constexpr (BW) {
         // ---- W2 rows i: this tile's 64 bytes ([parity][re, im][8 k']); lane m of an
-        // 8-lane group writes 8 bytes: segment m / 2 (parity, re/im), k' = 4 (m & 1) .. + 3
+        // 8-lane group writes 8 bytes: segment m / 2 (parity, re/im), k' = 4 (m & 1) .. + 3.
+        // A warp takes rows i0 + {0, 2, 4, 6}: their swizzles differ in bits 1 and 2,
+        // so its 16 distinct tile reads fall in 16 distinct bank pairs.
         uint8_t* __restrict__ w2 = w1 + kW1Bytes + (size_t)(kx0 / kC2Cols) * 64;
 #pragma unroll 4
-        for (int q = tid; q < Hs * 8; q += 128) {
-            const int i = q >> 3, m = q & 7, seg = m >> 1, h = m & 1;
+        for (int it = 0; it < Hs / 16; ++it) {
+            const int i = 16 * it + (warp & 1) + 8 * (warp >> 1) + 2 * (lane >> 3);
+            const int m = lane & 7, seg = m >> 1, h = m & 1;
             const int parity = seg >> 1, im = seg & 1;
             float v[4];
 #pragma unroll
@@ -348,9 +351,10 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
     // ---- W2 rows i0 .. i0 + 15 (2 KiB each: [column tile][parity][re, im][8 k']) -> planes
     const uint8_t* __restrict__ w2 =
         reinterpret_cast<const uint8_t*>(work + (size_t)blockIdx.y * Hs * LR) + kW1Bytes + (size_t)i0 * 2048;
-    for (int q = tid; q < kC2RowsI * 128; q += 128) {
-        const int r = q >> 7, tile = (q >> 2) & 31, par = (q >> 1) & 1, pl = q & 1;
-        cp_async16(plane_addr(plane(par, pl), r, tile), w2 + (size_t)q * 16, 16);
+    // a warp copies 16 tiles of one (parity, re/im): 32 chunks over all 8 bank groups
+    for (int r = 0; r < kC2RowsI; ++r) {
+        const int tile = 16 * (warp & 1) + (lane >> 1), par = warp >> 1, pl = lane & 1;
+        cp_async16(plane_addr(plane(par, pl), r, tile), w2 + (size_t)r * 2048 + tile * 64 + par * 32 + pl * 16, 16);
     }
     cp_async_commit();
     uint2 f16[3][2], w256[4];
