@@ -124,10 +124,10 @@ __device__ __forceinline__ void inner_rows(uint32_t sre, uint32_t sim, const int
 // the staging planes x, times w when gated), times W_M^{q k_p}, stored
 // transposed into S[k_p][q].  Shared by the forward kernel and the spectrum
 // kernel of the largest transforms.
-template <int P, int NW, bool GATED, bool PRE1, bool IP, int F1, int F2>
+template <int P, int NW, bool GATED, bool PRE1, bool IP, bool RS, int F1, int F2>
 __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t wre, uint32_t wim, uint32_t sre,
                                             uint32_t sim, int lane, int warp, const uint2 (&fp)[F1][F2][3],
-                                            const TcTables& tb) {
+                                            const TcTables& tb, uint32_t rsm) {
     using S = TcShape<P>;
     constexpr bool TW_PREFETCH = S::NT1 <= 4;  // small tables: fetch the next tile's twiddles early
     const int m8 = lane >> 3, r8 = lane & 7;
@@ -141,6 +141,11 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
     }
     for (int qt = warp; qt < 16; qt += NW) {
         uint2 twc[TW_PREFETCH ? S::NT1 : 1][2];
+        uint2 tq0, tq1;  // otherwise: the next n-tile's twiddles, one tile ahead
+        if (!TW_PREFETCH) {
+            tq0 = __ldg(&tb.tw1[((qt * S::NT1) * 2 + 0) * 32 + lane]);
+            tq1 = __ldg(&tb.tw1[((qt * S::NT1) * 2 + 1) * 32 + lane]);
+        }
         if (TW_PREFETCH) {
 #pragma unroll
             for (int j = 0; j < S::NT1; ++j) {
@@ -187,8 +192,12 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
                 tw0 = twc[TW_PREFETCH ? j : 0][0];
                 tw1 = twc[TW_PREFETCH ? j : 0][1];
             } else {
-                tw0 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 0) * 32 + lane]);
-                tw1 = __ldg(&tb.tw1[((qt * S::NT1 + j) * 2 + 1) * 32 + lane]);
+                tw0 = tq0;
+                tw1 = tq1;
+                if (j + 1 < S::NT1) {
+                    tq0 = __ldg(&tb.tw1[((qt * S::NT1 + j + 1) * 2 + 0) * 32 + lane]);
+                    tq1 = __ldg(&tb.tw1[((qt * S::NT1 + j + 1) * 2 + 1) * 32 + lane]);
+                }
             }
             float yr[4], yi[4];
 #pragma unroll
@@ -198,6 +207,15 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
                     b0 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][0];
                     b1 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][1];
                     b2 = fp[PRE1 ? ks : 0][PRE1 ? j : 0][2];
+                } else if (RS) {
+                    // B[k = p][n = k_p] from the shared matrix rows k_p = 8 j + (0..7):
+                    // matrices (cos, p lo), (cos, p hi), (-sin, p lo), (-sin, p hi)
+                    uint32_t r[4];
+                    ldsm_x4(r, rsm + (uint32_t)((lane >> 4) * (P * P)) +
+                                   wr_off<P>(8 * j + (lane & 7), 2 * ks + ((lane >> 3) & 1)));
+                    b0 = make_uint2(r[0], r[1]);
+                    b1 = make_uint2(r[2], r[3]);
+                    b2 = make_uint2(r[2] ^ 0x80008000u, r[3] ^ 0x80008000u);
                 } else {
                     const uint2* fb = tb.fp + ((size_t)(ks * S::NT1 + j) * 3) * 32 + lane;
                     b0 = __ldg(fb);
@@ -300,6 +318,15 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
                         __ldg(&tb.fpi[((ks * S::NT3 + j) * 3 + part) * 32 + lane]);
     }
 
+    const uint32_t rsm = sre + SM::kROff;  // the outer DFT matrix (P >= 64)
+    if constexpr (SM::kRS) {
+        constexpr int RCH = P * P / 8;  // 16-byte chunks of both planes (P rows of P bytes each)
+        for (int i = tid; i < RCH; i += NT) {
+            const int plane = i / (RCH / 2), rem = i % (RCH / 2), r = rem / (P / 16), c = rem % (P / 16);
+            cp_async16(rsm + (uint32_t)(plane * (P * P)) + wr_off<P>(r, c), tb.wr + i, 16);
+        }
+        cp_async_commit();
+    }
     if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3, 0);
 
     int k = 0;  // items done by this CTA
@@ -320,7 +347,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         const uint32_t xre = xre0 + buf * SM::kX, xim = xre + SM::kX / 2;
 
         // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
-        outer_step1<P, NW, GATED, PRE1, IP>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb);
+        outer_step1<P, NW, GATED, PRE1, IP, SM::kRS>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb, rsm);
         __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
         if (SM::kNBuf == 1 && item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3, 0);
@@ -379,6 +406,15 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
                         b0 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][0];
                         b1 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][1];
                         b2 = fpi[PRE3 ? ks : 0][PRE3 ? j : 0][2];
+                    } else if (SM::kRS) {
+                        // B[k = k_p][n = p] = conj(W_P^{k_p p}): the shared matrix transposed,
+                        // rows k_p = 16 ks + (0..15), chunk j (p = 8 j + 0..7)
+                        uint32_t r[4];
+                        ldsm_x4_t(r, rsm + (uint32_t)((lane >> 4) * (P * P)) +
+                                         wr_off<P>(16 * ks + 8 * ((lane >> 3) & 1) + (lane & 7), j));
+                        b0 = make_uint2(r[0], r[1]);                                    // cos
+                        b1 = make_uint2(r[2] ^ 0x80008000u, r[3] ^ 0x80008000u);        // +sin
+                        b2 = make_uint2(r[2], r[3]);                                    // -sin
                     } else {
                         const uint2* fb = tb.fpi + ((size_t)(ks * S::NT3 + j) * 3) * 32 + lane;
                         b0 = __ldg(fb);
@@ -494,7 +530,7 @@ tc_spectrum_mma(const float* __restrict__ k, int L, uint4* __restrict__ khat, Tc
                      : "memory");
     }
     __syncthreads();
-    outer_step1<P, NW, false, PRE1, true>(xre, xim, 0u, 0u, sre, sim, lane, warp, fp, tb);
+    outer_step1<P, NW, false, PRE1, true, false>(xre, xim, 0u, 0u, sre, sim, lane, warp, fp, tb, 0u);
     __syncthreads();
     const uint32_t a = r8 + 8 * (m8 >> 1), chunk = 2 * a + (m8 & 1);
     const float inv_m = 1.0f / (float)S::M;
@@ -616,7 +652,7 @@ void push_bfrags(std::vector<float2>& out, int ksteps, int ntiles, F value) {
 
 bool tc_supported(int log2M) { return log2M >= 12 && log2M <= 15; }
 
-bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]) {
+bool tc_tables(int log2M, std::vector<float2>& out, size_t off[7]) {
     if (!tc_supported(log2M)) return false;
     const int64_t M = int64_t(1) << log2M;
     const int P = (int)(M / 256);
@@ -687,6 +723,22 @@ bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]) {
                 cs((int64_t)(16 * (a0 + 1) + b) * kp, M, &cb, &sb);
                 push_u2(out, pack_host(ca, cb), pack_host(sa, sb));
             }
+    // wr (P >= 64): W_P^{k_p p} for k_p < P, p < P/2 as two bf16 planes, cos and -sin,
+    // rows k_p of P/2 values; 16-byte aligned (the kernels copy it to shared memory)
+    if (out.size() & 1) out.push_back(make_float2(0.f, 0.f));
+    off[6] = out.size();
+    if (P >= 64)
+        for (int plane = 0; plane < 2; ++plane)
+            for (int kp = 0; kp < P; ++kp)
+                for (int p0 = 0; p0 < P / 2; p0 += 4) {
+                    double v[4];
+                    for (int i = 0; i < 4; ++i) {
+                        double c, sn;
+                        cs((int64_t)kp * (p0 + i), P, &c, &sn);
+                        v[i] = plane ? -sn : c;
+                    }
+                    push_u2(out, pack_host(v[0], v[1]), pack_host(v[2], v[3]));
+                }
     return true;
 }
 

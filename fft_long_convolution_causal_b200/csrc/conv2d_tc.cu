@@ -465,7 +465,7 @@ bool c2tc_rows_supported(const fftconv_plan_s& p) { return p.tc2d && p.Ws == 256
 // (shared with the 1-D kernel's tables), W_512^{i} as packed bf16 pairs in
 // A-fragment order and as fp32 in accumulator order.
 bool c2tc_tables(std::vector<float2>& out, size_t off[4]) {
-    size_t o1[6];
+    size_t o1[7];
     if (!tc_tables(12, out, o1)) return false;
     off[0] = o1[0];
     off[1] = o1[1];

@@ -109,7 +109,7 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
     cudaGetDevice(&p->device);
     std::vector<float2> host;
     const int64_t M = int64_t(1) << p->log2M;
-    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[6] = {0, 0, 0, 0, 0, 0}, offU = 0;
+    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0;
     const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && !getenv("FFTCONV_NO_TC");
     if (use_tc) {
         p->path = fftc::PATH_FUSED_TC;
@@ -170,6 +170,7 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         p->tc.fpi = (const uint2*)(base + offTc[3]);
         p->tc.tw1 = (const uint2*)(base + offTc[4]);
         p->tc.tw3 = (const uint2*)(base + offTc[5]);
+        p->tc.wr = (const uint4*)(base + offTc[6]);
     }
     *out = p;
     return FFTCONV_OK;

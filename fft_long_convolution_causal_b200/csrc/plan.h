@@ -31,6 +31,7 @@ struct TcTablePtrs {
     const uint2* fpi = nullptr;   // [kstep][ntile][part 3][lane]   outer inverse, conj(W_P^{k_p p}), p < P/2
     const uint2* tw1 = nullptr;   // [qt 16][ntile][half 2][lane]   (cos, sin) of W_M^{q k_p}
     const uint2* tw3 = nullptr;   // [k_p][reg 4][lane]             (cos, sin) of W_M^{q k_p}, q = 16 a + b
+    const uint4* wr = nullptr;    // P >= 64: [plane 2][k_p][p < P/2] bf16 cos / -sin of W_P^{k_p p}
 };
 
 // Constant tables of the 2-D tensor-core column pass.
@@ -81,7 +82,7 @@ bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_
 
 // 1-D bf16 tensor-core fused path (2N in {4096, 8192, 16384}).
 bool tc_supported(int log2M);
-bool tc_tables(int log2M, std::vector<float2>& out, size_t off[6]);
+bool tc_tables(int log2M, std::vector<float2>& out, size_t off[7]);
 cudaError_t launch_tc_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s);
 cudaError_t launch_tc_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const void* khat,
                           const float* D, void* y, cudaStream_t s);

@@ -35,6 +35,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
 __device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
     asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0),
                  "r"(r1), "r"(r2), "r"(r3)
@@ -201,8 +206,22 @@ struct TcSmem {
     // Ungated transforms up to 2N = 8192 keep two staging buffers, used by
     // alternate items, so the next item's rows are requested one item earlier.
     static constexpr int kNBuf = (!GATED && P <= 32) ? 2 : 1;
-    static constexpr int kBytes = kS + kNBuf * kX * ((GATED && !kWInS) ? 2 : 1);
+    // P >= 64: the outer DFT matrix (two bf16 planes of P x P/2), after the
+    // staging buffers; its fragments are read with ldmatrix instead of from L2
+    static constexpr bool kRS = P >= 64;
+    static constexpr int kR = kRS ? 2 * P * P : 0;  // two planes of P rows x P bytes
+    static constexpr int kROff = kS + kNBuf * kX * ((GATED && !kWInS) ? 2 : 1);
+    static constexpr int kBytes = kROff + kR;
 };
+
+// Byte offset of the 16-byte chunk c of row r of one plane of the outer DFT
+// matrix (rows of P/2 bf16 = P/16 chunks), XOR-swizzled so that the 8 rows
+// of an 8 x 8 ldmatrix block fall in 8 distinct 16-byte bank groups.
+template <int P>
+__device__ __forceinline__ uint32_t wr_off(int r, int c) {
+    constexpr int CPR = P / 16;
+    return (uint32_t)(r * P + ((c ^ ((r * CPR / 8) & (CPR - 1))) * 16));
+}
 
 // fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
 // registers of the 16x16 A fragment they form.
