@@ -232,31 +232,37 @@ __device__ __forceinline__ int c2_rowpos(int r, int kx) { return r * 512 + (kx ^
 
 // Forward row pass (images of 256 x 256): rows i of the pair's two images
 // (real, imaginary part), 512-point DFT over j < 256 as two 256-point
-// Monarch DFTs (kx even: of x; kx odd: of x W_512^j) -> work[pair][i][kx].
-constexpr int kC2RowsF = 8;  // rows per CTA
+// Monarch DFTs (kx even: of x; kx odd: of x W_512^j) -> W1 of the pair.
+// Persistent: a CTA walks work items (8 rows of one pair; consecutive items
+// share the pair) with stride gridDim.x, staging the next item's rows with
+// cp.async into the other buffer while it transforms the current one.
+constexpr int kC2RowsF = 8;  // rows per work item
 __global__ void __launch_bounds__(128, 4)
 c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2TcTables tb, int B, int C,
-              int64_t first) {
-    constexpr int Hs = 256, Ws = 256, LR = 512;
-    __shared__ __align__(128) uint8_t smem[2 * kC2RowsF * 512];   // re, im planes: row r, 256 j
-    __shared__ __align__(16) float2 otile[kC2RowsF * LR];          // row spectra before the coalesced store
+              int64_t first, int items) {
+    constexpr int Hs = 256, Ws = 256, LR = 512, RBLK = Hs / kC2RowsF;
+    __shared__ __align__(128) uint8_t smem[2][2 * kC2RowsF * 512];  // two staging buffers: re, im planes, rows r
+    __shared__ __align__(16) float2 otile[kC2RowsF * LR];           // row spectra before the W1 stores
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m8 = lane >> 3, r8 = lane & 7;
-    const int64_t P = first + blockIdx.y;
-    const int i0 = blockIdx.x * kC2RowsF;
     const int npp = (B + 1) / 2;
-    const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
-    const bool has1 = b0 + 1 < B;
-    const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
-    const uint32_t pre = smem_u32(smem), pim = pre + kC2RowsF * 512;
-    // ---- rows i0 .. i0 + 7 of both images -> planes (16-byte chunks)
-    for (int idx = tid; idx < 2 * kC2RowsF * 32; idx += 128) {
-        const int plane = idx / (kC2RowsF * 32), r = (idx / 32) % kC2RowsF, chunk = idx % 32;
-        const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing image
-        const size_t off = (plane ? (has1 ? img1 : img0) : img0) + (size_t)(i0 + r) * Ws + chunk * 8;
-        cp_async16(plane_addr(plane ? pim : pre, r, chunk), u + off, bytes);
-    }
-    cp_async_commit();
+    // rows i0 .. i0 + 7 of both images of the item's pair -> planes of buffer buf (16-byte chunks)
+    auto stage = [&](int item, int buf) {
+        const int64_t P = first + item / RBLK;
+        const int i0 = (item % RBLK) * kC2RowsF;
+        const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
+        const bool has1 = b0 + 1 < B;
+        const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
+        const uint32_t pre = smem_u32(smem[buf]), pim = pre + kC2RowsF * 512;
+        for (int idx = tid; idx < 2 * kC2RowsF * 32; idx += 128) {
+            const int plane = idx / (kC2RowsF * 32), r = (idx / 32) % kC2RowsF, chunk = idx % 32;
+            const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing image
+            const size_t off = (plane ? (has1 ? img1 : img0) : img0) + (size_t)(i0 + r) * Ws + chunk * 8;
+            cp_async16(plane_addr(plane ? pim : pre, r, chunk), u + off, bytes);
+        }
+        cp_async_commit();
+    };
+    if ((int)blockIdx.x < items) stage(blockIdx.x, 0);
     uint2 f16[3][2], w256[4], t512[4];
 #pragma unroll
     for (int part = 0; part < 3; ++part)
@@ -267,65 +273,79 @@ c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2
         w256[i] = __ldg(&tb.w256[i * 32 + lane]);
         t512[i] = __ldg(&tb.t512[i * 32 + lane]);
     }
-    cp_async_wait_all();
-    __syncthreads();
     const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
     const int g = lane >> 2, t = lane & 3;
+    int k = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++k) {
+        const int buf = k & 1;
+        if (item + (int)gridDim.x < items) {
+            // the other buffer was last read by the previous item (two barriers ago)
+            stage(item + gridDim.x, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        const uint32_t pre = smem_u32(smem[buf]), pim = pre + kC2RowsF * 512;
 #pragma unroll 1
-    for (int rr = 0; rr < kC2RowsF / 4; ++rr) {
-        const int r = 2 * warp + rr;
-        uint32_t xr[2][4], xi[2][4];
-        ldsm_x4_t(xr[0], plane_addr(pre, r, ichunk));
-        ldsm_x4_t(xi[0], plane_addr(pim, r, ichunk));
+        for (int rr = 0; rr < kC2RowsF / 4; ++rr) {
+            const int r = 2 * warp + rr;
+            uint32_t xr[2][4], xi[2][4];
+            ldsm_x4_t(xr[0], plane_addr(pre, r, ichunk));
+            ldsm_x4_t(xi[0], plane_addr(pim, r, ichunk));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xr[1][i] = xr[0][i];
-            xi[1][i] = xi[0][i];
-            twiddle2<true>(xr[1][i], xi[1][i], t512[i]);  // odd kx: x W_512^{j}
+            for (int i = 0; i < 4; ++i) {
+                xr[1][i] = xr[0][i];
+                xi[1][i] = xi[0][i];
+                twiddle2<true>(xr[1][i], xi[1][i], t512[i]);  // odd kx: x W_512^{j}
+            }
+            float acr[2][2][4], aci[2][2][4];
+#pragma unroll
+            for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                uint32_t tr[4], ti[4];
+                pack_tile(tr, acr[v]);
+                pack_tile(ti, aci[v]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
+                transpose_tile(xr[v], tr);
+                transpose_tile(xi[v], ti);
+            }
+#pragma unroll
+            for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
+            // accumulator (n, e) of unit v: c = g + 8 (e >> 1), d = 8 n + 2 t + (e & 1); kx = v + 2 (c + 16 d)
+#pragma unroll
+            for (int v = 0; v < 2; ++v)
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = g + 8 * (e >> 1), d = 8 * n + 2 * t + (e & 1);
+                        otile[c2_rowpos(r, v + 2 * (c + 16 * d))] = make_float2(acr[v][n][e], aci[v][n][e]);
+                    }
         }
-        float acr[2][2][4], aci[2][2][4];
+        __syncthreads();
+        // ---- W1[kx][row tile i0 / 8][re, im][8 rows]: 32 bytes per column kx
+        static_assert(kC2RowsF == 8, "one row tile of W1 per item");
+        uint8_t* __restrict__ w1 = reinterpret_cast<uint8_t*>(work + (size_t)(item / RBLK) * Hs * LR) +
+                                   (size_t)(item % RBLK) * 32;
 #pragma unroll
-        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
+        for (int kx = tid; kx < LR; kx += 128) {
+            float re[8], im[8];
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-            uint32_t tr[4], ti[4];
-            pack_tile(tr, acr[v]);
-            pack_tile(ti, aci[v]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) twiddle2<true>(tr[i], ti[i], w256[i]);
-            transpose_tile(xr[v], tr);
-            transpose_tile(xi[v], ti);
+            for (int r = 0; r < 8; ++r) {
+                const float2 z = otile[c2_rowpos(r, kx)];
+                re[r] = z.x;
+                im[r] = z.y;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(w1 + (size_t)kx * 1024);
+            dst[0] = make_uint4(pack2(re[0], re[1]), pack2(re[2], re[3]), pack2(re[4], re[5]), pack2(re[6], re[7]));
+            dst[1] = make_uint4(pack2(im[0], im[1]), pack2(im[2], im[3]), pack2(im[4], im[5]), pack2(im[6], im[7]));
         }
-#pragma unroll
-        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[1], f16[2]);
-        // accumulator (n, e) of unit v: c = g + 8 (e >> 1), d = 8 n + 2 t + (e & 1); kx = v + 2 (c + 16 d)
-#pragma unroll
-        for (int v = 0; v < 2; ++v)
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = g + 8 * (e >> 1), d = 8 * n + 2 * t + (e & 1);
-                    otile[c2_rowpos(r, v + 2 * (c + 16 * d))] = make_float2(acr[v][n][e], aci[v][n][e]);
-                }
+        // the next item's wait + barrier orders these reads before otile is rewritten
     }
-    __syncthreads();
-    // ---- W1[kx][row tile i0 / 8][re, im][8 rows]: 32 bytes per column kx
-    static_assert(kC2RowsF == 8, "one row tile of W1 per CTA");
-    uint8_t* __restrict__ w1 = reinterpret_cast<uint8_t*>(work + (size_t)blockIdx.y * Hs * LR) + (size_t)(i0 / 8) * 32;
-#pragma unroll
-    for (int kx = tid; kx < LR; kx += 128) {
-        float re[8], im[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float2 z = otile[c2_rowpos(r, kx)];
-            re[r] = z.x;
-            im[r] = z.y;
-        }
-        uint4* dst = reinterpret_cast<uint4*>(w1 + (size_t)kx * 1024);
-        dst[0] = make_uint4(pack2(re[0], re[1]), pack2(re[2], re[3]), pack2(re[4], re[5]), pack2(re[6], re[7]));
-        dst[1] = make_uint4(pack2(im[0], im[1]), pack2(im[2], im[3]), pack2(im[4], im[5]), pack2(im[6], im[7]));
-    }
+    cp_async_wait_all();
 }
 
 // Inverse row pass (images of 256 x 256): work[pair][i][kx] -> 512-point
@@ -512,8 +532,18 @@ static cudaError_t c2tc_go(const fftconv_plan_s& p, float2* work, const void* kh
 
 cudaError_t launch_c2tc_rows_fwd(const fftconv_plan_s& p, const void* u, float2* work, int g, int64_t first,
                                  cudaStream_t s) {
-    tc::c2tc_rows_fwd<<<dim3(256 / tc::kC2RowsF, g), 128, 0, s>>>((const __nv_bfloat16*)u, work, p.c2tc, p.B, p.H,
-                                                                  first);
+    // persistent grid: as many CTAs as are resident at once (computed once)
+    static int resident = 0;
+    if (resident == 0) {
+        int per_sm = 0, sms = 0, dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::c2tc_rows_fwd, 128, 0);
+        resident = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    }
+    const int items = (256 / tc::kC2RowsF) * g;
+    tc::c2tc_rows_fwd<<<items < resident ? items : resident, 128, 0, s>>>((const __nv_bfloat16*)u, work, p.c2tc, p.B,
+                                                                          p.H, first, items);
     return cudaGetLastError();
 }
 
