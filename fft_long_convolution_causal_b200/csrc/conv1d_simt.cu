@@ -223,8 +223,11 @@ using ColG = Geometry<LOG2N1, kColTile<LOG2N1>, true>;
 // most 16 rows), so short rows do not leave single-warp CTAs.
 constexpr int row_batch(int log2n2) { return log2n2 >= 12 ? 1 : ((4096 >> log2n2) > 16 ? 16 : (4096 >> log2n2)); }
 
+// One row per CTA (2^12 points and up): a pad slot every 16 values, so the
+// first stage's writes (16 consecutive outputs per thread, stride 16 across
+// the lanes) land in distinct bank pairs; several rows: every 32.
 template <int LOG2N2>
-using RowG = Geometry<LOG2N2, row_batch(LOG2N2), false>;
+using RowG = Geometry<LOG2N2, row_batch(LOG2N2), false, row_batch(LOG2N2) == 1 ? 4 : 5>;
 
 // Outputs per exact twiddle lookup in the pass epilogues; in between the
 // twiddle is advanced by one fp32 complex product (at most kTwRun - 1 chained

@@ -133,14 +133,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 
 // ------------------------------------------------------------ smem layout
 // L-point transforms of C columns.  BF (batch-fast): element (i, c) at i*C + c;
-// otherwise at c*L + i.  One pad slot per 32 complex values breaks the bank
-// conflicts of the strided Stockham writes.
-template <int L, int C, bool BF>
+// otherwise at c*L + i.  One pad slot per 2^PADSH complex values (default 32)
+// breaks the bank conflicts of the strided Stockham writes.
+template <int L, int C, bool BF, int PADSH = 5>
 struct Layout {
-    static constexpr int kWords = L * C + (L * C) / 32;  // float2 slots
+    static constexpr int kWords = L * C + ((L * C) >> PADSH);  // float2 slots
     static __device__ __forceinline__ int at(int i, int c) {
         const int x = BF ? i * C + c : c * L + i;
-        return x + (x >> 5);
+        return x + (x >> PADSH);
     }
 };
 
@@ -156,7 +156,7 @@ struct RadixPlan {
 };
 
 // Geometry of a batched transform: L points x C columns on T threads.
-template <int LOG2L_, int C_, bool BF_>
+template <int LOG2L_, int C_, bool BF_, int PADSH_ = 5>
 struct Geometry {
     static constexpr int LOG2L = LOG2L_;
     static constexpr int L = 1 << LOG2L_;
@@ -169,7 +169,7 @@ struct Geometry {
     static constexpr int T = (kTotal / 16) < 32 ? 32 : ((kTotal / 16) > 512 ? 512 : (kTotal / 16));
     static constexpr int LOG2E = ilog2(kTotal / T);
     using Plan = RadixPlan<LOG2L, LOG2E>;
-    using Lay = Layout<L, C, BF>;
+    using Lay = Layout<L, C, BF, PADSH_>;
 };
 
 // Twiddles of every stage of a geometry, one table: stage s holds
