@@ -348,35 +348,38 @@ c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2
     cp_async_wait_all();
 }
 
-// Inverse row pass (images of 256 x 256): work[pair][i][kx] -> 512-point
+// Inverse row pass (images of 256 x 256): W2 of the pair -> 512-point
 // inverse DFT over kx keeping j < 256, as two 256-point Monarch inverses
 // (kx even, kx odd) recombined with W_512^{-j} -> y rows of both images.
-constexpr int kC2RowsI = 16;  // rows per CTA
+// Persistent like the forward row pass: work items of 8 rows, the next
+// item's W2 rows staged with cp.async into the other buffer.
+constexpr int kC2RowsI = 8;  // rows per work item
 __global__ void __launch_bounds__(128, 4)
 c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2TcTables tb, int B, int C,
-              int64_t first) {
-    constexpr int Hs = 256, Ws = 256, LR = 512;
-    // planes (row r, 256 k'): [parity][re, im]; then y planes (row r, 256 j) [image]
-    __shared__ __align__(128) uint8_t smem[4 * kC2RowsI * 512 + 2 * kC2RowsI * 512];
+              int64_t first, int items) {
+    constexpr int Hs = 256, Ws = 256, LR = 512, RBLK = Hs / kC2RowsI;
+    // two staging buffers of planes (row r, 256 k'): [parity][re, im]; then y planes (row r, 256 j) [image]
+    __shared__ __align__(128) uint8_t smem[2 * 4 * kC2RowsI * 512 + 2 * kC2RowsI * 512];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m8 = lane >> 3, r8 = lane & 7;
-    const int64_t P = first + blockIdx.y;
-    const int i0 = blockIdx.x * kC2RowsI;
     const int npp = (B + 1) / 2;
-    const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
-    const bool has1 = b0 + 1 < B;
     const uint32_t base = smem_u32(smem);
-    auto plane = [&](int par, int im) { return base + (uint32_t)((2 * par + im) * kC2RowsI * 512); };
-    const uint32_t y0p = base + 4 * kC2RowsI * 512, y1p = y0p + kC2RowsI * 512;
-    // ---- W2 rows i0 .. i0 + 15 (2 KiB each: [column tile][parity][re, im][8 k']) -> planes
-    const uint8_t* __restrict__ w2 =
-        reinterpret_cast<const uint8_t*>(work + (size_t)blockIdx.y * Hs * LR) + kW1Bytes + (size_t)i0 * 2048;
+    auto plane = [&](int buf, int par, int im) {
+        return base + (uint32_t)((buf * 4 + 2 * par + im) * kC2RowsI * 512);
+    };
+    const uint32_t y0p = base + 8 * kC2RowsI * 512, y1p = y0p + kC2RowsI * 512;
+    // W2 rows i0 .. i0 + 7 of the item's pair (2 KiB each: [column tile][parity][re, im][8 k']) -> buffer buf;
     // a warp copies 16 tiles of one (parity, re/im): 32 chunks over all 8 bank groups
-    for (int r = 0; r < kC2RowsI; ++r) {
+    auto stage = [&](int item, int buf) {
+        const uint8_t* __restrict__ w2 = reinterpret_cast<const uint8_t*>(work + (size_t)(item / RBLK) * Hs * LR) +
+                                         kW1Bytes + (size_t)(item % RBLK) * kC2RowsI * 2048;
         const int tile = 16 * (warp & 1) + (lane >> 1), par = warp >> 1, pl = lane & 1;
-        cp_async16(plane_addr(plane(par, pl), r, tile), w2 + (size_t)r * 2048 + tile * 64 + par * 32 + pl * 16, 16);
-    }
-    cp_async_commit();
+        for (int r = 0; r < kC2RowsI; ++r)
+            cp_async16(plane_addr(plane(buf, par, pl), r, tile), w2 + (size_t)r * 2048 + tile * 64 + par * 32 + pl * 16,
+                       16);
+        cp_async_commit();
+    };
+    if ((int)blockIdx.x < items) stage(blockIdx.x, 0);
     uint2 f16[3][2], w256[4];
     float2 tz[2][4];
 #pragma unroll
@@ -389,64 +392,80 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
     for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tz[j][e] = __ldg(&tb.t512f[(j * 4 + e) * 32 + lane]);
-    cp_async_wait_all();
-    __syncthreads();
     const uint32_t ia = r8 + 8 * (m8 >> 1), ichunk = 2 * ia + (m8 & 1);
+    int k = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++k) {
+        const int buf = k & 1;
+        if (item + (int)gridDim.x < items) {
+            // the other buffer was last read by the previous item (two barriers ago)
+            stage(item + gridDim.x, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            cp_async_wait_all();
+        }
+        __syncthreads();
 #pragma unroll 1
-    for (int rr = 0; rr < kC2RowsI / 4; ++rr) {
-        const int r = 4 * warp + rr;
-        // A = [c][d], k' = c + 16 d, of the even and odd columns
-        uint32_t xr[2][4], xi[2][4];
+        for (int rr = 0; rr < kC2RowsI / 4; ++rr) {
+            const int r = 2 * warp + rr;
+            // A = [c][d], k' = c + 16 d, of the even and odd columns
+            uint32_t xr[2][4], xi[2][4];
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-            ldsm_x4_t(xr[v], plane_addr(plane(v, 0), r, ichunk));
-            ldsm_x4_t(xi[v], plane_addr(plane(v, 1), r, ichunk));
-        }
-        float acr[2][2][4], aci[2][2][4];
-        // [c][d] x conj(F16) -> [c][b]; transpose -> [b][c]; x W_256^{-b c}; x conj(F16) -> [b][a]
-#pragma unroll
-        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-            uint32_t gr[4], gi[4];
-            pack_tile(gr, acr[v]);
-            pack_tile(gi, aci[v]);
-            transpose_tile(xr[v], gr);
-            transpose_tile(xi[v], gi);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) twiddle2<false>(xr[v][i], xi[v][i], w256[i]);
-        }
-#pragma unroll
-        for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
-        // z[j] = Z_even[j] + W_512^{-j} Z_odd[j]: re -> image b0, im -> image b0 + 1
-        float zr[2][4], zi[2][4];
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 w = tz[n][e];
-                const float orr = acr[1][n][e], oi = aci[1][n][e];
-                zr[n][e] = acr[0][n][e] + fmaf(orr, w.x, -oi * w.y);
-                zi[n][e] = aci[0][n][e] + fmaf(oi, w.x, orr * w.y);
+            for (int v = 0; v < 2; ++v) {
+                ldsm_x4_t(xr[v], plane_addr(plane(buf, v, 0), r, ichunk));
+                ldsm_x4_t(xi[v], plane_addr(plane(buf, v, 1), r, ichunk));
             }
-        uint32_t pr[4], pi[4];
-        pack_tile(pr, zr);
-        pack_tile(pi, zi);
-        stsm_x4_t(plane_addr(y0p, r, ichunk), pr[0], pr[1], pr[2], pr[3]);
-        stsm_x4_t(plane_addr(y1p, r, ichunk), pi[0], pi[1], pi[2], pi[3]);
+            float acr[2][2][4], aci[2][2][4];
+            // [c][d] x conj(F16) -> [c][b]; transpose -> [b][c]; x W_256^{-b c}; x conj(F16) -> [b][a]
+#pragma unroll
+            for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                uint32_t gr[4], gi[4];
+                pack_tile(gr, acr[v]);
+                pack_tile(gi, aci[v]);
+                transpose_tile(xr[v], gr);
+                transpose_tile(xi[v], gi);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) twiddle2<false>(xr[v][i], xi[v][i], w256[i]);
+            }
+#pragma unroll
+            for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
+            // z[j] = Z_even[j] + W_512^{-j} Z_odd[j]: re -> image b0, im -> image b0 + 1
+            float zr[2][4], zi[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 w = tz[n][e];
+                    const float orr = acr[1][n][e], oi = aci[1][n][e];
+                    zr[n][e] = acr[0][n][e] + fmaf(orr, w.x, -oi * w.y);
+                    zi[n][e] = aci[0][n][e] + fmaf(oi, w.x, orr * w.y);
+                }
+            uint32_t pr[4], pi[4];
+            pack_tile(pr, zr);
+            pack_tile(pi, zi);
+            stsm_x4_t(plane_addr(y0p, r, ichunk), pr[0], pr[1], pr[2], pr[3]);
+            stsm_x4_t(plane_addr(y1p, r, ichunk), pi[0], pi[1], pi[2], pi[3]);
+        }
+        __syncthreads();
+        // ---- y rows i0 .. i0 + 7 of both images, 16-byte chunks
+        const int64_t P = first + item / RBLK;
+        const int i0 = (item % RBLK) * kC2RowsI;
+        const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
+        const bool has1 = b0 + 1 < B;
+        const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
+        for (int idx = tid; idx < 2 * kC2RowsI * 32; idx += 128) {
+            const int im = idx / (kC2RowsI * 32), r = (idx / 32) % kC2RowsI, chunk = idx % 32;
+            if (im == 1 && !has1) continue;
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(plane_addr(im ? y1p : y0p, r, chunk)));
+            *reinterpret_cast<uint4*>(y + (im ? img1 : img0) + (size_t)(i0 + r) * Ws + chunk * 8) = val;
+        }
+        // the next item's wait + barrier orders these reads before the y planes are rewritten
     }
-    __syncthreads();
-    // ---- y rows i0 .. i0 + 15 of both images, 16-byte chunks
-    const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
-    for (int idx = tid; idx < 2 * kC2RowsI * 32; idx += 128) {
-        const int im = idx / (kC2RowsI * 32), r = (idx / 32) % kC2RowsI, chunk = idx % 32;
-        if (im == 1 && !has1) continue;
-        uint4 val;
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
-                     : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                     : "r"(plane_addr(im ? y1p : y0p, r, chunk)));
-        *reinterpret_cast<uint4*>(y + (im ? img1 : img0) + (size_t)(i0 + r) * Ws + chunk * 8) = val;
-    }
+    cp_async_wait_all();
 }
 
 }  // namespace tc
@@ -549,7 +568,17 @@ cudaError_t launch_c2tc_rows_fwd(const fftconv_plan_s& p, const void* u, float2*
 
 cudaError_t launch_c2tc_rows_inv(const fftconv_plan_s& p, const float2* work, void* y, int g, int64_t first,
                                  cudaStream_t s) {
-    tc::c2tc_rows_inv<<<dim3(256 / tc::kC2RowsI, g), 128, 0, s>>>(work, (__nv_bfloat16*)y, p.c2tc, p.B, p.H, first);
+    static int resident = 0;  // persistent grid, as for the forward row pass
+    if (resident == 0) {
+        int per_sm = 0, sms = 0, dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::c2tc_rows_inv, 128, 0);
+        resident = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    }
+    const int items = (256 / tc::kC2RowsI) * g;
+    tc::c2tc_rows_inv<<<items < resident ? items : resident, 128, 0, s>>>(work, (__nv_bfloat16*)y, p.c2tc, p.B, p.H,
+                                                                          first, items);
     return cudaGetLastError();
 }
 
