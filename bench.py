@@ -18,7 +18,8 @@ rows are independent so no collective is on the data path).
 
 e2e: the same step through the public API from pinned host buffers, with the
 host->device copy of the inputs and the device->host copy of y inside the
-timed region.
+timed region; steps alternate between two streams with their own buffers, so
+one step's input copy overlaps the previous step's output copy.
 
 cpu_baseline (rank 0, N=1): the CPU fp64 oracle, as it stands, on a bounded
 uniform sample of the same workload's outputs.
@@ -199,14 +200,15 @@ class Runner:
         self.ws = self.plan.new_workspace()
         torch.cuda.synchronize()
 
-    def step(self, y=None, u=None, v=None, w=None):
+    def step(self, y=None, u=None, v=None, w=None, ws=None):
         y = self.y if y is None else y
         u = self.u if u is None else u
+        ws = self.ws if ws is None else ws
         if self.is2d:
-            self.plan.fwd(u, self.khat, y=y, workspace=self.ws)
+            self.plan.fwd(u, self.khat, y=y, workspace=ws)
         else:
             self.plan.fwd(u, self.khat, D=self.D, v=self.v if v is None else v, w=self.w if w is None else w,
-                          y=y, workspace=self.ws)
+                          y=y, workspace=ws)
 
     def launches_per_step(self):
         if self.plan.path in ("fused", "fused_tc", "fused_umma"):
@@ -243,37 +245,50 @@ def time_steps(r, steps, torch, flush):
 
 
 def time_e2e(r, steps, torch):
-    """Host buffers in, host buffer out, copies inside the timed region."""
-    wl = r.wl
+    """Host buffers in, host buffer out, copies inside the timed region.
+
+    Steps alternate between two CUDA streams, each with its own device
+    buffers, workspace and pinned output buffer (double buffering, as a
+    streaming caller would run it): step i+1's host-to-device copy overlaps
+    step i's device-to-host copy on the full-duplex link.  Every step still
+    copies all of its inputs in and its whole result out."""
     pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
     hu, hv, hw = pin(r.u), pin(r.v), pin(r.w)
-    hy = torch.empty(r.y.shape, dtype=r.y.dtype).pin_memory()
-    du, dy = torch.empty_like(r.u), torch.empty_like(r.y)
-    dv = None if r.v is None else torch.empty_like(r.v)
-    dw = None if r.w is None else torch.empty_like(r.w)
-    stream = torch.cuda.current_stream()
     h2d = sum(t.numel() * t.element_size() for t in (hu, hv, hw) if t is not None)
-    d2h = hy.numel() * hy.element_size()
-
-    def one():
-        du.copy_(hu, non_blocking=True)
-        if dv is not None:
-            dv.copy_(hv, non_blocking=True)
-            dw.copy_(hw, non_blocking=True)
-        r.step(y=dy, u=du, v=dv, w=dw)
-        hy.copy_(dy, non_blocking=True)
-
+    sets = []
     for _ in range(2):
-        one()
+        sets.append(dict(
+            du=torch.empty_like(r.u), dy=torch.empty_like(r.y),
+            dv=None if r.v is None else torch.empty_like(r.v), dw=None if r.w is None else torch.empty_like(r.w),
+            ws=r.plan.new_workspace(), hy=torch.empty(r.y.shape, dtype=r.y.dtype).pin_memory(),
+            stream=torch.cuda.Stream()))
+    d2h = sets[0]["hy"].numel() * sets[0]["hy"].element_size()
+    main = torch.cuda.current_stream()
+
+    def one(i):
+        b = sets[i % 2]
+        with torch.cuda.stream(b["stream"]):
+            b["du"].copy_(hu, non_blocking=True)
+            if b["dv"] is not None:
+                b["dv"].copy_(hv, non_blocking=True)
+                b["dw"].copy_(hw, non_blocking=True)
+            r.step(y=b["dy"], u=b["du"], v=b["dv"], w=b["dw"], ws=b["ws"])
+            b["hy"].copy_(b["dy"], non_blocking=True)
+
+    for i in range(4):
+        one(i)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(main)
+    for b in sets:
+        b["stream"].wait_event(a)
+    for i in range(steps):
+        one(i)
+    for b in sets:
+        main.wait_stream(b["stream"])
+    e.record(main)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    del wl
+    ms = a.elapsed_time(e) / steps
     return ms, h2d, d2h
 
 
