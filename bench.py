@@ -18,8 +18,9 @@ rows are independent so no collective is on the data path).
 
 e2e: the same step through the public API from pinned host buffers, with the
 host->device copy of the inputs and the device->host copy of y inside the
-timed region; steps alternate between two streams with their own buffers, so
-one step's input copy overlaps the previous step's output copy.
+timed region; steps of 1 MiB of input or more alternate between two streams
+with their own buffers, so one step's input copy overlaps the previous step's
+output copy.
 
 cpu_baseline (rank 0, N=1): the CPU fp64 oracle, as it stands, on a bounded
 uniform sample of the same workload's outputs.
@@ -247,26 +248,29 @@ def time_steps(r, steps, torch, flush):
 def time_e2e(r, steps, torch):
     """Host buffers in, host buffer out, copies inside the timed region.
 
-    Steps alternate between two CUDA streams, each with its own device
-    buffers, workspace and pinned output buffer (double buffering, as a
-    streaming caller would run it): step i+1's host-to-device copy overlaps
-    step i's device-to-host copy on the full-duplex link.  Every step still
-    copies all of its inputs in and its whole result out."""
+    Steps of at least 1 MiB of input alternate between two CUDA streams,
+    each with its own device buffers, workspace and pinned output buffer
+    (double buffering, as a streaming caller would run it): step i+1's
+    host-to-device copy overlaps step i's device-to-host copy on the
+    full-duplex link.  Smaller steps, bound by per-call latency, run on the
+    current stream alone.  Every step copies all of its inputs in and its
+    whole result out."""
     pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
     hu, hv, hw = pin(r.u), pin(r.v), pin(r.w)
     h2d = sum(t.numel() * t.element_size() for t in (hu, hv, hw) if t is not None)
+    main = torch.cuda.current_stream()
+    nsets = 2 if h2d >= (1 << 20) else 1
     sets = []
-    for _ in range(2):
+    for _ in range(nsets):
         sets.append(dict(
             du=torch.empty_like(r.u), dy=torch.empty_like(r.y),
             dv=None if r.v is None else torch.empty_like(r.v), dw=None if r.w is None else torch.empty_like(r.w),
             ws=r.plan.new_workspace(), hy=torch.empty(r.y.shape, dtype=r.y.dtype).pin_memory(),
-            stream=torch.cuda.Stream()))
+            stream=torch.cuda.Stream() if nsets > 1 else main))
     d2h = sets[0]["hy"].numel() * sets[0]["hy"].element_size()
-    main = torch.cuda.current_stream()
 
     def one(i):
-        b = sets[i % 2]
+        b = sets[i % nsets]
         with torch.cuda.stream(b["stream"]):
             b["du"].copy_(hu, non_blocking=True)
             if b["dv"] is not None:
@@ -281,11 +285,13 @@ def time_e2e(r, steps, torch):
     a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(main)
     for b in sets:
-        b["stream"].wait_event(a)
+        if b["stream"] is not main:
+            b["stream"].wait_event(a)
     for i in range(steps):
         one(i)
     for b in sets:
-        main.wait_stream(b["stream"])
+        if b["stream"] is not main:
+            main.wait_stream(b["stream"])
     e.record(main)
     torch.cuda.synchronize()
     ms = a.elapsed_time(e) / steps
