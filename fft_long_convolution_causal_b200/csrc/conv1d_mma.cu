@@ -38,6 +38,7 @@
 #include "plan.h"
 #include "tables.h"
 #include "tc_common.cuh"
+#include "umma.cuh"
 
 namespace fftc {
 namespace tc {
@@ -237,6 +238,102 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
     }
 }
 
+// Step 1 for P = 128 on tcgen05: for each 128-row tile t of q, the complex
+// product D[q][k_p] = X[q][p] W_128^{p k_p} over the 64 nonzero p as real
+// products with W = C + i F (C = cos, F = -sin: the two stored planes):
+// D_re = X_re C - X_im F (the negate-B bit), D_im = X_re F + X_im C; A = the staging planes
+// (MN-major), B = the outer DFT matrix (K-major), fp32 accumulators in TMEM
+// columns 256 t + 128 part.  Then every warp reads its quarter of the lanes
+// (tile warp / 4 % 2, column half warp / 8) in the mma.sync accumulator
+// layout, multiplies by W_M^{q k_p} on packed pairs and stores transposed
+// into S[k_p][q], as the mma.sync step 1 does.  Returns false when the wait
+// for the products gave up.
+template <int NW, bool IP>
+__device__ __forceinline__ bool outer_step1_umma(uint32_t xre, uint32_t xim, uint32_t rsm, uint32_t sre, uint32_t sim,
+                                                 uint32_t tmem, uint32_t mbar, uint32_t phase, int tid, int lane,
+                                                 int warp, const TcTables& tb) {
+    constexpr int P = 128;
+    static_assert(NW == 16, "one warp per (tile, lane quarter, column half)");
+    if (tid == 0) {
+        um::fence_after();
+        const uint32_t id = um::idesc_bf16(128, 128) | (1u << 15);  // A MN-major
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int xi = 0; xi < 2; ++xi) {
+                        // (part, x plane) -> B plane and sign: re: (re, C) (im, -F); im: (re, F) (im, C)
+                        const int bplane = (part ^ xi) & 1;
+                        const uint32_t neg = (part == 0 && xi == 1) ? (1u << 14) : 0u;
+                        const uint32_t a = (xi ? xim : xre) + (uint32_t)(16 * t * 1024 + 2 * ks * 128);
+                        const uint32_t b = rsm + (uint32_t)(bplane * P * P + 2 * ks * 128);
+                        const uint64_t ad = (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) |
+                                            ((uint64_t)(1024u >> 4) << 32) | (1ull << 46);
+                        const uint64_t bd = (uint64_t)((b >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) |
+                                            ((uint64_t)(1024u >> 4) << 32) | (1ull << 46);
+                        asm volatile(
+                            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                                tmem + (uint32_t)(256 * t + 128 * part)),
+                            "l"(ad), "l"(bd), "r"(id | neg), "r"((uint32_t)(ks | xi)));
+                    }
+            um::mma_commit(mbar + 8u * t);  // each tile's products on their own barrier
+        }
+    }
+    const int t = (warp >> 2) & 1, qr = warp & 3, ch = warp >> 3;
+    const int m8 = lane >> 3, r8 = lane & 7;
+    // twiddles W_M^{q k_p} of the 4 blocks of iteration it (rg = it / 2, jh = it % 2), fetched one iteration ahead
+    uint2 tw[4][2];
+    auto fetch_tw = [&](int it) {
+        const int qt = 8 * t + 2 * qr + (it >> 1);
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+            const int j = 8 * ch + 4 * (it & 1) + jb;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) tw[jb][hh] = __ldg(&tb.tw1[((qt * 16 + j) * 2 + hh) * 32 + lane]);
+        }
+    };
+    fetch_tw(0);
+    const bool ok = um::mbar_wait(mbar + 8u * t, phase);
+    um::fence_after();
+#pragma unroll 1
+    for (int it = 0; it < 4; ++it) {
+        const int rg = it >> 1, jh = it & 1;
+        const int qt = 8 * t + 2 * qr + rg;  // 16-row tile of q
+        const uint32_t lrow = (uint32_t)(32 * qr + 16 * rg) << 16;
+        uint32_t dr[16], di[16];
+        const uint32_t col = (uint32_t)(256 * t + 64 * ch + 32 * jh);
+        um::ld16x256<4>(tmem + lrow + col, dr);
+        um::ld16x256<4>(tmem + lrow + col + 128, di);
+        uint2 twc[4][2];
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+            twc[jb][0] = tw[jb][0];
+            twc[jb][1] = tw[jb][1];
+        }
+        if (it + 1 < 4) fetch_tw(it + 1);
+        um::wait_ld<16>(dr);
+        um::wait_ld<16>(di);
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+            const int j = 8 * ch + 4 * jh + jb;  // 8-column block of k_p
+            const float* yr = reinterpret_cast<const float*>(&dr[4 * jb]);
+            const float* yi = reinterpret_cast<const float*>(&di[4 * jb]);
+            uint32_t pr[2] = {pack2<IP>(yr[0], yr[1]), pack2<IP>(yr[2], yr[3])};
+            uint32_t pi[2] = {pack2<IP>(yi[0], yi[1]), pack2<IP>(yi[2], yi[3])};
+            twiddle2<true>(pr[0], pi[0], twc[jb][0]);
+            twiddle2<true>(pr[1], pi[1], twc[jb][1]);
+            const uint32_t krow = 8 * j + r8, chunk = 2 * qt + (m8 & 1);
+            stsm_x4_t(plane_addr((m8 >> 1) ? sim : sre, krow, chunk), pr[0], pr[1], pi[0], pi[1]);
+        }
+    }
+    um::fence_before();
+    return ok;
+}
+
 // Persistent: each CTA walks work items (pair pp of channel h) with stride
 // gridDim.x; items of one channel are consecutive so concurrent CTAs share
 // Khat[h] in L2.  The next item's input is fetched with cp.async into the
@@ -245,7 +342,7 @@ template <int P, int NW, bool GATED>
 __global__ void __launch_bounds__(NW * 32, P <= 32 ? 3 : (P <= 64 ? 2 : 1))
 fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
              const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
-             __nv_bfloat16* __restrict__ y, TcTables tb, int B, int H) {
+             __nv_bfloat16* __restrict__ y, TcTables tb, int* __restrict__ err, int B, int H) {
     using S = TcShape<P>;
     using SM = TcSmem<P, GATED>;
     static_assert(P >= 16 && P <= 128, "outer factor");
@@ -274,11 +371,24 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         const size_t r0 = ((size_t)b0 * H + hh) * S::N;
         const size_t r1 = has1 ? ((size_t)(b0 + 1) * H + hh) * S::N : r0;
         for (int i = tid; i < 2 * CH; i += NT) {
-            const int plane = i / CH, n0 = (i % CH) * 8;
-            const uint32_t p = n0 >> 8, chunk = (n0 & 255) >> 3;
+            const int plane = i / CH;
+            uint32_t p, chunk;
+            if (SM::kUM1) {
+                // a warp takes rows p0 .. p0 + 7 x chunks c0 .. c0 + 3: 64-byte global
+                // runs, and 8 distinct bank groups in the canonical layout
+                const int rem = i % CH;
+                chunk = (rem >> 8) * 4 + ((rem & 31) >> 3);
+                p = ((rem >> 5) & 7) * 8 + (rem & 7);
+            } else {
+                const int n0 = (i % CH) * 8;
+                p = n0 >> 8;
+                chunk = (n0 & 255) >> 3;
+            }
             const int bytes = (plane == 0 || has1) ? 16 : 0;  // zero-fill the missing row
-            const size_t off = (plane ? r1 : r0) + n0;
-            if (which & 1) cp_async16(plane_addr(plane ? xim : xre, p, chunk), u + off, bytes);
+            const size_t off = (plane ? r1 : r0) + 256 * p + 8 * chunk;
+            if (which & 1)
+                cp_async16(SM::kUM1 ? (plane ? xim : xre) + xcan_off(p, chunk) : plane_addr(plane ? xim : xre, p, chunk),
+                           u + off, bytes);
             if (GATED && (which & 2)) cp_async16(plane_addr(plane ? wim : wre, p, chunk), w + off, bytes);
         }
         cp_async_commit();
@@ -327,6 +437,25 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         }
         cp_async_commit();
     }
+    // P = 128: TMEM for the tcgen05 step 1 (all 512 columns: one CTA per SM) and its mbarrier
+    __shared__ uint32_t s_tmem;
+    __shared__ __align__(8) uint64_t s_mbar[2];
+    uint32_t tmem = 0, mphase = 0;
+    const uint32_t mbar = smem_u32(&s_mbar[0]);
+    if constexpr (SM::kUM1) {
+        if (warp == 0) {
+            um::tmem_alloc(smem_u32(&s_tmem), 512);
+            um::tmem_relinquish();
+        }
+        if (tid == 0) {
+            um::mbar_init(mbar, 1);
+            um::mbar_init(mbar + 8u, 1);
+        }
+        um::fence_before();
+        __syncthreads();
+        um::fence_after();
+        tmem = s_tmem;
+    }
     if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3, 0);
 
     int k = 0;  // items done by this CTA
@@ -347,7 +476,38 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         const uint32_t xre = xre0 + buf * SM::kX, xim = xre + SM::kX / 2;
 
         // ---- step 1: outer DFT over p for 16 q at a time; times W_M^{q k_p}
-        outer_step1<P, NW, GATED, PRE1, IP, SM::kRS>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb, rsm);
+        if constexpr (SM::kUM1) {
+            if constexpr (GATED) {
+                // x = u w in place in the staging planes (w sits in S rows P/2 .. P-1)
+                for (int i = tid; i < 2 * (P / 2) * 32; i += NT) {
+                    // consecutive threads on consecutive 16-byte chunks of the canonical planes
+                    const int plane = i / ((P / 2) * 32), rem = i % ((P / 2) * 32), c = rem / (P / 2), p = rem % (P / 2);
+                    const uint32_t ua = (plane ? xim : xre) + xcan_off(p, c);
+                    const uint32_t wa = plane_addr(plane ? wim : wre, p, c);
+                    uint4 a, g;
+                    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w)
+                                 : "r"(ua));
+                    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                                 : "=r"(g.x), "=r"(g.y), "=r"(g.z), "=r"(g.w)
+                                 : "r"(wa));
+                    a.x = as_u(__hmul2(as_b2(a.x), as_b2(g.x)));
+                    a.y = as_u(__hmul2(as_b2(a.y), as_b2(g.y)));
+                    a.z = as_u(__hmul2(as_b2(a.z), as_b2(g.z)));
+                    a.w = as_u(__hmul2(as_b2(a.w), as_b2(g.w)));
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(ua), "r"(a.x), "r"(a.y), "r"(a.z),
+                                 "r"(a.w)
+                                 : "memory");
+                }
+            }
+            um::fence_proxy_async();  // the staged (and gated) x is read by the tensor core
+            __syncthreads();
+            if (!outer_step1_umma<NW, IP>(xre, xim, rsm, sre, sim, tmem, mbar, mphase, tid, lane, warp, tb))
+                atomicExch(err, 1);
+            mphase ^= 1u;
+        } else {
+            outer_step1<P, NW, GATED, PRE1, IP, SM::kRS>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb, rsm);
+        }
         __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
         if (SM::kNBuf == 1 && item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3, 0);
@@ -505,6 +665,14 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         // the next iteration's wait + barrier orders these reads before S is rewritten
     }
     cp_async_wait_all();
+    if constexpr (SM::kUM1) {
+        um::fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            um::fence_after();
+            um::tmem_dealloc(tmem, 512);
+        }
+    }
 }
 
 // Spectrum on the tensor cores, for transforms too long for one CTA's SIMT
@@ -792,7 +960,7 @@ static cudaError_t tc_fwd_go(const fftconv_plan_s& p, const void* u, const void*
     const int items = ((p.B + 1) / 2) * p.H;
     dim3 grid(items < resident ? items : resident);
     kern<<<grid, NW * 32, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
-                                     (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.B, p.H);
+                                     (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.d_err, p.B, p.H);
     return cudaGetLastError();
 }
 

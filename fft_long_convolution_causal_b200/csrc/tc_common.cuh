@@ -212,15 +212,26 @@ struct TcSmem {
     static constexpr int kR = kRS ? 2 * P * P : 0;  // two planes of P rows x P bytes
     static constexpr int kROff = kS + kNBuf * kX * ((GATED && !kWInS) ? 2 : 1);
     static constexpr int kBytes = kROff + kR;
+    // P = 128 (one CTA per SM): step 1 runs on tcgen05 from the staging planes
+    // (canonical MN-major layout) and the outer DFT matrix, into 512 TMEM columns
+    static constexpr bool kUM1 = P == 128;
 };
 
-// Byte offset of the 16-byte chunk c of row r of one plane of the outer DFT
-// matrix (rows of P/2 bf16 = P/16 chunks), XOR-swizzled so that the 8 rows
-// of an 8 x 8 ldmatrix block fall in 8 distinct 16-byte bank groups.
+// Byte offset of the 16-byte chunk c (8 values p) of row r (k_p) of one plane
+// of the outer DFT matrix, in the canonical no-swizzle K-major core-matrix
+// layout: core matrix (r / 8, c) of 8 rows x 16 bytes at (r / 8) (P / 16) 128
+// + 128 c.  The 8 rows of an 8 x 8 ldmatrix block are one 128-byte core
+// matrix (conflict-free), and the same bytes are the tcgen05 B operand
+// (LBO 128 along p, SBO (P / 16) 128 along k_p).
 template <int P>
 __device__ __forceinline__ uint32_t wr_off(int r, int c) {
-    constexpr int CPR = P / 16;
-    return (uint32_t)(r * P + ((c ^ ((r * CPR / 8) & (CPR - 1))) * 16));
+    return (uint32_t)((r >> 3) * (P / 16) * 128 + c * 128 + (r & 7) * 16);
+}
+// Byte offset of chunk c (8 values q) of row p of one staging plane of the
+// P = 128 kernel, canonical MN-major for tcgen05 (A operand, M = q, K = p):
+// core matrix (p / 8, c) at 1024 c + 128 (p / 8); LBO 128 along p, SBO 1024 along q.
+__device__ __forceinline__ uint32_t xcan_off(int p, int c) {
+    return (uint32_t)(c * 1024 + (p >> 3) * 128 + (p & 7) * 16);
 }
 
 // fp32 accumulators of two 16x8 tiles (n-tiles 0, 1) -> the four bf16x2
