@@ -437,7 +437,10 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         }
         cp_async_commit();
     }
-    // P = 128: TMEM for the tcgen05 step 1 (all 512 columns: one CTA per SM) and its mbarrier
+    // P = 128: TMEM for the tcgen05 step 1 and its mbarriers.  The CTA takes all 512
+    // columns; the allocation cannot wait on another CTA, because this kernel's
+    // 224 KiB of shared memory leaves no room on the SM for a second CTA of it or
+    // of the other TMEM user (the tcgen05 kernel of 2N <= 8192, 40-80 KiB each)
     __shared__ uint32_t s_tmem;
     __shared__ __align__(8) uint64_t s_mbar[2];
     uint32_t tmem = 0, mphase = 0;
