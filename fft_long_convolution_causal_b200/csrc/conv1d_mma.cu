@@ -347,7 +347,9 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     using SM = TcSmem<P, GATED>;
     static_assert(P >= 16 && P <= 128, "outer factor");
     static_assert((P / NW) % 2 == 0, "step 3 takes rows in pairs");
-    constexpr bool IP = P >= 128;  // integer packing measured faster only for the largest transform
+    // bf16 packing by the conversion instruction at every size (the integer form measured
+    // 3.7% slower at 2N = 32768 once step 1 ran on tcgen05, and slower at 2N = 8192)
+    constexpr bool IP = false;
     constexpr int NT = NW * 32;
     constexpr int CH = S::N / 8;                          // 16-byte chunks per row of u
     constexpr bool PRE1 = S::NT1 * S::KS1 <= 4;           // keep step-1 B fragments in registers
