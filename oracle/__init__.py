@@ -9,6 +9,8 @@ Definitions (see fftconv_oracle.c for the page citations):
 * ``causal_conv1d``: y[b,h,t] = sum_{s<=t, s<L} k[h,s] x[b,h,t-s] (+ D[h] x[b,h,t]),
   x = u (ungated) or u*w (gated, then y *= v).  This is
   irfft(rfft(x,2N) * rfft(k,2N))[:N] (+ D x) evaluated as the direct sum.
+* ``causal_conv1d_bwd``: the gradients du (dv, dw), dk, dD of that y for an
+  upstream gradient dy, by the chain rule written as direct sums.
 * ``causal_conv2d``: y[b,c,i,j] = sum_{p<=i,q<=j} k[c,p,q] u[b,c,i-p,j-q].
 * ``dft_causal_conv1d`` / ``dft_causal_conv2d``: the same results through an
   explicit O(M^2) DFT product (tiny sizes only), the independent second route.
@@ -31,6 +33,7 @@ def bind(path):
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_causal_conv1d.argtypes = [_i64] * 4 + [_f64p] * 6
     lib.oracle_causal_conv1d_points.argtypes = [_i64] * 4 + [_f64p] * 5 + [_i64] + [_i64p] * 3 + [_f64p]
+    lib.oracle_causal_conv1d_bwd.argtypes = [_i64] * 4 + [_f64p] * 11
     lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
     lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
     lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
@@ -110,6 +113,27 @@ def causal_conv1d_points(u, k, b_idx, h_idx, t_idx, D=None, w=None, v=None) -> n
     return out
 
 
+def causal_conv1d_bwd(u, k, dy, D=None, w=None, v=None) -> dict:
+    """fp64 gradients of y = causal_conv1d(u, k, D, w, v) for the upstream
+    gradient dy [B,H,N]: du (and dv, dw when gated) [B,H,N], dk [H,L],
+    dD [H] (when D is given).  The chain rule of the forward definition,
+    evaluated as direct sums (see fftconv_oracle.c)."""
+    u, k, D, w, v = _check_1d(u, k, D, w, v)
+    dy = _f64(dy)
+    if dy.shape != u.shape:
+        raise ValueError("dy must have u's shape")
+    B, H, N = u.shape
+    L = k.shape[1]
+    du = np.empty_like(u)
+    dv = np.empty_like(u) if w is not None else None
+    dw = np.empty_like(u) if w is not None else None
+    dk = np.empty((H, L))
+    dD = np.empty(H) if D is not None else None
+    _load().oracle_causal_conv1d_bwd(B, H, N, L, _p(u), _p(w), _p(v), _p(k), _p(D), _p(dy), _p(du), _p(dv),
+                                     _p(dw), _p(dk), _p(dD))
+    return {"du": du, "dv": dv, "dw": dw, "dk": dk, "dD": dD}
+
+
 def _check_2d(u, k):
     u = _f64(u)
     k = _f64(k)
@@ -170,5 +194,5 @@ def dft_causal_conv2d(x, k) -> np.ndarray:
     return y
 
 
-__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv2d", "causal_conv2d_points",
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv2d", "causal_conv2d_points",
            "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

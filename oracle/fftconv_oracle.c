@@ -117,6 +117,87 @@ void oracle_causal_conv1d_points(int64_t B, int64_t H, int64_t N, int64_t L,
     }
 }
 
+/*
+ * Gradients of the 1-D causal convolution (the backward pass that training
+ * the learned long filters of "Simple Hardware-Efficient Long Convolutions
+ * for Sequence Modeling" (abstract) and "FlashFFTConv" (abstract) needs),
+ * written as the chain rule applied to the forward definition above, term
+ * by term, for a loss whose gradient with respect to y is dy:
+ *   x = u (.) w (gated) or u;      g = dy (.) v (gated) or dy
+ *   s[t]  = sum_{j <= min(t, L-1)} k[j] x[t-j] + D x[t]        (pre-gate output)
+ *   dx[t] = sum_{j <= min(L-1, N-1-t)} k[j] g[t+j] + D g[t]     (y[t+j] depends on x[t] via k[j])
+ *   du = dx (.) w or dx;   dw = dx (.) u;   dv = dy (.) s
+ *   dk[h][j] = sum_b sum_{t >= j} g[b,h,t] x[b,h,t-j],  j < L
+ *   dD[h]    = sum_b sum_t g[b,h,t] x[b,h,t]
+ * Shapes as oracle_causal_conv1d; dv, dw are written only when gated (w, v
+ * non-NULL); dD only when D is non-NULL.  fp64, natural order.
+ */
+void oracle_causal_conv1d_bwd(int64_t B, int64_t H, int64_t N, int64_t L,
+                              const double* u, const double* w, const double* v,
+                              const double* k, const double* D, const double* dy,
+                              double* du, double* dv, double* dw, double* dk, double* dD)
+{
+    int64_t rows = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t h = r % H;
+        const double* kr = k + h * L;
+        const double* ur = u + r * N;
+        const double* dyr = dy + r * N;
+        for (int64_t t = 0; t < N; ++t) {
+            double acc = 0.0;
+            int64_t jmax = (L - 1 < N - 1 - t) ? L - 1 : N - 1 - t;
+            for (int64_t j = 0; j <= jmax; ++j) {
+                double g = v ? dyr[t + j] * v[r * N + t + j] : dyr[t + j];
+                acc += kr[j] * g;
+            }
+            if (D) {
+                double g = v ? dyr[t] * v[r * N + t] : dyr[t];
+                acc += D[h] * g;
+            }
+            if (w) {
+                du[r * N + t] = acc * w[r * N + t];
+                dw[r * N + t] = acc * ur[t];
+                /* dv = dy . s, s the pre-gate output at t */
+                double sacc = 0.0;
+                int64_t jtop = (t < L - 1) ? t : L - 1;
+                for (int64_t j = 0; j <= jtop; ++j) sacc += kr[j] * (ur[t - j] * w[r * N + t - j]);
+                if (D) sacc += D[h] * (ur[t] * w[r * N + t]);
+                dv[r * N + t] = dyr[t] * sacc;
+            } else {
+                du[r * N + t] = acc;
+            }
+        }
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t h = 0; h < H; ++h) {
+        for (int64_t j = 0; j < L; ++j) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < B; ++b) {
+                int64_t r = b * H + h;
+                for (int64_t t = j; t < N; ++t) {
+                    double g = v ? dy[r * N + t] * v[r * N + t] : dy[r * N + t];
+                    double x = w ? u[r * N + t - j] * w[r * N + t - j] : u[r * N + t - j];
+                    acc += g * x;
+                }
+            }
+            dk[h * L + j] = acc;
+        }
+        if (D) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < B; ++b) {
+                int64_t r = b * H + h;
+                for (int64_t t = 0; t < N; ++t) {
+                    double g = v ? dy[r * N + t] * v[r * N + t] : dy[r * N + t];
+                    double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];
+                    acc += g * x;
+                }
+            }
+            dD[h] = acc;
+        }
+    }
+}
+
 /* One output of the 2-D causal convolution of image (b,c) at (i,j). */
 static double conv2d_point(int64_t Ws, int64_t Kh, int64_t Kw, const double* ui,
                            const double* kc, int64_t i, int64_t j)

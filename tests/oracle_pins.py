@@ -244,9 +244,85 @@ def check_points_match_full_2d():
     assert np.array_equal(pts, full[tuple(idx)])
 
 
+def _loss(u, k, D, w, v, dy):
+    """The scalar <dy, y> of the forward oracle: its gradients are the backward."""
+    return float(np.sum(dy * oracle.causal_conv1d(u, k, D=D, w=w, v=v)))
+
+
+def check_bwd_central_differences():
+    """The backward oracle against central differences of the (pinned) forward
+    oracle.  The loss <dy, y> is linear in each of u, k, D, v and w separately,
+    so a central difference has no truncation error: the two agree to
+    rounding, for every gradient entry, gated and ungated, L < N."""
+    r = _rng(61)
+    for gated, L in ((False, 9), (True, 12), (True, 5)):
+        B, H, N = 2, 2, 12
+        u = r.standard_normal((B, H, N))
+        k = r.standard_normal((H, L))
+        D = r.standard_normal(H)
+        dy = r.standard_normal((B, H, N))
+        w = r.standard_normal((B, H, N)) if gated else None
+        v = r.standard_normal((B, H, N)) if gated else None
+        g = oracle.causal_conv1d_bwd(u, k, dy, D=D, w=w, v=v)
+        eps = 0.5
+        args = {"u": u, "k": k, "D": D, "w": w, "v": v}
+        for name in ("u", "k", "D") + (("w", "v") if gated else ()):
+            base = args[name]
+            num = np.empty_like(base)
+            for idx in np.ndindex(base.shape):
+                plus, minus = base.copy(), base.copy()
+                plus[idx] += eps
+                minus[idx] -= eps
+                lp = _loss(**{**args, name: plus}, dy=dy)
+                lm = _loss(**{**args, name: minus}, dy=dy)
+                num[idx] = (lp - lm) / (2 * eps)
+            got = g["d" + name]
+            assert np.allclose(got, num, rtol=1e-9, atol=1e-9), (name, gated, np.abs(got - num).max())
+
+
+def check_bwd_numpy_correlate():
+    """dx and dk against numpy.correlate (the library cross-correlation):
+    dx[t] = sum_j k[j] g[t+j] is correlate(g, k) at lags 0..N-1, and
+    dk[j] = sum_b sum_t g[t] x[t-j] is sum_b correlate(g_b, x_b) at lags 0..L-1."""
+    r = _rng(62)
+    B, H, N, L = 3, 2, 40, 17
+    u = r.standard_normal((B, H, N))
+    k = r.standard_normal((H, L))
+    dy = r.standard_normal((B, H, N))
+    g = oracle.causal_conv1d_bwd(u, k, dy)
+    for b in range(B):
+        for h in range(H):
+            full = np.correlate(dy[b, h], k[h], mode="full")  # index N-1+lag? see below
+            # numpy: c[n] = sum_m a[n+m-(len(v)-1)] v[m]; lag 0 of a against v is n = L-1
+            want = full[L - 1:L - 1 + N]
+            assert np.allclose(g["du"][b, h], want, rtol=1e-12, atol=1e-12)
+    for h in range(H):
+        acc = np.zeros(L)
+        for b in range(B):
+            c = np.correlate(dy[b, h], u[b, h], mode="full")  # lag j of dy against u at N-1+j
+            acc += c[N - 1:N - 1 + L]
+        assert np.allclose(g["dk"][h], acc, rtol=1e-12, atol=1e-11)
+
+
+def check_bwd_delta_kernel():
+    """k = delta, D = 0: y = u, so du = dy exactly and dk[j] = sum_b <dy, u shifted by j>."""
+    r = _rng(63)
+    B, H, N = 2, 1, 10
+    u = r.standard_normal((B, H, N))
+    dy = r.standard_normal((B, H, N))
+    k = np.zeros((H, 4))
+    k[:, 0] = 1.0
+    g = oracle.causal_conv1d_bwd(u, k, dy, D=np.zeros(H))
+    assert np.array_equal(g["du"], dy)
+    for j in range(4):
+        assert np.isclose(g["dk"][0, j], float(np.sum(dy[:, 0, j:] * u[:, 0, :N - j])), rtol=1e-13)
+    assert np.isclose(g["dD"][0], float(np.sum(dy * u)), rtol=1e-13)
+
+
 ALL_CHECKS = [
     check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
     check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
+    check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel,
 ]

@@ -34,6 +34,19 @@ MUTANTS = {
                          "double pr = Xr[f] * Kr[f] + Xi[f] * Ki[f];"),
     "dft2_inverse_sign": ("acc += Pr[fh * Mw + fw] * c - Pi[fh * Mw + fw] * s;",
                          "acc += Pr[fh * Mw + fw] * c + Pi[fh * Mw + fw] * s;"),
+    "bwd_correlation_as_convolution": ("double g = v ? dyr[t + j] * v[r * N + t + j] : dyr[t + j];",
+                                       "double g = v ? dyr[t - j < 0 ? 0 : t - j] * v[r * N + t + j] : "
+                                       "dyr[t - j < 0 ? 0 : t - j];"),
+    "bwd_drop_last_lag": ("int64_t jmax = (L - 1 < N - 1 - t) ? L - 1 : N - 1 - t;",
+                          "int64_t jmax = (L - 2 < N - 1 - t) ? L - 2 : N - 1 - t;"),
+    "bwd_du_not_gated": ("du[r * N + t] = acc * w[r * N + t];", "du[r * N + t] = acc;"),
+    "bwd_dw_times_w": ("dw[r * N + t] = acc * ur[t];", "dw[r * N + t] = acc * w[r * N + t];"),
+    "bwd_dk_lag_sign": ("double x = w ? u[r * N + t - j] * w[r * N + t - j] : u[r * N + t - j];",
+                        "double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];"),
+    "bwd_dD_ungated_g": ("                    double g = v ? dy[r * N + t] * v[r * N + t] : dy[r * N + t];\n"
+                         "                    double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];",
+                         "                    double g = dy[r * N + t];\n"
+                         "                    double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];"),
 }
 
 
