@@ -9,6 +9,7 @@ Definitions (see fftconv_oracle.c for the page citations):
 * ``causal_conv1d``: y[b,h,t] = sum_{s<=t, s<L} k[h,s] x[b,h,t-s] (+ D[h] x[b,h,t]),
   x = u (ungated) or u*w (gated, then y *= v).  This is
   irfft(rfft(x,2N) * rfft(k,2N))[:N] (+ D x) evaluated as the direct sum.
+* ``causal_conv1d_dynamic``: the same with one filter per batch row, k [B,H,L].
 * ``causal_conv1d_bwd``: the gradients du (dv, dw), dk, dD of that y for an
   upstream gradient dy, by the chain rule written as direct sums.
 * ``causal_conv2d``: y[b,c,i,j] = sum_{p<=i,q<=j} k[c,p,q] u[b,c,i-p,j-q].
@@ -34,6 +35,7 @@ def bind(path):
     lib.oracle_causal_conv1d.argtypes = [_i64] * 4 + [_f64p] * 6
     lib.oracle_causal_conv1d_points.argtypes = [_i64] * 4 + [_f64p] * 5 + [_i64] + [_i64p] * 3 + [_f64p]
     lib.oracle_causal_conv1d_bwd.argtypes = [_i64] * 4 + [_f64p] * 11
+    lib.oracle_causal_conv1d_dynamic.argtypes = [_i64] * 4 + [_f64p] * 6
     lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
     lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
     lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
@@ -111,6 +113,18 @@ def causal_conv1d_points(u, k, b_idx, h_idx, t_idx, D=None, w=None, v=None) -> n
     _load().oracle_causal_conv1d_points(B, H, N, k.shape[1], _p(u), _p(w), _p(v), _p(k), _p(D),
                                         bi.size, _ip(bi), _ip(hi), _ip(ti), _p(out))
     return out
+
+
+def causal_conv1d_dynamic(u, k, D=None, w=None, v=None) -> np.ndarray:
+    """fp64 oracle with one filter per batch row: k [B,H,L]; returns y [B,H,N]."""
+    k = _f64(k)
+    if k.ndim != 3 or k.shape[:2] != np.shape(u)[:2]:
+        raise ValueError("k must be [B,H,L]")
+    u, _, D, w, v = _check_1d(u, k[0], D, w, v)
+    B, H, N = u.shape
+    y = np.empty_like(u)
+    _load().oracle_causal_conv1d_dynamic(B, H, N, k.shape[2], _p(u), _p(w), _p(v), _p(k), _p(D), _p(y))
+    return y
 
 
 def causal_conv1d_bwd(u, k, dy, D=None, w=None, v=None) -> dict:
@@ -194,5 +208,5 @@ def dft_causal_conv2d(x, k) -> np.ndarray:
     return y
 
 
-__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv2d", "causal_conv2d_points",
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "causal_conv2d", "causal_conv2d_points",
            "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

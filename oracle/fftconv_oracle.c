@@ -198,6 +198,31 @@ void oracle_causal_conv1d_bwd(int64_t B, int64_t H, int64_t N, int64_t L,
     }
 }
 
+/*
+ * Input-dependent kernels ("Native Multi-Dimensional Subquadratic Operators
+ * via Input Dependent Long Convolutions", abstract: HyenaND convolves with
+ * input-dependent kernels): every batch row has its own filter,
+ *   y[b,h,t] = sum_{s <= min(t, L-1)} k[b,h,s] x[b,h,t-s] + D[h] x[b,h,t],
+ * x and the gate as in oracle_causal_conv1d.  k: [B][H][L].
+ */
+void oracle_causal_conv1d_dynamic(int64_t B, int64_t H, int64_t N, int64_t L,
+                                  const double* u, const double* w, const double* v,
+                                  const double* k, const double* D, double* y)
+{
+    int64_t rows = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t h = r % H;
+        const double* ur = u + r * N;
+        const double* wr = w ? w + r * N : NULL;
+        const double* vr = v ? v + r * N : NULL;
+        const double* kr = k + r * L;
+        const double* Dh = D ? D + h : NULL;
+        for (int64_t t = 0; t < N; ++t)
+            y[r * N + t] = conv1d_point(N, L, ur, wr, vr, kr, Dh, t);
+    }
+}
+
 /* One output of the 2-D causal convolution of image (b,c) at (i,j). */
 static double conv2d_point(int64_t Ws, int64_t Kh, int64_t Kw, const double* ui,
                            const double* kc, int64_t i, int64_t j)

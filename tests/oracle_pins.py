@@ -319,10 +319,36 @@ def check_bwd_delta_kernel():
     assert np.isclose(g["dD"][0], float(np.sum(dy * u)), rtol=1e-13)
 
 
+def check_dynamic_kernels():
+    """Per-row filters: numpy.convolve row by row (the library routine), the
+    shared-filter oracle when every row carries its channel's filter, and row
+    independence (changing one row's filter changes only that row)."""
+    r = _rng(64)
+    B, H, N, L = 3, 2, 33, 20
+    u = r.standard_normal((B, H, N))
+    k = r.standard_normal((B, H, L))
+    D = r.standard_normal(H)
+    y = oracle.causal_conv1d_dynamic(u, k, D=D)
+    for b in range(B):
+        for h in range(H):
+            want = np.convolve(u[b, h], k[b, h])[:N] + D[h] * u[b, h]
+            assert np.allclose(y[b, h], want, rtol=1e-12, atol=1e-12)
+    shared = np.broadcast_to(k[0][None], k.shape).copy()
+    w = r.standard_normal((B, H, N))
+    v = r.standard_normal((B, H, N))
+    assert np.array_equal(oracle.causal_conv1d_dynamic(u, shared, D=D, w=w, v=v),
+                          oracle.causal_conv1d(u, k[0], D=D, w=w, v=v))
+    k2 = k.copy()
+    k2[1, 0] += 1.0
+    y2 = oracle.causal_conv1d_dynamic(u, k2, D=D)
+    changed = np.any(y2 != y, axis=2)
+    assert changed[1, 0] and changed.sum() == 1
+
+
 ALL_CHECKS = [
     check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
     check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
-    check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel,
+    check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
 ]

@@ -47,6 +47,10 @@ MUTANTS = {
                          "                    double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];",
                          "                    double g = dy[r * N + t];\n"
                          "                    double x = w ? u[r * N + t] * w[r * N + t] : u[r * N + t];"),
+    "dynamic_channel_filter": ("        const double* kr = k + r * L;\n        const double* Dh = D ? D + h : NULL;\n"
+                               "        for (int64_t t = 0; t < N; ++t)\n            y[r * N + t] = conv1d_point",
+                               "        const double* kr = k + h * L;\n        const double* Dh = D ? D + h : NULL;\n"
+                               "        for (int64_t t = 0; t < N; ++t)\n            y[r * N + t] = conv1d_point"),
 }
 
 
