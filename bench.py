@@ -7,14 +7,23 @@ A step is one forward pass of the whole hot path (load, FFT, product with the
 cached kernel spectrum, inverse FFT, truncation, skip term / gate, store) over
 one batch of the named synthetic workload.  The kernel spectrum is computed
 once per plan, before timing.  Default workload: B=8, H=768, N=4096, bf16
-(the Hyena-style layer convolution).
+(the Hyena-style layer convolution); at one GPU the line also carries
+`per_config`, the same measurement for each of the other named workloads
+(N = 1K, 16K gated, 1M, and 2-D 256 x 256), fewer steps each.
 
 Timing: W untimed warm-up steps; then a barrier and a device synchronise; then
 exactly K steps, each bracketed by CUDA events on the launching stream with an
 L2 flush (a 256 MiB write, more than the 126 MB L2) between steps outside the
 events; a synchronise and a barrier; the max over ranks.  value = outputs of
-all ranks / that time (weak scaling: every rank runs the full workload; the
-rows are independent so no collective is on the data path).
+all ranks / that time.
+
+Several GPUs (torchrun, one rank per GPU): the channels are sharded, one
+contiguous block per rank, with no collective on the data path (rows are
+independent and every channel's spectrum is read-only).  --shard weak
+(default): the job at N ranks is the named workload with N times its channels,
+rank r holding block r (the named shape per GPU; each rank draws its block
+with its own seed).  --shard strong: the named workload's channels are split
+over the ranks (total work fixed).
 
 e2e: the same step through the public API from pinned host buffers, with the
 host->device copy of the inputs and the device->host copy of y inside the
@@ -42,8 +51,17 @@ METRIC = "FFT-conv output elems/s and % of HBM roofline (1 B200), N=1K–1M and 
 DEFAULT_CONFIG = "hyena_b8_h768_n4096_bf16"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ["fft_simt.cuh", "conv1d_simt.cu", "conv2d_simt.cu", "tc_common.cuh", "conv1d_mma.cu", "umma.cuh",
-                  "conv1d_umma.cu", "conv2d_tc.cu"]
+# Source files each dominant kernel is built from: a recorded DRAM-traffic
+# figure is valid only while the hash of these files matches.
+KERNEL_SOURCES = {
+    "fused_fwd_simt": ["fft_simt.cuh", "conv1d_simt.cu"],
+    "mp_pass2": ["fft_simt.cuh", "conv1d_simt.cu"],
+    "c2_pass2": ["fft_simt.cuh", "conv2d_simt.cu"],
+    "fused_fwd_tc": ["tc_common.cuh", "umma.cuh", "conv1d_mma.cu"],
+    "fused_fwd_umma": ["tc_common.cuh", "umma.cuh", "conv1d_umma.cu"],
+    "fused_fwd_t2": ["umma.cuh", "conv1d_t2.cu"],
+    "c2tc_cols": ["tc_common.cuh", "tables.h", "conv2d_tc.cu"],
+}
 
 
 def parse():
@@ -60,6 +78,15 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--channels", type=int, default=0,
                     help="override H (1-D) or C (2-D) for a smaller case, e.g. an ncu capture; 0 = as named")
+    ap.add_argument("--shard", default="weak", choices=["weak", "strong"],
+                    help="several GPUs: N x the channels (weak) or the named channels split (strong)")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "mma_sync", "tcgen05"],
+                    help="kernel family the plans may use (the library's choice by default)")
+    ap.add_argument("--no-per-config", action="store_true", help="headline workload only")
+    ap.add_argument("--per-config-steps", type=int, default=10)
+    ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
+                    help="write profiles/traffic.json's entry for --config from an ncu raw CSV and exit")
+    ap.add_argument("--traffic-command", default="", help="the capture command, stored with the record")
     return ap.parse_args()
 
 
@@ -68,37 +95,76 @@ def dist_env():
     return rank_env()
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def measured_peaks():
+    """(HBM GB/s, bf16 dense TFLOP/s burst, source) from MEASURED_PEAKS.json, else the fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         try:
             d = json.load(open(path))
-            return float(d["hbm_gbs"]), "measured"
+            return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
         except Exception:
             pass
-    return FALLBACK_HBM_GBS, "fallback"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "fft_long_convolution_causal_b200", "csrc", f), "rb").read())
+    for f in KERNEL_SOURCES.get(kernel, []):
+        path = os.path.join(ROOT, "fft_long_convolution_causal_b200", "csrc", f)
+        h.update(open(path, "rb").read() if os.path.exists(path) else b"")
     return h.hexdigest()[:16]
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+
+
 def recorded_traffic(config, kernel):
-    """DRAM bytes per launch from a committed ncu summary, if it still matches the sources."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    """DRAM bytes per launch of `kernel` on `config` from the committed record,
+    if the kernel's sources still hash to what they were when it was taken."""
+    if not os.path.exists(TRAFFIC_JSON):
         return None
     try:
-        d = json.load(open(path))
-        e = d.get(config, {})
-        if e.get("kernel") == kernel and e.get("source_hash") == kernel_source_hash():
+        e = json.load(open(TRAFFIC_JSON)).get(config, {})
+        if e.get("kernel") == kernel and e.get("source_hash") == kernel_source_hash(kernel):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         return None
     return None
+
+
+def record_traffic(csv_path, config, channels, command):
+    """Write profiles/traffic.json's entry for `config` from an ncu raw CSV
+    (`ncu -i X.ncu-rep --page raw --csv`) of the config's dominant kernel.
+    A capture on fewer channels (--channels) is scaled to the full workload by
+    the channel ratio (each launch processes every channel once)."""
+    import csv
+    from fft_long_convolution_causal_b200 import workloads
+    rows = list(csv.reader(open(csv_path)))
+    head = rows[0]
+    data = [r for r in rows[1:] if len(r) == len(head) and r[head.index("ID")].strip().isdigit()]
+    kcol, rcol, wcol = head.index("Kernel Name"), head.index("dram__bytes_read.sum"), head.index("dram__bytes_write.sum")
+    units = {rows[1][i] for i in (rcol, wcol)}
+
+    def to_bytes(v, unit):
+        f = float(v.replace(",", ""))
+        return f * {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}.get(unit, 1)
+
+    kname = data[0][kcol]
+    short = next((k for k in KERNEL_SOURCES if k in kname), None)
+    per = [to_bytes(r[rcol], rows[1][rcol]) + to_bytes(r[wcol], rows[1][wcol]) for r in data]
+    c = workloads.CONFIGS[config]
+    full = c["H"] if c["kind"] == "1d" else c["C"]
+    scale = full / channels if channels else 1.0
+    d = json.load(open(TRAFFIC_JSON)) if os.path.exists(TRAFFIC_JSON) else {}
+    d[config] = {"kernel": short, "dram_bytes_per_launch": float(np.mean(per)) * scale,
+                 "source_hash": kernel_source_hash(short), "launches_captured": len(per),
+                 "captured_channels": channels or full, "scaled_by": scale, "units_seen": sorted(units),
+                 "command": command}
+    json.dump(d, open(TRAFFIC_JSON, "w"), indent=1, sort_keys=True)
+    print(json.dumps(d[config]))
 
 
 # ----------------------------------------------------------------- clocks
@@ -156,23 +222,34 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- workload
-def build_workload(name, channels=0):
+def build_workload(name, channels=0, rank=0, world=1, shard="weak"):
+    """The named workload (or a smaller one with `channels`), as this rank's shard.
+
+    weak: the rank's block of a job with world x the channels, drawn with the
+    named seed + 1000 * rank (rank 0 draws exactly the named workload).
+    strong: the named workload's channel block shard_channels(H, world, rank)."""
+    from fft_long_convolution_causal_b200 import dist as fdist
     from fft_long_convolution_causal_b200 import workloads
-    if not channels:
-        return workloads.make_config(name)
     c = dict(workloads.CONFIGS[name])
     kind = c.pop("kind")
-    if kind == "1d":
-        c["H"] = channels
-        return workloads.make_1d(name=f"{name}_h{channels}", **c)
-    c["C"] = channels
-    return workloads.make_2d(name=f"{name}_c{channels}", **c)
+    label = name
+    if channels:
+        c["H" if kind == "1d" else "C"] = channels
+        label = f"{name}_{'h' if kind == '1d' else 'c'}{channels}"
+    if world > 1 and shard == "weak":
+        c["seed"] = c["seed"] + 1000 * rank
+    wl = workloads.make_1d(name=label, **c) if kind == "1d" else workloads.make_2d(name=label, **c)
+    if world > 1 and shard == "strong":
+        nch = wl.H if kind == "1d" else wl.C
+        a, b = fdist.shard_channels(nch, world, rank)
+        wl = fdist.slice_channels_1d(wl, a, b) if kind == "1d" else fdist.slice_channels_2d(wl, a, b)
+    return wl
 
 
 class Runner:
     """Device-resident workload + plan; step() enqueues one forward."""
 
-    def __init__(self, wl, torch):
+    def __init__(self, wl, torch, kernel="auto"):
         from fft_long_convolution_causal_b200 import binding
         self.torch = torch
         self.wl = wl
@@ -185,14 +262,14 @@ class Runner:
 
         self.is2d = hasattr(wl, "C")
         if self.is2d:
-            self.plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, wl.dtype)
+            self.plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, wl.dtype, kernel=kernel)
             self.khat = self.plan.kernel_spectrum(torch.from_numpy(wl.k).to(dev))
             self.u = up(wl.u)
             self.v = self.w = self.D = None
             self.y = torch.empty_like(self.u)
             self.outputs = wl.B * wl.C * wl.Hs * wl.Ws
         else:
-            self.plan = binding.Plan(wl.B, wl.H, wl.N, wl.dtype, gated=wl.gated)
+            self.plan = binding.Plan(wl.B, wl.H, wl.N, wl.dtype, gated=wl.gated, kernel=kernel)
             self.khat = self.plan.kernel_spectrum(torch.from_numpy(wl.k).to(dev))
             self.u, self.v, self.w = up(wl.u), up(wl.v), up(wl.w)
             self.D = None if wl.D is None else torch.from_numpy(wl.D).to(dev)
@@ -212,7 +289,7 @@ class Runner:
                           y=y, workspace=ws)
 
     def launches_per_step(self):
-        if self.plan.path in ("fused", "fused_tc", "fused_umma"):
+        if self.plan.path in ("fused", "fused_tc", "fused_umma", "fused_t2"):
             return 1
         pairs = ((self.wl.B + 1) // 2) * (self.wl.C if self.is2d else self.wl.H)
         group = max(1, self.plan.workspace_bytes // self._pair_bytes())
@@ -224,11 +301,11 @@ class Runner:
         return 2 * self.wl.N * 8
 
     def compute_dtype(self):
-        return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16",
+        return {"fused": "f32", "multipass": "f32", "2d": "f32", "fused_tc": "bf16", "fused_t2": "bf16",
                 "fused_umma": "bf16", "2d_tc": "f32+bf16"}.get(self.plan.path, "f32")
 
     def dominant_kernel(self):
-        return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2",
+        return {"fused": "fused_fwd_simt", "multipass": "mp_pass2", "2d": "c2_pass2", "fused_t2": "fused_fwd_t2",
                 "fused_tc": "fused_fwd_tc", "fused_umma": "fused_fwd_umma", "2d_tc": "c2tc_cols"}.get(self.plan.path)
 
 
@@ -348,26 +425,35 @@ def cpu_oracle_rate(wl, target_s, seed=0):
 
 
 # ------------------------------------------------------------------ main
-def main():
-    args = parse()
-    rank, world, local = dist_env()
-    import torch
-    if args.impl == "reference":
-        return main_reference(args, rank, world)
-    torch.cuda.set_device(local)
-    pg = None
+def workload_config(wl, path=None, world=1, shard="weak"):
+    """The `config` object of a line: the workload by name and shape."""
+    cfg = {"workload": wl.name, "dtype_io": wl.dtype,
+           "l2": "flushed between timed steps (256 MiB write outside the events)"}
+    if path:
+        cfg["path"] = path
     if world > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-        pg = dist
-    wl = build_workload(args.config, args.channels)
-    r = Runner(wl, torch)
+        cfg["parallelism"] = (f"channels sharded over {world} ranks, {shard} scaling, no collective on the data path")
+    else:
+        cfg["parallelism"] = "1 GPU"
+    if hasattr(wl, "C"):
+        cfg.update(B=wl.B, C=wl.C, Hs=wl.Hs, Ws=wl.Ws)
+    else:
+        cfg.update(B=wl.B, H=wl.H, N=wl.N, gated=wl.gated, skip_term=wl.D is not None)
+    return cfg
+
+
+def measure(wl, args, torch, steps, warmup, pg=None, world=1, clocks=False, e2e=True, cpu_seconds=0.0,
+            config_name=None):
+    """Time one workload: K device-timed steps (max over ranks), optional
+    e2e, the roofline of the dominant kernel, the tensor-pipe fraction and the
+    CPU oracle baseline.  Returns the result dict (the line's fields)."""
+    rank = pg.get_rank() if pg else 0
+    r = Runner(wl, torch, kernel=args.kernel)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         r.step()
     torch.cuda.synchronize()
-    sampler = None if (args.no_clocks or rank != 0) else ClockSampler(local)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if (clocks and rank == 0) else None
     if sampler:
         sampler.start()
         # keep the GPU busy for a moment so the clock samples see it under load
@@ -380,64 +466,106 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    per_step = time_steps(r, args.steps, torch, flush)
+    per_step = time_steps(r, steps, torch, flush)
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    clocks = sampler.stop() if sampler else None
+    clk = sampler.stop() if sampler else None
     from fft_long_convolution_causal_b200.dist import job_throughput, max_over_ranks
     total_ms = max_over_ranks(float(np.sum(per_step)), pg, device="cuda")
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / steps
     value = job_throughput(r.outputs, world, ms_per_step * 1e-3)
 
-    e2e = None
-    if not args.no_e2e:
-        e2e_ms, h2d, d2h = time_e2e(r, max(3, min(args.steps, 20)), torch)
+    e2e_d = None
+    if e2e:
+        e2e_ms, h2d, d2h = time_e2e(r, max(3, min(steps, 20)), torch)
         e2e_ms = max_over_ranks(e2e_ms, pg, device="cuda")
-        e2e = {"value": job_throughput(r.outputs, world, e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        e2e_d = {"value": job_throughput(r.outputs, world, e2e_ms * 1e-3), "unit": "elems/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    peak, peak_kind = measured_peaks()
+    hbm, bf16, peak_kind = measured_peaks()
     alg_bytes = wl.io_bytes()
-    launches = r.launches_per_step()
-    # The fused path is one launch per step, so the step's event time is that
+    # The fused paths are one launch per step, so the step's event time is that
     # kernel's time; for multi-launch paths the whole step is charged to the
     # dominant kernel (a lower bound on its achieved rate).
     achieved = alg_bytes / (ms_per_step * 1e-3) / 1e9
     kname = r.dominant_kernel()
-    traffic = recorded_traffic(args.config, kname)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kname,
-                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": alg_bytes}
-
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": recorded_traffic(config_name or wl.name, kname),
+                "kernel": kname, "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": alg_bytes}
+    mma = r.plan.mma_flops
+    tensor = {"mma_flops_per_step": mma, "achieved_tflops": round(mma / (ms_per_step * 1e-3) / 1e12, 2),
+              "peak_tflops": bf16, "peak_source": f"{peak_kind} bf16_tflops (burst)",
+              "frac": round(mma / (ms_per_step * 1e-3) / 1e12 / bf16, 4)}
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_rate(wl, args.cpu_seconds)
+    if cpu_seconds > 0 and rank == 0 and world == 1:
+        cpu = cpu_oracle_rate(wl, cpu_seconds)
+    res = {"value": value, "unit": "elems/s", "ms_per_step": ms_per_step, "steps": steps, "warmup": warmup,
+           "ms_per_step_min": float(np.min(per_step)), "ms_per_step_median": float(np.median(per_step)),
+           "dtype": r.compute_dtype(), "config": workload_config(wl, r.plan.path, world, args.shard),
+           "roofline": roofline, "tensor_pipe": tensor, "cpu_baseline": cpu, "e2e": e2e_d,
+           "gpu_launches": r.launches_per_step() * steps, "clocks": clk}
+    del r
+    torch.cuda.empty_cache()
+    return res
 
+
+def main():
+    args = parse()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.config, args.channels, args.traffic_command)
+        return 0
+    rank, world, local = dist_env()
+    import torch
+    if args.impl == "reference":
+        return main_reference(args, rank, world)
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        pg = dist
+    wl = build_workload(args.config, args.channels, rank, world, args.shard)
+    head = measure(wl, args, torch, args.steps, args.warmup, pg=pg, world=world, clocks=not args.no_clocks,
+                   e2e=not args.no_e2e, cpu_seconds=0.0 if args.no_cpu_baseline else args.cpu_seconds,
+                   config_name=args.config)
+    del wl
+    per_config = None
+    if world == 1 and not args.no_per_config and not args.channels:
+        from fft_long_convolution_causal_b200 import workloads
+        per_config = {}
+        for name in workloads.CONFIG_ORDER:
+            if name == args.config:
+                continue
+            w2 = build_workload(name)
+            res = measure(w2, args, torch, args.per_config_steps, 3, clocks=False, e2e=not args.no_e2e,
+                          cpu_seconds=0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 5.0),
+                          config_name=name)
+            del w2
+            per_config[name] = res
     if pg:
         pg.barrier()
         pg.destroy_process_group()
     if rank != 0:
         return 0
-    cfg = {"workload": wl.name, "dtype_io": wl.dtype, "path": r.plan.path,
-           "l2": "flushed between timed steps (256 MiB write outside the events)",
-           "parallelism": f"replicas x{world} (independent rows, no collective)"}
-    if r.is2d:
-        cfg.update(B=wl.B, C=wl.C, Hs=wl.Hs, Ws=wl.Ws)
-    else:
-        cfg.update(B=wl.B, H=wl.H, N=wl.N, gated=wl.gated, skip_term=wl.D is not None)
-    line = {"metric": METRIC, "value": value, "unit": "elems/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": r.compute_dtype(), "data": "synthetic", "config": cfg,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches * args.steps, "clocks": clocks,
-            "ms_per_step_min": float(np.min(per_step)), "ms_per_step_median": float(np.median(per_step))}
+    line = {"metric": METRIC, "value": head["value"], "unit": "elems/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak" if (world == 1 or args.shard == "weak") else "strong", "vs_baseline": None,
+            "dtype": head["dtype"], "data": "synthetic", "config": head["config"],
+            "roofline": head["roofline"], "tensor_pipe": head["tensor_pipe"], "cpu_baseline": head["cpu_baseline"],
+            "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+            "ms_per_step_min": head["ms_per_step_min"], "ms_per_step_median": head["ms_per_step_median"]}
+    if per_config is not None:
+        line["per_config"] = per_config
     print(json.dumps(line))
     return 0
 
 
 def main_reference(args, rank, world):
-    """The oracle as the reference arm: rank 0 times it on the host cores."""
+    """The oracle as the reference arm: rank 0 times it on the host cores, each
+    step a bounded uniform sample of the workload's outputs."""
     if rank != 0:
         return 0
     wl = build_workload(args.config, args.channels)
@@ -448,10 +576,11 @@ def main_reference(args, rank, world):
         s.run(max(n // 8, 64))
     times = [s.run(n) for _ in range(args.steps)]
     value = n * len(times) / float(np.sum(times))
+    cfg = workload_config(wl, "oracle (CPU fp64 direct sum)", 1, args.shard)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "elems/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s.total / value * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.config, "dtype_io": wl.dtype},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean(times)) * 1e3,
+            "outputs_per_step": n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg,
             "cpu_baseline": {"value": value, "unit": "elems/s", "cores": s.oracle.num_threads(), "kind": "oracle",
                              "sample": "each step: " + s.describe(n, float(np.mean(times)))},
             "e2e": {"value": value, "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -22,10 +22,31 @@ STATUS = {
 }
 DTYPES = {"f32": 0, "bf16": 1}
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+KERNELS = {"auto": 0, "simt": 1, "mma_sync": 2, "tcgen05": 3}  # fftconv_kernel
+DEFAULT_WAIT_PROBES = 65536
+
+
+class PlanOptions(ctypes.Structure):
+    """fftconv_plan_options."""
+    _fields_ = [("kernel", ctypes.c_int), ("group_bytes", ctypes.c_size_t)]
+
 
 # name -> (restype, argtypes); mirrors include/fftconv.h
 _vp = ctypes.c_void_p
+_optp = ctypes.POINTER(PlanOptions)
 _SIGS = {
+    "fftconv_plan_options_init": (None, [_optp]),
+    "fftconv_plan_create_ex": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                              ctypes.c_int, ctypes.c_int, _optp]),
+    "fftconv2d_plan_create_ex": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, _optp]),
+    "fftconv_plan_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint32]),
+    "fftconv_spectrum_conjugate": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
+    "fftconv_fwd_dynamic": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp]),
+    "fftconv_bwd_workspace_bytes": (ctypes.c_size_t, [_vp]),
+    "fftconv_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp]),
+    "fftconv_plan_mma_flops": (ctypes.c_double, [_vp]),
     "fftconv_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int64,
                                            ctypes.c_int, ctypes.c_int]),
     "fftconv2d_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -131,6 +152,15 @@ class _PlanBase:
     def path(self) -> str:
         return self.lib.fftconv_plan_path(self._handle).decode()
 
+    @property
+    def mma_flops(self) -> float:
+        """Tensor-core flops of one forward call (0 for SIMT paths)."""
+        return float(self.lib.fftconv_plan_mma_flops(self._handle))
+
+    def set_wait_limit(self, probes: int = DEFAULT_WAIT_PROBES):
+        """Probes per bounded device wait (0: give up at the first check)."""
+        _check(self.lib.fftconv_plan_set_wait_limit(self._handle, int(probes)), "fftconv_plan_set_wait_limit")
+
     def device_status(self, stream=None) -> int:
         """Synchronise the stream; 0, or 6 (timed out) once after a launch whose device wait gave up."""
         return int(self.lib.fftconv_device_status(self._handle, _stream(stream)))
@@ -152,16 +182,29 @@ class _PlanBase:
         return workspace
 
 
-class Plan(_PlanBase):
-    """1-D plan: fftconv_plan_create(B, H, N, dtype, gated)."""
+def _options(lib, kernel: str, group_bytes: int) -> PlanOptions:
+    o = PlanOptions()
+    lib.fftconv_plan_options_init(ctypes.byref(o))
+    o.kernel = KERNELS[kernel]
+    o.group_bytes = int(group_bytes)
+    return o
 
-    def __init__(self, B: int, H: int, N: int, dtype: str = "bf16", gated: bool = False):
+
+class Plan(_PlanBase):
+    """1-D plan: fftconv_plan_create_ex(B, H, N, dtype, gated, options).
+
+    kernel: "auto" (default), "simt", "mma_sync" or "tcgen05"; group_bytes:
+    multi-pass workspace per group of row pairs (0 = the library default)."""
+
+    def __init__(self, B: int, H: int, N: int, dtype: str = "bf16", gated: bool = False, kernel: str = "auto",
+                 group_bytes: int = 0):
         self.lib = load_library()
         self.B, self.H, self.N, self.dtype, self.gated = B, H, N, dtype, bool(gated)
         self.torch_dtype = TORCH_DTYPES[dtype]
         h = ctypes.c_void_p()
-        _check(self.lib.fftconv_plan_create(ctypes.byref(h), B, H, N, DTYPES[dtype], int(bool(gated))),
-               "fftconv_plan_create")
+        opts = _options(self.lib, kernel, group_bytes)
+        _check(self.lib.fftconv_plan_create_ex(ctypes.byref(h), B, H, N, DTYPES[dtype], int(bool(gated)),
+                                               ctypes.byref(opts)), "fftconv_plan_create_ex")
         self._handle = h
         self._workspace = None
 
@@ -201,16 +244,76 @@ class Plan(_PlanBase):
         return y
 
 
-class Plan2D(_PlanBase):
-    """2-D plan: fftconv2d_plan_create(B, C, Hs, Ws, dtype)."""
+    def fwd_dynamic(self, u: torch.Tensor, k: torch.Tensor, D: Optional[torch.Tensor] = None,
+                    v: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None,
+                    y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """y with one filter per batch row: k [B, H, L] fp32, transformed in the same launch."""
+        shape = (self.B, self.H, self.N)
+        _need(u, "u", shape, self.torch_dtype)
+        if k.dim() != 3:
+            raise ValueError("k must be [B, H, L]")
+        _need(k, "k", (self.B, self.H, k.shape[2]), torch.float32)
+        if self.gated:
+            _need(v, "v", shape, self.torch_dtype)
+            _need(w, "w", shape, self.torch_dtype)
+        if D is not None:
+            _need(D, "D", (self.H,), torch.float32)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        _check(self.lib.fftconv_fwd_dynamic(self._handle, _ptr(u), _ptr(v), _ptr(w), _ptr(k), k.shape[2], _ptr(D),
+                                            _ptr(y), _stream(stream)), "fftconv_fwd_dynamic")
+        return y
 
-    def __init__(self, B: int, C: int, Hs: int, Ws: int, dtype: str = "bf16"):
+    def spectrum_conjugate(self, khat: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """conj(khat) in the plan's layout: the spectrum of the correlation with k."""
+        if out is None:
+            out = torch.empty_like(khat)
+        _check(self.lib.fftconv_spectrum_conjugate(self._handle, _ptr(khat), _ptr(out), _stream(stream)),
+               "fftconv_spectrum_conjugate")
+        return out
+
+    @property
+    def bwd_workspace_bytes(self) -> int:
+        return int(self.lib.fftconv_bwd_workspace_bytes(self._handle))
+
+    def bwd(self, dy: torch.Tensor, u: torch.Tensor, khat: torch.Tensor, khat_conj: torch.Tensor,
+            D: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None,
+            L: int = 0, filter_grad: bool = True, stream=None) -> dict:
+        """Gradients of y = fwd(u, khat, D, v, w) for the upstream gradient dy:
+        du (dv, dw gated) of the plan's dtype, dk [H, L] and dD [H] fp32
+        (dk only with filter_grad, dD only with D)."""
+        shape = (self.B, self.H, self.N)
+        _need(dy, "dy", shape, self.torch_dtype)
+        _need(u, "u", shape, self.torch_dtype)
+        if self.gated:
+            _need(v, "v", shape, self.torch_dtype)
+            _need(w, "w", shape, self.torch_dtype)
+        du = torch.empty_like(u)
+        dv = torch.empty_like(u) if self.gated else None
+        dw = torch.empty_like(u) if self.gated else None
+        L = L or self.N
+        dk = torch.empty(self.H, L, dtype=torch.float32, device=u.device) if filter_grad else None
+        dD = torch.empty(self.H, dtype=torch.float32, device=u.device) if (filter_grad and D is not None) else None
+        n = self.bwd_workspace_bytes
+        ws = torch.empty(n, dtype=torch.uint8, device=u.device) if n else None
+        _check(self.lib.fftconv_bwd(self._handle, _ptr(dy), _ptr(u), _ptr(v), _ptr(w), _ptr(khat), _ptr(khat_conj),
+                                    _ptr(D), L, _ptr(du), _ptr(dv), _ptr(dw), _ptr(dk), _ptr(dD), _ptr(ws),
+                                    _stream(stream)), "fftconv_bwd")
+        return {"du": du, "dv": dv, "dw": dw, "dk": dk, "dD": dD}
+
+
+class Plan2D(_PlanBase):
+    """2-D plan: fftconv2d_plan_create_ex(B, C, Hs, Ws, dtype, options)."""
+
+    def __init__(self, B: int, C: int, Hs: int, Ws: int, dtype: str = "bf16", kernel: str = "auto",
+                 group_bytes: int = 0):
         self.lib = load_library()
         self.B, self.C, self.Hs, self.Ws, self.dtype = B, C, Hs, Ws, dtype
         self.torch_dtype = TORCH_DTYPES[dtype]
         h = ctypes.c_void_p()
-        _check(self.lib.fftconv2d_plan_create(ctypes.byref(h), B, C, Hs, Ws, DTYPES[dtype]),
-               "fftconv2d_plan_create")
+        opts = _options(self.lib, kernel, group_bytes)
+        _check(self.lib.fftconv2d_plan_create_ex(ctypes.byref(h), B, C, Hs, Ws, DTYPES[dtype], ctypes.byref(opts)),
+               "fftconv2d_plan_create_ex")
         self._handle = h
         self._workspace = None
 

@@ -251,7 +251,7 @@ __device__ __forceinline__ void outer_step1(uint32_t xre, uint32_t xim, uint32_t
 template <int NW, bool IP>
 __device__ __forceinline__ bool outer_step1_umma(uint32_t xre, uint32_t xim, uint32_t rsm, uint32_t sre, uint32_t sim,
                                                  uint32_t tmem, uint32_t mbar, uint32_t phase, int tid, int lane,
-                                                 int warp, const TcTables& tb) {
+                                                 int warp, const TcTables& tb, uint32_t wait_limit) {
     constexpr int P = 128;
     static_assert(NW == 16, "one warp per (tile, lane quarter, column half)");
     if (tid == 0) {
@@ -297,7 +297,7 @@ __device__ __forceinline__ bool outer_step1_umma(uint32_t xre, uint32_t xim, uin
         }
     };
     fetch_tw(0);
-    const bool ok = um::mbar_wait(mbar + 8u * t, phase);
+    const bool ok = um::mbar_wait(mbar + 8u * t, phase, wait_limit);
     um::fence_after();
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
@@ -342,7 +342,8 @@ template <int P, int NW, bool GATED>
 __global__ void __launch_bounds__(NW * 32, P <= 32 ? 3 : (P <= 64 ? 2 : 1))
 fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
              const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
-             __nv_bfloat16* __restrict__ y, TcTables tb, int* __restrict__ err, int B, int H) {
+             __nv_bfloat16* __restrict__ y, TcTables tb, int* __restrict__ err, int B, int H,
+             uint32_t wait_limit) {
     using S = TcShape<P>;
     using SM = TcSmem<P, GATED>;
     static_assert(P >= 16 && P <= 128, "outer factor");
@@ -444,7 +445,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     // 224 KiB of shared memory leaves no room on the SM for a second CTA of it or
     // of the other TMEM user (the tcgen05 kernel of 2N <= 8192, 40-80 KiB each)
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(8) uint64_t s_mbar[2];
+    __shared__ __align__(8) uint64_t s_mbar[3];  // tile 0, tile 1, drain
     uint32_t tmem = 0, mphase = 0;
     const uint32_t mbar = smem_u32(&s_mbar[0]);
     if constexpr (SM::kUM1) {
@@ -455,6 +456,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
         if (tid == 0) {
             um::mbar_init(mbar, 1);
             um::mbar_init(mbar + 8u, 1);
+            um::mbar_init(mbar + 16u, 1);
         }
         um::fence_before();
         __syncthreads();
@@ -463,6 +465,7 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     }
     if ((int)blockIdx.x < items) stage_input(blockIdx.x, 3, 0);
 
+    bool dead = false;  // a bounded wait of this CTA gave up (P = 128 only)
     int k = 0;  // items done by this CTA
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++k) {
         const int h = item / npp, b0 = 2 * (item % npp);
@@ -507,13 +510,19 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
             }
             um::fence_proxy_async();  // the staged (and gated) x is read by the tensor core
             __syncthreads();
-            if (!outer_step1_umma<NW, IP>(xre, xim, rsm, sre, sim, tmem, mbar, mphase, tid, lane, warp, tb))
-                atomicExch(err, 1);
+            const bool ok =
+                outer_step1_umma<NW, IP>(xre, xim, rsm, sre, sim, tmem, mbar, mphase, tid, lane, warp, tb, wait_limit);
             mphase ^= 1u;
+            // a wait that gave up abandons the launch: the whole CTA leaves the item loop
+            // (its S holds garbage) and drains the products before freeing TMEM below
+            if (__syncthreads_or(!ok)) {
+                dead = true;
+                break;
+            }
         } else {
             outer_step1<P, NW, GATED, PRE1, IP, SM::kRS>(xre, xim, wre, wim, sre, sim, lane, warp, fp, tb, rsm);
+            __syncthreads();
         }
-        __syncthreads();
         // the staging planes are free: fetch the next item while this one runs
         if (SM::kNBuf == 1 && item + (int)gridDim.x < items) stage_input(item + gridDim.x, SM::kWInS ? 1 : 3, 0);
 
@@ -671,9 +680,17 @@ fused_fwd_tc(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restric
     }
     cp_async_wait_all();
     if constexpr (SM::kUM1) {
+        // drain: the issuing thread commits once more and waits (bounded, default
+        // limit) until every product it issued is complete; TMEM is freed only then
+        __shared__ int s_drained;
+        if (tid == 0) {
+            um::mma_commit(mbar + 16u);
+            s_drained = um::mbar_wait(mbar + 16u, 0u) ? 1 : 0;
+            if (dead || !s_drained) atomicExch(err, 1);
+        }
         um::fence_before();
         __syncthreads();
-        if (warp == 0) {
+        if (warp == 0 && s_drained) {
             um::fence_after();
             um::tmem_dealloc(tmem, 512);
         }
@@ -965,7 +982,8 @@ static cudaError_t tc_fwd_go(const fftconv_plan_s& p, const void* u, const void*
     const int items = ((p.B + 1) / 2) * p.H;
     dim3 grid(items < resident ? items : resident);
     kern<<<grid, NW * 32, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
-                                     (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.d_err, p.B, p.H);
+                                     (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, p.d_err, p.B, p.H,
+                                     p.wait_limit);
     return cudaGetLastError();
 }
 

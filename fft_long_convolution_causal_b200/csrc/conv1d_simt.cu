@@ -23,6 +23,8 @@
 //   pass 3: per column n2, inverse DFT_N1, only n1 < N1/2 (n < N) kept.
 // Pairs are processed in groups (the plan sizes them, up to 1 GiB of
 // workspace) and the workspace is reused group after group.
+#include <cuda_bf16.h>
+
 #include "fft_simt.cuh"
 #include "plan.h"
 #include "tables.h"
@@ -130,6 +132,164 @@ fused_spectrum_simt(const float* __restrict__ k, int L, float2* __restrict__ kha
         tid, tw, lds, [&](int i, int, float2 z) { out[i] = cscale(z, 1.0f / M); });
 }
 
+// The spectrum in the layout of the two-stage tensor-core kernel (2N = 8192 =
+// 128 x 64, frequency k = k_p + 128 c): per channel, row k_p and column half
+// c / 32, 32 words: 16 bf16 pairs of Re (c, c + 1) then 16 of -Im, scaled 1/M.
+__global__ void __launch_bounds__(FusedG<13>::T)
+t2_spectrum_simt(const float* __restrict__ k, int L, uint16_t* __restrict__ khat, const float2* __restrict__ tw) {
+    using G = FusedG<13>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, NS = G::Plan::kStages;
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, h = blockIdx.x;
+    const float* __restrict__ kr = k + (size_t)h * L;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return make_float2(n < L ? kr[n] : 0.f, 0.f); }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, false>(smem, tid, tw);
+    uint16_t* __restrict__ out = khat + (size_t)h * M * 2;
+    stage<G, NS - 1, false, RL, RL, false>(tid, tw, lds, [&](int i, int, float2 z) {
+        const int kp = i & 127, c = i >> 7;
+        const size_t word = ((size_t)kp * 2 + (c >> 5)) * 32 + ((c & 31) >> 1);
+        const __nv_bfloat16 re = __float2bfloat16_rn(z.x * (1.0f / M)), nim = __float2bfloat16_rn(-z.y * (1.0f / M));
+        out[2 * word + (c & 1)] = *reinterpret_cast<const uint16_t*>(&re);
+        out[2 * (word + 16) + (c & 1)] = *reinterpret_cast<const uint16_t*>(&nim);
+    });
+}
+
+// Filter gradient of the backward pass, one CTA per channel: for every pair
+// of batch rows, Zx = DFT_M(pad(x_b + i x_b+1)) and Zg = DFT_M(pad(g_b + i g_b+1))
+// (x = u or u w, g = dy or dy v), accumulated as T = sum conj(Zx) Zg in acc
+// ([H][M] fp32 complex, each thread its own frequencies f = tid + T m).  The
+// real part of the inverse of T is sum_b corr(g_b, x_b): the cross terms of
+// the packed pair land in the imaginary part.  dk[h][j] = that at lags
+// j < L, dD[h] = that at lag 0 (when dD is given).
+template <int LOG2M, typename IO, bool GATED>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+kgrad_simt(const IO* __restrict__ u, const IO* __restrict__ w, const IO* __restrict__ dy, const IO* __restrict__ v,
+           float2* __restrict__ acc, float* __restrict__ dk, float* __restrict__ dD, const float2* __restrict__ tw,
+           int B, int H, int L) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, N = M / 2, NS = G::Plan::kStages, T = G::T, FPT = M / T;
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, h = blockIdx.x;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    float2* __restrict__ a = acc + (size_t)h * M;
+    const int npp = (B + 1) / 2;
+    for (int pp = 0; pp < npp; ++pp) {
+        const int b0 = 2 * pp;
+        const bool has1 = b0 + 1 < B;
+        const size_t row0 = ((size_t)b0 * H + h) * N;
+        const size_t row1 = ((size_t)(b0 + 1) * H + h) * N;
+        stage<G, 0, false, R0 / 2, R0, false>(
+            tid, tw, [&](int n, int) { return load_pair<IO, GATED>(u, w, row0, row1, has1, n); }, sts);
+        __syncthreads();
+        smem_stages<G, 1, NS, false>(smem, tid, tw);
+        float2 zx[FPT];
+#pragma unroll
+        for (int m = 0; m < FPT; ++m) zx[m] = smem[Lay::at(tid + T * m, 0)];
+        __syncthreads();
+        stage<G, 0, false, R0 / 2, R0, false>(
+            tid, tw, [&](int n, int) { return load_pair<IO, GATED>(dy, v, row0, row1, has1, n); }, sts);
+        __syncthreads();
+        smem_stages<G, 1, NS, false>(smem, tid, tw);
+#pragma unroll
+        for (int m = 0; m < FPT; ++m) {
+            const int f = tid + T * m;
+            const float2 t = cmulc(smem[Lay::at(f, 0)], zx[m]);  // Zg conj(Zx)
+            a[f] = pp == 0 ? t : cadd(a[f], t);
+        }
+        __syncthreads();
+    }
+    // inverse DFT of T (unnormalised), real part / M at lags n < N
+#pragma unroll
+    for (int m = 0; m < FPT; ++m) smem[Lay::at(tid + T * m, 0)] = a[tid + T * m];
+    __syncthreads();
+    smem_stages<G, 0, NS - 1, true>(smem, tid, tw);
+    stage<G, NS - 1, true, RL, RL / 2, false>(tid, tw, lds, [&](int n, int, float2 z) {
+        const float c = z.x * (1.0f / M);
+        if (dk && n < L) dk[(size_t)h * L + n] = c;
+        if (n == 0 && dD) dD[h] = c;
+    });
+}
+
+// Input-dependent filters ("Native Multi-Dimensional Subquadratic Operators
+// via Input Dependent Long Convolutions", abstract: input-dependent long
+// convolutions), one CTA per (pair of batch rows, channel), 2N <= 8192: each
+// row's filter k[b][h] is transformed in the same launch.  Row b is packed
+// with its own filter, z = x_b + i k_b, so one transform gives both spectra
+// (X = (Z[f] + conj Z[-f]) / 2, K = (Z[f] - conj Z[-f]) / 2i); the products
+// P_b = X_b (K_b + D) of the two rows are packed again, W = P_b + i P_b+1
+// (P is Hermitian, so W[-f] = conj P_b[f] + i conj P_b+1[f]), and one inverse
+// transform gives both outputs.  Two transforms in shared memory.
+template <int LOG2M, typename IO, bool GATED>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+fused_dyn_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __restrict__ w,
+               const float* __restrict__ k, int L, const float* __restrict__ D, IO* __restrict__ y,
+               const float2* __restrict__ tw, int B, int H) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, N = M / 2, NS = G::Plan::kStages;
+    static_assert(NS >= 2, "transform too short");
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    float2* sa = smem;
+    float2* sb = smem + Lay::kWords;
+    const int tid = threadIdx.x, h = blockIdx.y;
+    const int b0 = 2 * blockIdx.x;
+    const bool has1 = b0 + 1 < B;
+    const size_t row0 = ((size_t)b0 * H + h) * N;
+    const size_t row1 = ((size_t)(b0 + 1) * H + h) * N;
+    const float* __restrict__ k0 = k + ((size_t)b0 * H + h) * L;
+    const float* __restrict__ k1 = k + ((size_t)(b0 + 1) * H + h) * L;
+    // z_b = x_b + i k_b, zero-padded, for both rows
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw,
+        [&](int n, int) {
+            const float2 xx = load_pair<IO, GATED>(u, w, row0, row1, false, n);
+            return make_float2(xx.x, n < L ? k0[n] : 0.f);
+        },
+        [&](int i, int, float2 z) { sa[Lay::at(i, 0)] = z; });
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw,
+        [&](int n, int) {
+            if (!has1) return make_float2(0.f, 0.f);
+            const float2 xx = load_pair<IO, GATED>(u, w, row1, row1, false, n);
+            return make_float2(xx.x, n < L ? k1[n] : 0.f);
+        },
+        [&](int i, int, float2 z) { sb[Lay::at(i, 0)] = z; });
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(sa, tid, tw);
+    smem_stages<G, 1, NS, false>(sb, tid, tw);
+    // P = X (K + D) per row, packed W = P_b + i P_b+1 (scaled 1/M) into sa
+    const float dd = D ? D[h] : 0.f;
+    auto prod = [&](float2 zf, float2 zg) {
+        const float2 X = make_float2(0.5f * (zf.x + zg.x), 0.5f * (zf.y - zg.y));
+        const float2 K = make_float2(0.5f * (zf.y + zg.y) + dd, 0.5f * (zg.x - zf.x));
+        return cmul(X, K);
+    };
+    for (int f = tid; f <= M / 2; f += G::T) {
+        const int g = (M - f) & (M - 1);
+        const float2 af = sa[Lay::at(f, 0)], ag = sa[Lay::at(g, 0)];
+        const float2 bf = sb[Lay::at(f, 0)], bg = sb[Lay::at(g, 0)];
+        const float2 p1 = prod(af, ag), p2 = prod(bf, bg);
+        constexpr float s = 1.0f / M;
+        sa[Lay::at(f, 0)] = make_float2((p1.x - p2.y) * s, (p1.y + p2.x) * s);
+        if (g != f) sa[Lay::at(g, 0)] = make_float2((p1.x + p2.y) * s, (p2.x - p1.y) * s);
+    }
+    __syncthreads();
+    smem_stages<G, 0, NS - 1, true>(sa, tid, tw);
+    stage<G, NS - 1, true, RL, RL / 2, false>(
+        tid, tw, [&](int i, int) { return sa[Lay::at(i, 0)]; },
+        [&](int n, int, float2 z) { store_pair<IO, GATED>(y, v, row0, row1, has1, n, z); });
+}
+
 template <int LOG2M>
 static size_t fused_smem() { return FusedG<LOG2M>::Lay::kWords * sizeof(float2); }
 
@@ -193,6 +353,82 @@ cudaError_t launch_fused_fwd(const fftconv_plan_s& p, const void* u, const void*
         case 14: return fused_fwd_dtype<14>(p, u, v, w, khat, D, y, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <int LOG2M, typename IO, bool GATED>
+static cudaError_t kgrad_go(const fftconv_plan_s& p, const void* u, const void* w, const void* dy, const void* v,
+                            float2* acc, float* dk, float* dD, int L, cudaStream_t s) {
+    auto kern = kgrad_simt<LOG2M, IO, GATED>;
+    const size_t smem = fused_smem<LOG2M>();
+    ensure_smem(kern, smem);
+    kern<<<p.H, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)w, (const IO*)dy, (const IO*)v, acc, dk, dD,
+                                              p.tw.wL, p.B, p.H, L);
+    return cudaGetLastError();
+}
+
+template <int LOG2M>
+static cudaError_t kgrad_dt(const fftconv_plan_s& p, const void* u, const void* w, const void* dy, const void* v,
+                            float2* acc, float* dk, float* dD, int L, cudaStream_t s) {
+    if (p.dtype == FFTCONV_BF16)
+        return p.gated ? kgrad_go<LOG2M, __nv_bfloat16, true>(p, u, w, dy, v, acc, dk, dD, L, s)
+                       : kgrad_go<LOG2M, __nv_bfloat16, false>(p, u, w, dy, v, acc, dk, dD, L, s);
+    return p.gated ? kgrad_go<LOG2M, float, true>(p, u, w, dy, v, acc, dk, dD, L, s)
+                   : kgrad_go<LOG2M, float, false>(p, u, w, dy, v, acc, dk, dD, L, s);
+}
+
+bool kgrad_supported(int log2M) { return log2M >= 7 && log2M <= 14; }
+
+template <int LOG2M, typename IO, bool GATED>
+static cudaError_t dyn_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
+                          int L, const float* D, void* y, cudaStream_t s) {
+    auto kern = fused_dyn_simt<LOG2M, IO, GATED>;
+    const size_t smem = 2 * fused_smem<LOG2M>();
+    ensure_smem(kern, smem);
+    dim3 grid((p.B + 1) / 2, p.H);
+    kern<<<grid, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)v, (const IO*)w, k, L, D, (IO*)y, p.tw.wL,
+                                               p.B, p.H);
+    return cudaGetLastError();
+}
+
+template <int LOG2M>
+static cudaError_t dyn_dt(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
+                          int L, const float* D, void* y, cudaStream_t s) {
+    if (p.dtype == FFTCONV_BF16)
+        return p.gated ? dyn_go<LOG2M, __nv_bfloat16, true>(p, u, v, w, k, L, D, y, s)
+                       : dyn_go<LOG2M, __nv_bfloat16, false>(p, u, v, w, k, L, D, y, s);
+    return p.gated ? dyn_go<LOG2M, float, true>(p, u, v, w, k, L, D, y, s)
+                   : dyn_go<LOG2M, float, false>(p, u, v, w, k, L, D, y, s);
+}
+
+bool dyn_supported(int log2M) { return log2M >= 7 && log2M <= 13; }
+
+cudaError_t launch_dyn_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
+                           int64_t L, const float* D, void* y, cudaStream_t s) {
+    switch (p.log2M) {
+#define FFTC_D(X) case X: return dyn_dt<X>(p, u, v, w, k, (int)L, D, y, s);
+        FFTC_D(7) FFTC_D(8) FFTC_D(9) FFTC_D(10) FFTC_D(11) FFTC_D(12) FFTC_D(13)
+#undef FFTC_D
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_kgrad(const fftconv_plan_s& p, const void* u, const void* w, const void* dy, const void* v,
+                         float2* acc, float* dk, float* dD, int64_t L, cudaStream_t s) {
+    switch (p.log2M) {
+#define FFTC_K(X) case X: return kgrad_dt<X>(p, u, w, dy, v, acc, dk, dD, (int)L, s);
+        FFTC_K(7) FFTC_K(8) FFTC_K(9) FFTC_K(10) FFTC_K(11) FFTC_K(12) FFTC_K(13) FFTC_K(14)
+#undef FFTC_K
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_t2_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s) {
+    if (p.log2M != 13) return cudaErrorInvalidValue;
+    auto kern = t2_spectrum_simt;
+    const size_t smem = fused_smem<13>();
+    ensure_smem(kern, smem);
+    kern<<<p.H, FusedG<13>::T, smem, s>>>(k, (int)L, (uint16_t*)khat, p.tw.wL);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_fused_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, float2* khat,

@@ -92,6 +92,7 @@ constexpr int kUmmaThreads = kUmmaCompute + 32;
 struct UBars {
     uint64_t afull[3];
     uint64_t dfull[3];
+    uint64_t drain;  // the issuer's last commit: every MMA it issued is complete
 };
 
 template <int P, bool GATED>
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ v,
                const __nv_bfloat16* __restrict__ w, const uint4* __restrict__ khat, const float* __restrict__ D,
                __nv_bfloat16* __restrict__ y, TcTables tb, const uint4* __restrict__ bimg, int* __restrict__ err,
-               int B, int H) {
+               int B, int H, uint32_t wait_limit) {
     using S = TcShape<P>;
     using U = UShape<P>;
     using SM = USmem<P, GATED>;
@@ -108,6 +109,7 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ __align__(8) UBars s_bar;
+    __shared__ int s_drained;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m8 = lane >> 3, r8 = lane & 7;
     const int npp = (B + 1) / 2;
@@ -135,6 +137,7 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
             um::mbar_init(afull + 8 * i, kUmmaCompute / 32);
             um::mbar_init(dfull + 8 * i, 1);
         }
+        um::mbar_init(tc::smem_u32(&s_bar.drain), 1);
     }
     um::fence_before();
     __syncthreads();
@@ -148,7 +151,7 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
                            id3 = um::idesc_bf16(128, U::N3);
             uint32_t pa[3] = {0u, 0u, 0u};
             auto wait_a = [&](int i) {
-                const bool ok = um::mbar_wait(afull + 8 * i, pa[i]);
+                const bool ok = um::mbar_wait(afull + 8 * i, pa[i], wait_limit);
                 pa[i] ^= 1u;
                 um::fence_after();
                 return ok;
@@ -196,7 +199,11 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
                 }
                 um::mma_commit(dfull + 16);
             }
-            if (!ok) atomicExch(err, 1);
+            // drain: one more commit, waited for with the default limit, so that no
+            // product is in flight when TMEM is freed (after a give-up as well)
+            um::mma_commit(tc::smem_u32(&s_bar.drain));
+            s_drained = um::mbar_wait(tc::smem_u32(&s_bar.drain), 0u) ? 1 : 0;
+            if (!ok || !s_drained) atomicExch(err, 1);
         }
     } else {
         // ================= compute warps: TMEM lanes 32 q + 16 r .. + 15 of every 128-lane tile
@@ -216,7 +223,7 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
         };
         // wait for slot i's products (bounded); a timeout marks the CTA dead at the next named barrier
         auto wait_d = [&](int i) {
-            const bool ok = um::mbar_wait(dfull + 8 * i, pd[i]);
+            const bool ok = um::mbar_wait(dfull + 8 * i, pd[i], wait_limit);
             pd[i] ^= 1u;
             um::fence_after();
             dead |= !ok;
@@ -518,10 +525,12 @@ fused_fwd_umma(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restr
         cp_async_wait_all();
         if (dead && tid == 0) atomicExch(err, 1);
     }
-    // every wait above is bounded; in normal operation all MMAs are complete here
+    // every wait above is bounded, and the issuer has drained its products;
+    // should even that drain give up, TMEM is left allocated rather than freed
+    // under a running product (the status word is set)
     um::fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0 && s_drained) {
         um::fence_after();
         um::tmem_dealloc(tmem, U::kCols);
     }
@@ -655,7 +664,7 @@ static cudaError_t umma_fwd_go(const fftconv_plan_s& p, const void* u, const voi
     dim3 grid(items < resident ? items : resident);
     kern<<<grid, tc::kUmmaThreads, smem, s>>>((const __nv_bfloat16*)u, (const __nv_bfloat16*)v, (const __nv_bfloat16*)w,
                                  (const uint4*)khat, D, (__nv_bfloat16*)y, p.tc, (const uint4*)p.umma_b, p.d_err,
-                                 p.B, p.H);
+                                 p.B, p.H, p.wait_limit);
     return cudaGetLastError();
 }
 

@@ -17,12 +17,29 @@ constexpr int kFusedMaxLog2M = 14;
 // Workspace of one multi-pass / 2-D group: the pairs a pass covers per
 // launch.  Measured on B200 (same box, both builds): fewer, larger launches
 // beat groups sized to stay in L2 -- 1 GiB against 64 MiB is 14% faster at
-// N = 2^20 and 17% faster on 256 x 256 images.  FFTCONV_GROUP_MB (MiB, read
-// at plan creation) overrides it, e.g. to exercise several groups in tests.
-size_t group_bytes() {
-    const char* e = getenv("FFTCONV_GROUP_MB");
-    const long mb = e ? atol(e) : 0;
-    return mb > 0 ? (size_t)mb << 20 : size_t(1) << 30;
+// N = 2^20 and 17% faster on 256 x 256 images.  The plan option group_bytes
+// overrides it (smaller workspaces; the tests use it to run several groups).
+size_t group_bytes(const fftconv_plan_options& o) { return o.group_bytes ? o.group_bytes : size_t(1) << 30; }
+
+fftconv_plan_options defaults() {
+    fftconv_plan_options o;
+    o.kernel = FFTCONV_KERNEL_AUTO;
+    o.group_bytes = 0;
+    return o;
+}
+
+bool valid_options(const fftconv_plan_options& o) {
+    return o.kernel >= FFTCONV_KERNEL_AUTO && o.kernel <= FFTCONV_KERNEL_TCGEN05;
+}
+
+// The plan's device must be current for every call that launches on it.
+bool on_plan_device(const fftconv_plan_s* p) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return dev == p->device;
 }
 
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -73,6 +90,38 @@ fftconv_status cuda_status(cudaError_t e) {
 
 }  // namespace
 
+namespace fftc {
+
+// Tensor-core multiply-adds of one forward call, from each kernel's structure
+// (every product as issued, K padding included), times 2.
+double plan_mma_flops(const fftconv_plan_s& p) {
+    double mac_pair = 0.0;
+    if (p.path == PATH_FUSED_TC) {
+        if (p.t2) {
+            // two-stage kernel (2N = 128 x 64): four stages of 128 x 128 x 128 real
+            // products per pair (stage A and the last inverse stage as 128 x 64 halves)
+            mac_pair = 4.0 * 128 * 128 * 128;
+        } else {
+            // outer DFT_P over p < P/2 (K padded to 16), the 16 x 16 inner 256-point
+            // DFT forward and inverse per row k_p, outer inverse to p < P/2; complex
+            // products as four real ones
+            const double P = (double)((int64_t(1) << p.log2M) / 256);
+            const double kp1 = P / 2 < 16 ? 16 : P / 2;
+            mac_pair = 4.0 * 256 * (P * kp1 + (P / 2) * P) + 65536.0 * P;
+        }
+    } else if (p.path == PATH_2D && p.tc2d) {
+        // per 512-point line with 256 nonzero (or kept) points: two 256-point
+        // 16 x 16 DFTs of 2 x 4 x 16^3 real multiply-adds each
+        const double line = 2.0 * 2 * 4 * 4096;
+        const double cols = 2.0 * p.Ws * 2 * line;  // forward and inverse per column
+        const double rows = (p.Ws == 256) ? 2.0 * 256 * line : 0.0;
+        mac_pair = cols + rows;
+    }
+    return 2.0 * mac_pair * (double)p.pairs;
+}
+
+}  // namespace fftc
+
 extern "C" {
 
 const char* fftconv_status_string(fftconv_status s) {
@@ -88,12 +137,23 @@ const char* fftconv_status_string(fftconv_status s) {
     return "unknown status";
 }
 
-int fftconv_version(void) { return 100; }
+int fftconv_version(void) { return 200; }
+
+void fftconv_plan_options_init(fftconv_plan_options* opts) {
+    if (opts) *opts = defaults();
+}
 
 fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N, fftconv_dtype dtype,
                                    int gated) {
+    return fftconv_plan_create_ex(out, B, H, N, dtype, gated, nullptr);
+}
+
+fftconv_status fftconv_plan_create_ex(fftconv_plan_t* out, int B, int H, int64_t N, fftconv_dtype dtype,
+                                      int gated, const fftconv_plan_options* opts) {
     if (!out) return FFTCONV_ERR_INVALID_ARG;
     *out = nullptr;
+    const fftconv_plan_options o = opts ? *opts : defaults();
+    if (!valid_options(o)) return FFTCONV_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
     if (!is_pow2(N) || N < FFTCONV_MIN_N || N > FFTCONV_MAX_N) return FFTCONV_ERR_UNSUPPORTED;
     fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
@@ -106,18 +166,27 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
     p->gated = gated ? 1 : 0;
     p->log2M = log2i(2 * N);
     p->pairs = (int64_t)((B + 1) / 2) * H;
+    p->kernel = o.kernel;
     cudaGetDevice(&p->device);
     std::vector<float2> host;
     const int64_t M = int64_t(1) << p->log2M;
-    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0;
-    const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && !getenv("FFTCONV_NO_TC");
-    if (use_tc) {
+    size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0, offT2[2] = {0, 0};
+    const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && o.kernel != FFTCONV_KERNEL_SIMT;
+    if (use_tc && o.kernel == FFTCONV_KERNEL_TCGEN05 && fftc::t2_supported(p->log2M, p->gated)) {
+        // two-stage tcgen05 kernel, data in tensor memory between the stages
+        p->path = fftc::PATH_FUSED_TC;
+        p->t2 = true;
+        fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the SIMT spectrum transform
+        fftc::t2_tables(host, offT2);
+        p->spectrum_bytes = (size_t)H * M * sizeof(uint32_t);  // bf16 Re pairs and -Im pairs per row k_p
+        p->workspace_bytes = 0;
+    } else if (use_tc) {
         p->path = fftc::PATH_FUSED_TC;
         fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the spectrum transform
         fftc::tc_tables(p->log2M, host, offTc);
-        // tcgen05 kernel: opt-in (FFTCONV_UMMA=1) until it is the faster one
-        const char* um = getenv("FFTCONV_UMMA");
-        if (fftc::umma_supported(p->log2M) && um && um[0] == '1') {
+        // the tcgen05 kernel of the same factorisation: on request only (the
+        // mma.sync kernel measured faster at these sizes)
+        if (fftc::umma_supported(p->log2M) && o.kernel == FFTCONV_KERNEL_TCGEN05) {
             p->umma = true;
             fftc::umma_bimages(p->log2M, host, &offU);
         }
@@ -140,7 +209,7 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
         offHi = host.size();
         fill_roots(host, M, M / S, S);            // wHi: W_M^(e S)
         const size_t per_pair = (size_t)M * sizeof(float2);
-        int64_t g = (int64_t)(group_bytes() / per_pair);
+        int64_t g = (int64_t)(group_bytes(o) / per_pair);
         if (g < 1) g = 1;
         const int64_t most = p->pairs > H ? p->pairs : H;
         if (g > most) g = most;
@@ -157,13 +226,17 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
     const float2* base = (const float2*)p->d_tables;
     p->d_err = (int*)(base + offErr);
     if (p->umma) p->umma_b = base + offU;
+    if (p->t2) {
+        p->t2_mats = (const uint4*)(base + offT2[0]);
+        p->t2_twid = (const uint2*)(base + offT2[1]);
+    }
     p->tw.wL = base + offL;
     if (p->path == fftc::PATH_MULTIPASS) {
         p->tw.wC = base + offC;
         p->tw.wLo = base + offLo;
         p->tw.wHi = base + offHi;
     }
-    if (p->path == fftc::PATH_FUSED_TC) {
+    if (p->path == fftc::PATH_FUSED_TC && !p->t2) {
         p->tc.f16 = (const uint2*)(base + offTc[0]);
         p->tc.w256 = (const uint2*)(base + offTc[1]);
         p->tc.fp = (const uint2*)(base + offTc[2]);
@@ -177,8 +250,15 @@ fftconv_status fftconv_plan_create(fftconv_plan_t* out, int B, int H, int64_t N,
 }
 
 fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, int Ws, fftconv_dtype dtype) {
+    return fftconv2d_plan_create_ex(out, B, C, Hs, Ws, dtype, nullptr);
+}
+
+fftconv_status fftconv2d_plan_create_ex(fftconv_plan_t* out, int B, int C, int Hs, int Ws, fftconv_dtype dtype,
+                                        const fftconv_plan_options* opts) {
     if (!out) return FFTCONV_ERR_INVALID_ARG;
     *out = nullptr;
+    const fftconv_plan_options o = opts ? *opts : defaults();
+    if (!valid_options(o)) return FFTCONV_ERR_INVALID_ARG;
     if (B < 1 || C < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
     if (!is_pow2(Hs) || !is_pow2(Ws) || Hs < FFTCONV2D_MIN_SIDE || Ws < FFTCONV2D_MIN_SIDE ||
         Hs > FFTCONV2D_MAX_SIDE || Ws > FFTCONV2D_MAX_SIDE)
@@ -193,18 +273,19 @@ fftconv_status fftconv2d_plan_create(fftconv_plan_t* out, int B, int C, int Hs, 
     p->Ws = Ws;
     p->dtype = dtype;
     p->pairs = (int64_t)((B + 1) / 2) * C;
+    p->kernel = o.kernel;
     cudaGetDevice(&p->device);
     const int64_t LR = 2 * (int64_t)Ws, LC = 2 * (int64_t)Hs;
     std::vector<float2> host;
     size_t offR = 0, offC = 0, offT[4] = {0, 0, 0, 0};
     fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
-    if (fftc::c2tc_supported(Hs, Ws, dtype) && !getenv("FFTCONV_NO_TC")) {
+    if (fftc::c2tc_supported(Hs, Ws, dtype) && o.kernel != FFTCONV_KERNEL_SIMT) {
         p->tc2d = true;
         fftc::c2tc_tables(host, offT);
     }
     const size_t offErr = append_status_word(host);
     const size_t per_pair = (size_t)Hs * LR * sizeof(float2);
-    int64_t g = (int64_t)(group_bytes() / per_pair);
+    int64_t g = (int64_t)(group_bytes(o) / per_pair);
     // whole channels per group: a channel's pairs then run together and share
     // the channel's spectrum in L2
     const int64_t npp = (B + 1) / 2;
@@ -250,7 +331,7 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
     if (!p) return "none";
     switch (p->path) {
         case fftc::PATH_FUSED: return "fused";
-        case fftc::PATH_FUSED_TC: return p->umma ? "fused_umma" : "fused_tc";
+        case fftc::PATH_FUSED_TC: return p->t2 ? "fused_t2" : (p->umma ? "fused_umma" : "fused_tc");
         case fftc::PATH_MULTIPASS: return "multipass";
         case fftc::PATH_2D: return p->tc2d ? "2d_tc" : "2d";
     }
@@ -262,9 +343,12 @@ fftconv_status fftconv_kernel_spectrum(fftconv_plan_t p, const float* k, int64_t
     if (!p || p->kind != 1 || !k || !khat || L < 1 || L > p->N) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(khat)) return FFTCONV_ERR_INVALID_ARG;
     if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (p->path == fftc::PATH_FUSED_TC)
+    if (p->t2)
+        e = fftc::launch_t2_spectrum(*p, k, L, khat, s);
+    else if (p->path == fftc::PATH_FUSED_TC)
         e = fftc::launch_tc_spectrum(*p, k, L, khat, s);
     else if (p->path == fftc::PATH_FUSED)
         e = fftc::launch_fused_spectrum(*p, k, L, (float2*)khat, s);
@@ -283,10 +367,13 @@ fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const
         return FFTCONV_ERR_INVALID_ARG;
     if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
     if (y == u || y == v || y == w) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (p->path == fftc::PATH_FUSED_TC)
+    if (p->t2)
+        e = fftc::launch_t2_fwd(*p, u, khat, D, y, s);
+    else if (p->path == fftc::PATH_FUSED_TC)
         e = p->umma ? fftc::launch_umma_fwd(*p, u, v, w, khat, D, y, s) : fftc::launch_tc_fwd(*p, u, v, w, khat, D, y, s);
     else if (p->path == fftc::PATH_FUSED)
         e = fftc::launch_fused_fwd(*p, u, v, w, (const float2*)khat, D, y, s);
@@ -295,11 +382,26 @@ fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const
     return cuda_status(e);
 }
 
+fftconv_status fftconv_fwd_dynamic(fftconv_plan_t p, const void* u, const void* v, const void* w, const float* k,
+                                   int64_t L, const float* D, void* y, void* stream) {
+    if (!p || p->kind != 1 || !u || !k || !y) return FFTCONV_ERR_INVALID_ARG;
+    if (p->gated ? (!v || !w) : (v || w)) return FFTCONV_ERR_INVALID_ARG;
+    if (L < 1 || L > p->N) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(k) || !aligned16(y) || (v && !aligned16(v)) || (w && !aligned16(w)) ||
+        (D && !aligned16(D)))
+        return FFTCONV_ERR_INVALID_ARG;
+    if (y == u || y == v || y == w) return FFTCONV_ERR_INVALID_ARG;
+    if (!fftc::dyn_supported(p->log2M) || p->path == fftc::PATH_MULTIPASS) return FFTCONV_ERR_UNSUPPORTED;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    return cuda_status(fftc::launch_dyn_fwd(*p, u, v, w, k, L, D, y, (cudaStream_t)stream));
+}
+
 fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t p, const float* k, int Kh, int Kw, void* khat, void* work,
                                          void* stream) {
     if (!p || p->kind != 2 || !k || !khat || !work) return FFTCONV_ERR_INVALID_ARG;
     if (Kh < 1 || Kw < 1 || Kh > p->Hs || Kw > p->Ws) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(khat) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     cudaError_t e = fftc::launch_conv2d_spectrum(*p, k, Kh, Kw, (float2*)khat, (float2*)work, (cudaStream_t)stream);
     if (e == cudaSuccess) p->spectrum_ready = true;
     return cuda_status(e);
@@ -309,13 +411,23 @@ fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, 
     if (!p || p->kind != 2 || !u || !khat || !y || !work) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
     if (y == u) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     return cuda_status(
         fftc::launch_conv2d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream));
 }
 
+fftconv_status fftconv_plan_set_wait_limit(fftconv_plan_t p, uint32_t probes) {
+    if (!p) return FFTCONV_ERR_INVALID_ARG;
+    p->wait_limit = probes;
+    return FFTCONV_OK;
+}
+
+double fftconv_plan_mma_flops(fftconv_plan_t p) { return p ? fftc::plan_mma_flops(*p) : 0.0; }
+
 fftconv_status fftconv_device_status(fftconv_plan_t p, void* stream) {
     if (!p || !p->d_err) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FFTCONV_ERR_CUDA;
     int word = 0;
     if (cudaMemcpy(&word, p->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FFTCONV_ERR_CUDA;

@@ -25,10 +25,12 @@
 #include "fftconv.h"
 #include "plan.h"
 
+// the scratch array itself: file scope, internal linkage
+static __device__ __align__(256) uint8_t g_static_scratch[FFTCONV_STATIC_WORKSPACE_BYTES];
+
 namespace {
 
 constexpr size_t kStaticScratchBytes = FFTCONV_STATIC_WORKSPACE_BYTES;
-__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
@@ -66,6 +68,12 @@ fftconv_status fftconv_fwd_static_workspace(fftconv_plan_t p, const void* u, con
         (D && !aligned16(D)))
         return FFTCONV_ERR_INVALID_ARG;
     if (y == u || y == v || y == w) return FFTCONV_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FFTCONV_ERR_CUDA;
+    }
+    if (dev != p->device) return FFTCONV_ERR_INVALID_ARG;  // the plan's tables live on its own device
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     // one pair of rows needs a full transform of length 2N in fp32 complex
     const size_t per_pair = (size_t(1) << p->log2M) * sizeof(float2);

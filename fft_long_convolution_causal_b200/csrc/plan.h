@@ -64,12 +64,17 @@ struct fftconv_plan_s {
     fftc::Tables tw;
     fftc::TcTablePtrs tc;
     bool umma = false;              // fused tensor-core path on tcgen05 (else mma.sync)
+    bool t2 = false;                // two-stage tcgen05 kernel (2N = 8192)
+    const uint4* t2_mats = nullptr; // its shared-memory matrix image
+    const uint2* t2_twid = nullptr; // its twiddle pairs
     const void* umma_b = nullptr;   // tcgen05 path: B operand images of the DFT matrices
     int* d_err = nullptr;           // device status word: nonzero after a timed-out device wait
     bool tc2d = false;              // 2-D: column pass on the tensor cores (bf16, Hs = 256)
     fftc::C2TcTables c2tc;
     bool spectrum_ready = false;
     int device = 0;
+    int kernel = 0;                 // fftconv_kernel the caller asked for at creation
+    uint32_t wait_limit = 1u << 16; // probes per bounded device wait (fftconv_plan_set_wait_limit)
 };
 
 namespace fftc {
@@ -79,6 +84,22 @@ namespace fftc {
 bool fused_tables(int log2M, std::vector<float2>& out, size_t* offL);
 bool multipass_tables(int log2M, std::vector<float2>& out, size_t* offC, size_t* offR);
 bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_t* offC);
+
+// 1-D bf16 two-stage tcgen05 path (2N = 8192, ungated): tables, spectrum
+// (fp32 SIMT transform written in the kernel's bf16 layout), forward.
+bool t2_supported(int log2M, int gated);
+bool t2_tables(std::vector<float2>& out, size_t off[2]);
+cudaError_t launch_t2_spectrum(const fftconv_plan_s& p, const float* k, int64_t L, void* khat, cudaStream_t s);
+cudaError_t launch_t2_fwd(const fftconv_plan_s& p, const void* u, const void* khat, const float* D, void* y,
+                          cudaStream_t s);
+
+// Input-dependent filters, fused fp32 SIMT (2N <= 8192).
+bool dyn_supported(int log2M);
+cudaError_t launch_dyn_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
+                           int64_t L, const float* D, void* y, cudaStream_t s);
+
+// Tensor-core flops of one forward call (0 for SIMT paths).
+double plan_mma_flops(const fftconv_plan_s& p);
 
 // 1-D bf16 tensor-core fused path (2N in {4096, 8192, 16384}).
 bool tc_supported(int log2M);

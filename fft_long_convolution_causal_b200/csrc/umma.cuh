@@ -59,6 +59,22 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, u
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
         "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// D[tmem] (+)= A[smem] x B[smem]; issued by one thread
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// shared-memory matrix descriptor, no swizzle, with the core-matrix strides:
+// lbo between core matrices adjacent along K, sbo along M or N (both majors)
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// instruction-descriptor bits: negate the A x B product; A / B MN-major
+constexpr uint32_t kNegA = 1u << 13, kAmn = 1u << 15, kBmn = 1u << 16;
+
 // arrive on the mbarrier once every MMA issued so far by this thread is complete
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
@@ -79,11 +95,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Probes of a bounded wait by default (on the order of a second) and for the
+// drain that precedes freeing tensor memory after a wait gave up.
+constexpr uint32_t kDefaultWaitProbes = 1u << 16;
 // Bounded wait for the phase with the given parity to complete: false when
-// the limit (2^16 probes, on the order of a second) is reached first; the
-// caller then reports a timeout instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity) {
-    for (int i = 0; i < (1 << 16); ++i)
+// `limit` probes pass first (limit 0: give up at once); the caller then
+// reports a timeout instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, uint32_t limit = kDefaultWaitProbes) {
+    for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(addr, parity)) return true;
     return false;
 }
@@ -137,6 +156,28 @@ __device__ __forceinline__ void wait_ld(uint32_t* r) {
 #pragma unroll
     for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
 }
+// Shape 32x32b: thread t of the warp reads / writes TMEM lane (lane base of
+// taddr) + t, consecutive 32-bit columns from the column of taddr; register i
+// is column i.  Each warp may touch only its own quarter of the 128 lanes.
+__device__ __forceinline__ void ld32x32_x32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void st32x32_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 // one 16x16 bf16 A tile (re) and its partner (im) into 16 TMEM columns: the
 // A fragment registers (0: rows 0-7 k 0-7, 1: rows 8-15 k 0-7, 2: rows 0-7
 // k 8-15, 3: rows 8-15 k 8-15) go to columns so that column c holds

@@ -175,7 +175,8 @@ def make_config(name: str):
 
 def sample_points_1d(B, H, N, n_per_row, seed=0):
     """Seeded output positions for sampled parity: every row, the edge times
-    {0, 1, N/2-1, N/2, N-1}, the powers of two below N, plus uniform draws."""
+    {0, 1, N/2-1, N/2, N-1} and the powers of two below N, plus n_per_row
+    uniform draws on top of that fixed set."""
     rng = np.random.default_rng(1_000_003 + seed)
     fixed = sorted({0, 1, max(N // 2 - 1, 0), N // 2, N - 1} |
                    {1 << i for i in range(N.bit_length()) if (1 << i) < N})
@@ -183,7 +184,7 @@ def sample_points_1d(B, H, N, n_per_row, seed=0):
     bs, hs, ts = [], [], []
     for b in range(B):
         for h in range(H):
-            extra = rng.integers(0, N, size=max(n_per_row - len(fixed), 0))
+            extra = rng.integers(0, N, size=max(int(n_per_row), 0))
             tt = np.concatenate([np.asarray(fixed, dtype=np.int64), extra.astype(np.int64)])
             bs.append(np.full(tt.size, b, np.int64))
             hs.append(np.full(tt.size, h, np.int64))

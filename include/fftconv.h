@@ -75,6 +75,30 @@ typedef enum {
     FFTCONV_BF16 = 1  /* u, v, w, y in bf16; transforms on bf16 tensor cores, fp32 accumulate */
 } fftconv_dtype;
 
+/* Kernel family a plan may use (fftconv_plan_options.kernel).  Every choice
+ * computes the same convolution and passes the same parity tests; the choice
+ * exists for measurement and for callers that pin one implementation. */
+typedef enum {
+    FFTCONV_KERNEL_AUTO = 0,     /* the library's choice: the fastest measured kernel for the size  */
+    FFTCONV_KERNEL_SIMT = 1,     /* fp32 SIMT transforms only (bf16 I/O is still accepted)          */
+    FFTCONV_KERNEL_MMA_SYNC = 2, /* bf16 plans: warp-level mma.sync tensor-core kernels             */
+    FFTCONV_KERNEL_TCGEN05 = 3   /* bf16 plans: tcgen05 kernels where one exists for the size, else */
+                                 /* the AUTO choice                                                  */
+} fftconv_kernel;
+
+/* Plan options.  Zero-initialise, or call fftconv_plan_options_init, then set
+ * the fields to change; a NULL options pointer means the defaults. */
+typedef struct {
+    int kernel;          /* fftconv_kernel; default FFTCONV_KERNEL_AUTO                           */
+    size_t group_bytes;  /* multi-pass and 2-D paths: workspace per group of row pairs processed  */
+                         /* per launch; 0 = the default (1 GiB).  Smaller groups need less       */
+                         /* workspace and run more launches; a group always holds >= 1 pair.     */
+} fftconv_plan_options;
+
+/* Default probes of a bounded device wait (each probe sleeps up to about
+ * 20 us, so the default gives up after roughly a second). */
+#define FFTCONV_DEFAULT_WAIT_PROBES 65536u
+
 /* Supported sizes: 1-D N a power of two, FFTCONV_MIN_N <= N <= FFTCONV_MAX_N;
  * 2-D Hs, Ws powers of two in [FFTCONV2D_MIN_SIDE, FFTCONV2D_MAX_SIDE]. */
 #define FFTCONV_MIN_N 64
@@ -82,16 +106,29 @@ typedef enum {
 #define FFTCONV2D_MIN_SIDE 16
 #define FFTCONV2D_MAX_SIDE 256
 
+/* Fill *opts with the defaults. */
+FFTCONV_API void fftconv_plan_options_init(fftconv_plan_options* opts);
+
 /*
  * Create a 1-D plan for B batch rows, H channels, sequence length N, I/O type
  * dtype, gated (nonzero) or not.  Chooses the execution path: a single fused
  * kernel per (channel, pair of batch rows) when the transform of length 2N
- * fits on chip, else the multi-pass path that stages partial transforms in
- * the caller's workspace.  Uploads the plan's twiddle tables (synchronously).
- * On success *plan receives the handle.
+ * fits on chip ("FlashConv", Mechanism: FFT, product and inverse fused on
+ * chip), else the multi-pass path that stages partial transforms in the
+ * caller's workspace (same block: chunking past the on-chip capacity).
+ * Uploads the plan's twiddle tables (synchronously) on the current device,
+ * which every later call on the plan must also have current.  On success
+ * *plan receives the handle.  Same as fftconv_plan_create_ex with NULL
+ * options.
  */
 FFTCONV_API fftconv_status fftconv_plan_create(fftconv_plan_t* plan, int B, int H, int64_t N,
                                    fftconv_dtype dtype, int gated);
+
+/* fftconv_plan_create with options (NULL = defaults).  FFTCONV_ERR_INVALID_ARG
+ * for an unknown kernel choice. */
+FFTCONV_API fftconv_status fftconv_plan_create_ex(fftconv_plan_t* plan, int B, int H, int64_t N,
+                                                  fftconv_dtype dtype, int gated,
+                                                  const fftconv_plan_options* opts);
 
 /*
  * Create a 2-D plan: B images, C channels, Hs x Ws pixels, I/O type dtype.
@@ -99,6 +136,11 @@ FFTCONV_API fftconv_status fftconv_plan_create(fftconv_plan_t* plan, int B, int 
  */
 FFTCONV_API fftconv_status fftconv2d_plan_create(fftconv_plan_t* plan, int B, int C, int Hs, int Ws,
                                      fftconv_dtype dtype);
+
+/* fftconv2d_plan_create with options (NULL = defaults; FFTCONV_KERNEL_SIMT
+ * keeps bf16 plans off the tensor cores, the other choices mean AUTO). */
+FFTCONV_API fftconv_status fftconv2d_plan_create_ex(fftconv_plan_t* plan, int B, int C, int Hs, int Ws,
+                                                    fftconv_dtype dtype, const fftconv_plan_options* opts);
 
 /* Release a plan and its tables.  NULL is accepted.  Not valid while work
  * using the plan's tables is still pending on a stream. */
@@ -113,32 +155,67 @@ FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
 
 /* Name of the execution path the plan chose: "fused" (fp32 on-chip),
  * "fused_tc" (bf16 on-chip, 2N <= 32768, warp-level mma.sync tensor cores),
- * "fused_umma" (the same on tcgen05 tensor cores, 2N = 4096 or 8192, chosen
- * when the environment variable FFTCONV_UMMA=1 is set at plan creation),
- * "multipass", "2d". */
+ * "fused_umma" (the same factorisation on tcgen05 tensor cores, 2N = 4096 or
+ * 8192), "fused_t2" (two-stage tcgen05 kernel, data held in tensor memory
+ * between the stages, 2N = 8192), "multipass", "2d", "2d_tc". */
 FFTCONV_API const char* fftconv_plan_path(fftconv_plan_t plan);
+
+/* Tensor-core floating-point operations (2 per multiply-add, as executed,
+ * padding included) of one fftconv_fwd / fftconv2d_fwd call on this plan;
+ * 0 for paths that run no tensor-core products.  Lets a caller report the
+ * tensor-pipe fraction of a measured time. */
+FFTCONV_API double fftconv_plan_mma_flops(fftconv_plan_t plan);
+
+/* Probes each bounded device wait of this plan's kernels makes before it
+ * gives up (default FFTCONV_DEFAULT_WAIT_PROBES; 0 = give up at the first
+ * check).  A wait that gives up abandons its launch after draining the
+ * products it has in flight, leaves y incomplete and sets the status word
+ * that fftconv_device_status reports.  Takes effect from the next launch.
+ * Plans whose kernels never wait accept and ignore it. */
+FFTCONV_API fftconv_status fftconv_plan_set_wait_limit(fftconv_plan_t plan, uint32_t probes);
 
 /*
  * Kernel spectrum: khat <- DFT_{2N}(k[h] zero-padded) / (2N) for every
  * channel, in the plan's internal order and precision.  k is [H][L] fp32 on
- * the device with 1 <= L <= N (taps past L are zero: a partial convolution).
- * Computed once per filter set and reused by every fftconv_fwd of the plan.
+ * the device with 1 <= L <= N (taps past L are zero: a partial convolution,
+ * "FlashFFTConv", abstract).  Computed once per filter set and reused by
+ * every fftconv_fwd of the plan (the filter's FFT is the operand of the
+ * pointwise spectral product, "FlashConv", Mechanism).
  */
 FFTCONV_API fftconv_status fftconv_kernel_spectrum(fftconv_plan_t plan, const float* k, int64_t L,
                                        void* khat, void* workspace, void* stream);
 
 /*
- * Forward: y = the causal convolution above.  u is [B][H][N]; v and w are
- * [B][H][N] for a gated plan and must be NULL otherwise; khat is the output
- * of fftconv_kernel_spectrum on this plan; D is [H] fp32 or NULL (no skip
- * term); y is [B][H][N] and must not alias any input.
+ * Forward: y = the causal convolution above ("FlashFFTConv", abstract: the
+ * exact FFT convolution; "RubiConv -- Efficient Boundary-Respecting
+ * Convolutions", Caracal abstract: causal by padding to 2N and truncating).
+ * u is [B][H][N]; v and w are [B][H][N] for a gated plan and must be NULL
+ * otherwise; khat is the output of fftconv_kernel_spectrum on this plan; D is
+ * [H] fp32 or NULL (no skip term); y is [B][H][N] and must not alias any
+ * input.  FFTCONV_ERR_INVALID_ARG also when the current device is not the
+ * plan's.
  */
 FFTCONV_API fftconv_status fftconv_fwd(fftconv_plan_t plan, const void* u, const void* v, const void* w,
                            const void* khat, const float* D, void* y, void* workspace,
                            void* stream);
 
 /*
- * 2-D kernel spectrum: khat <- DFT_{2Hs x 2Ws}(k[c] zero-padded) / (4 Hs Ws).
+ * Forward with input-dependent filters: every batch row has its own filter,
+ *     y[b,h,:] = (x[b,h,:] * k[b,h,:])[:N] + D[h] x[b,h,:]   (gated: times v),
+ * the input-dependent long convolution of "Native Multi-Dimensional
+ * Subquadratic Operators via Input Dependent Long Convolutions" (abstract).
+ * k is [B][H][L] fp32 on the device, 1 <= L <= N, and is transformed inside
+ * the same launch (no cached spectrum; fftconv_kernel_spectrum is not needed).
+ * Other arguments as fftconv_fwd.  Runs an fp32 fused kernel for 2N <= 8192
+ * on any 1-D plan of that size; FFTCONV_ERR_UNSUPPORTED for longer N.
+ */
+FFTCONV_API fftconv_status fftconv_fwd_dynamic(fftconv_plan_t plan, const void* u, const void* v, const void* w,
+                                               const float* k, int64_t L, const float* D, void* y, void* stream);
+
+/*
+ * 2-D kernel spectrum: khat <- DFT_{2Hs x 2Ws}(k[c] zero-padded) / (4 Hs Ws)
+ * ("Native Multi-Dimensional Subquadratic Operators via Input Dependent Long
+ * Convolutions", abstract: global multi-dimensional kernels on the FFT path).
  * k is [C][Kh][Kw] fp32 with 1 <= Kh <= Hs, 1 <= Kw <= Ws.
  */
 FFTCONV_API fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t plan, const float* k, int Kh, int Kw,
@@ -147,10 +224,47 @@ FFTCONV_API fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t plan, const 
 /*
  * 2-D forward: y[b,c,i,j] = sum_{p<=i, q<=j} k[c,p,q] u[b,c,i-p,j-q] for
  * 0 <= i < Hs, 0 <= j < Ws (the first-quadrant crop of the zero-padded
- * linear convolution).  u, y: [B][C][Hs][Ws] of the plan's dtype.
+ * linear convolution, the 2-D analogue of [:N]; same page as the spectrum).
+ * u, y: [B][C][Hs][Ws] of the plan's dtype.  FFTCONV_ERR_INVALID_ARG also
+ * when the current device is not the plan's.
  */
 FFTCONV_API fftconv_status fftconv2d_fwd(fftconv_plan_t plan, const void* u, const void* khat, void* y,
                              void* workspace, void* stream);
+
+/*
+ * Conjugate spectrum: khat_conj <- conj(khat) in the plan's layout, the
+ * spectrum of the correlation with k (the backward pass's filter).  khat is
+ * the output of fftconv_kernel_spectrum on this plan; khat_conj is a buffer of
+ * fftconv_spectrum_bytes() bytes and may equal khat (in place).
+ */
+FFTCONV_API fftconv_status fftconv_spectrum_conjugate(fftconv_plan_t plan, const void* khat, void* khat_conj,
+                                                      void* stream);
+
+/* Bytes of device workspace fftconv_bwd needs (0: none). */
+FFTCONV_API size_t fftconv_bwd_workspace_bytes(fftconv_plan_t plan);
+
+/*
+ * Backward pass: the gradients of the forward's y with respect to its inputs
+ * for an upstream gradient dy ([B][H][N], the plan's dtype).  Training the
+ * learned long filters of "Simple Hardware-Efficient Long Convolutions for
+ * Sequence Modeling" (abstract) and of "FlashFFTConv" (abstract) needs them;
+ * the pages give no formula, so these are the chain rule of the forward:
+ *   g = dy (.) v (gated) or dy,  x = u (.) w (gated) or u
+ *   du = dx (.) w (gated) or dx,  dx[t] = sum_j k[j] g[t+j] + D g[t]
+ *   dw = dx (.) u,  dv = dy (.) (x * k + D x)          (gated plans only)
+ *   dk[h][j] = sum_b sum_t g[b,h,t] x[b,h,t-j], j < L  (fp32 [H][L])
+ *   dD[h] = sum_b sum_t g[b,h,t] x[b,h,t]              (fp32 [H])
+ * dx runs through the plan's forward kernel with khat_conj (the output of
+ * fftconv_spectrum_conjugate); dk and dD through an fp32 transform of the
+ * pairs (N <= 8192: otherwise FFTCONV_ERR_UNSUPPORTED when dk or dD is
+ * requested).  dk and dD may be NULL (not computed); dD requires D.  v, w, dv,
+ * dw must be given for a gated plan and NULL otherwise.  Outputs must not
+ * alias inputs.  workspace: fftconv_bwd_workspace_bytes() bytes.
+ */
+FFTCONV_API fftconv_status fftconv_bwd(fftconv_plan_t plan, const void* dy, const void* u, const void* v,
+                                       const void* w, const void* khat, const void* khat_conj, const float* D,
+                                       int64_t L, void* du, void* dv, void* dw, float* dk, float* dD,
+                                       void* workspace, void* stream);
 
 /*
  * Forward without a workspace argument: the same result as fftconv_fwd on a
@@ -184,10 +298,11 @@ FFTCONV_API size_t fftconv_static_workspace_bytes(void);
 /*
  * Device status of a plan: synchronises the stream, then reads and clears the
  * plan's device status word.  Kernels that wait on the tensor cores bound
- * every wait; a wait that gives up (the hardware never signalled) abandons
- * the launch, leaves y incomplete and sets the word.  Returns FFTCONV_OK, or
- * FFTCONV_ERR_TIMEOUT once after such a launch; FFTCONV_ERR_CUDA if the
- * synchronisation or the read fails.  No counterpart on the pages.
+ * every wait (fftconv_plan_set_wait_limit); a wait that gives up abandons
+ * the launch once the products in flight have drained, leaves y incomplete
+ * and sets the word.  Returns FFTCONV_OK, or FFTCONV_ERR_TIMEOUT once after
+ * such a launch; FFTCONV_ERR_CUDA if the synchronisation or the read fails.
+ * No counterpart on the pages.
  */
 FFTCONV_API fftconv_status fftconv_device_status(fftconv_plan_t plan, void* stream);
 

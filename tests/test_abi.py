@@ -97,3 +97,27 @@ def test_binding_refuses_missing_library(tmp_path, monkeypatch):
     monkeypatch.setattr(binding, "_LIB", None)
     with pytest.raises(FileNotFoundError):
         binding.load_library()
+
+
+def test_plan_options_defaults_and_validation(lib):
+    o = binding.PlanOptions()
+    o.kernel, o.group_bytes = 7, 123
+    lib.fftconv_plan_options_init(ctypes.byref(o))
+    assert (o.kernel, o.group_bytes) == (0, 0)
+    h = ctypes.c_void_p()
+    for bad in (-1, 4, 99):
+        o.kernel = bad
+        assert lib.fftconv_plan_create_ex(ctypes.byref(h), 1, 4, 1024, 0, 0, ctypes.byref(o)) == 1
+        assert lib.fftconv2d_plan_create_ex(ctypes.byref(h), 1, 1, 16, 16, 1, ctypes.byref(o)) == 1
+        assert not h.value
+    # size errors are reported the same way with or without options
+    o.kernel = 0
+    assert lib.fftconv_plan_create_ex(ctypes.byref(h), 1, 4, 1000, 0, 0, ctypes.byref(o)) == 2
+    assert lib.fftconv_plan_create_ex(ctypes.byref(h), 1, 4, 1000, 0, 0, None) == 2
+
+
+def test_null_plan_option_calls(lib):
+    assert lib.fftconv_plan_set_wait_limit(None, 0) == 1
+    assert lib.fftconv_plan_mma_flops(None) == 0.0
+    assert lib.fftconv_device_status(None, None) == 1
+    assert lib.fftconv_fwd_static_workspace(None, None, None, None, None, None, None, None) == 1

@@ -25,9 +25,13 @@ def _lib():
     binding.load_library()
 
 
-def run_1d(wl, khat_plan=None):
+def run_1d(wl, **plan_kw):
+    """One forward through the C ABI; returns (y, plan).  The device status
+    word of the plan that launched is read (and must be clear) after the
+    launch, so every parity case also checks that no bounded device wait of
+    its kernel gave up."""
     from fft_long_convolution_causal_b200 import binding
-    plan = binding.Plan(wl.B, wl.H, wl.N, wl.dtype, gated=wl.gated)
+    plan = binding.Plan(wl.B, wl.H, wl.N, wl.dtype, gated=wl.gated, **plan_kw)
     k = torch.from_numpy(wl.k).cuda()
     khat = plan.kernel_spectrum(k)
     u = to_dev(wl.u, wl.dtype)
@@ -36,7 +40,8 @@ def run_1d(wl, khat_plan=None):
     D = torch.from_numpy(wl.D).cuda() if wl.D is not None else None
     y = plan.fwd(u, khat, D=D, v=v, w=w)
     torch.cuda.synchronize()
-    return to_host(y), plan.path
+    assert plan.device_status() == 0, f"{plan.path}: a bounded device wait gave up"
+    return to_host(y), plan
 
 
 def oracle_full(wl):
@@ -51,9 +56,9 @@ FUSED_N = [64, 128, 256, 512, 1024, 2048, 4096, 8192]
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_fused_full_compare(N, dtype):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
-    y, path = run_1d(wl)
+    y, plan = run_1d(wl)
     want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 16384) else "fused"
-    assert path == want
+    assert plan.path == want
     assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}", scale=row_scale_1d(wl))
 
 
@@ -87,8 +92,8 @@ def test_partial_kernel(N, L):
 def test_tensor_core_path(N, B, gated, with_D, L):
     """bf16 tensor-core fused kernel: odd/even/single batch, gate, skip term, partial kernel."""
     wl = wlmod.make_1d(B, 3, N, dtype="bf16", gated=gated, seed=N + B, with_D=with_D, L=L)
-    y, path = run_1d(wl)
-    assert path == "fused_tc"
+    y, plan = run_1d(wl, kernel="mma_sync")
+    assert plan.path == "fused_tc"
     assert_close(y, oracle_full(wl), "bf16", f"tc N={N} B={B} gated={gated} D={with_D} L={L}",
                  gate=wl.v if gated else None, scale=row_scale_1d(wl))
 
@@ -96,18 +101,37 @@ def test_tensor_core_path(N, B, gated, with_D, L):
 @pytest.mark.parametrize("N", [2048, 4096])
 @pytest.mark.parametrize("B,gated,with_D,L", [(1, False, True, None), (5, True, True, None),
                                              (2, False, False, 333), (3, True, False, None), (8, False, True, None)])
-def test_umma_path(N, B, gated, with_D, L, monkeypatch):
-    """bf16 fused kernel on tcgen05 (opt-in at plan creation): same cases as the mma.sync kernel."""
-    monkeypatch.setenv("FFTCONV_UMMA", "1")
+def test_tcgen05_path(N, B, gated, with_D, L):
+    """bf16 fused kernels on tcgen05 (plan option kernel="tcgen05"): the
+    two-stage kernel for 2N = 8192 ungated, else the kernel with the mma.sync
+    kernel's factorisation; same cases as the mma.sync kernel.  run_1d checks
+    the status word of the plan that launched."""
     wl = wlmod.make_1d(B, 5, N, dtype="bf16", gated=gated, seed=3 * N + B, with_D=with_D, L=L)
-    y, path = run_1d(wl)
-    assert path == "fused_umma"
+    y, plan = run_1d(wl, kernel="tcgen05")
+    assert plan.path == ("fused_t2" if (N == 4096 and not gated) else "fused_umma")
     assert_close(y, oracle_full(wl), "bf16", f"umma N={N} B={B} gated={gated} D={with_D} L={L}",
                  gate=wl.v if gated else None, scale=row_scale_1d(wl))
-    from fft_long_convolution_causal_b200 import binding
-    plan = binding.Plan(B, 5, N, "bf16", gated=gated)
-    assert plan.path == "fused_umma"
-    assert plan.device_status() == 0
+
+
+@pytest.mark.parametrize("B,H,with_D,L", [(1, 3, True, None), (3, 4, True, None), (6, 5, False, None),
+                                         (7, 2, True, 1000), (4, 300, True, None), (2, 1, False, 1)])
+def test_two_stage_kernel(B, H, with_D, L):
+    """The two-stage tcgen05 kernel (2N = 8192): units of two row pairs with
+    a missing last row (odd B), single-pair units (B = 6: pairs 0-1 and 2),
+    many units per CTA (H = 300), partial kernels, no skip term; every output
+    compared."""
+    wl = wlmod.make_1d(B, H, 4096, dtype="bf16", gated=False, seed=17 * B + H, with_D=with_D, L=L)
+    y, plan = run_1d(wl, kernel="tcgen05")
+    assert plan.path == "fused_t2"
+    assert_close(y, oracle_full(wl), "bf16", f"t2 B={B} H={H} D={with_D} L={L}", scale=row_scale_1d(wl))
+
+
+def test_two_stage_kernel_named_full():
+    """The Hyena-style workload through the two-stage kernel, every output."""
+    wl = _named("hyena_b8_h768_n4096_bf16")
+    y, plan = run_1d(wl, kernel="tcgen05")
+    assert plan.path == "fused_t2"
+    assert_close(y, oracle_full(wl), "bf16", wl.name + " (t2, full)", scale=row_scale_1d(wl))
 
 
 def test_tensor_core_large_dynamic_range():
@@ -129,8 +153,8 @@ def test_no_skip_term_and_single_row():
                                            (32768, "bf16", True), (32768, "bf16", False)])
 def test_multipass_full_compare(N, dtype, gated):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=gated, seed=N + gated, with_D=True)
-    y, path = run_1d(wl)
-    assert path == "multipass"
+    y, plan = run_1d(wl)
+    assert plan.path == "multipass"
     assert_close(y, oracle_full(wl), dtype, f"multipass N={N} {dtype} gated={gated}",
                  gate=wl.v if gated else None, scale=row_scale_1d(wl))
 
@@ -139,19 +163,19 @@ def test_multipass_full_compare(N, dtype, gated):
 def test_multipass_sampled(log2N):
     N = 1 << log2N
     wl = wlmod.make_1d(3, 1, N, dtype="f32", seed=log2N, alpha=1e-5)
-    y, path = run_1d(wl)
-    assert path == "multipass"
+    y, plan = run_1d(wl)
+    assert plan.path == "multipass"
     b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 400, seed=log2N)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
     assert_close(y[b, h, t], ref, "f32", f"multipass N=2^{log2N}", scale=row_scale_1d(wl, b, h))
 
 
-def test_multipass_ragged_groups(monkeypatch):
+def test_multipass_ragged_groups():
     """More pairs than one workspace group holds, with a short last group."""
-    monkeypatch.setenv("FFTCONV_GROUP_MB", "64")  # 4 pairs of 16 MiB per group: groups of 4, 4, 2
     N = 1 << 20
     wl = wlmod.make_1d(3, 5, N, dtype="bf16", seed=99, alpha=1e-5)
-    y, _ = run_1d(wl)
+    y, plan = run_1d(wl, group_bytes=64 << 20)  # 4 pairs of 16 MiB per group: groups of 4, 4, 2
+    assert plan.workspace_bytes == 64 << 20
     b, h, t = wlmod.sample_points_1d(wl.B, wl.H, N, 64, seed=99)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D)
     assert_close(y[b, h, t], ref, "bf16", "ragged groups", scale=row_scale_1d(wl, b, h))
@@ -188,27 +212,84 @@ def _named(name):
 
 def test_pr1_full():
     wl = _named("pr1_b1_h4_n1024_f32")
-    y, path = run_1d(wl)
-    assert path == "fused"
+    y, plan = run_1d(wl)
+    assert plan.path == "fused"
     assert_close(y, oracle_full(wl), "f32", wl.name, scale=row_scale_1d(wl))
 
 
-@pytest.mark.parametrize("name,per_row", [("hyena_b8_h768_n4096_bf16", 12),
-                                          ("gated_b4_h1024_n16384_bf16", 6),
-                                          ("long_b2_h64_n1048576_f32", 96)])
-def test_named_1d_sampled(name, per_row):
-    wl = _named(name)
+def test_named_hyena_full():
+    """The Hyena-style workload at full size in the bench's launch (persistent
+    CTAs, several row pairs each): every one of its 25,165,824 outputs against
+    the oracle."""
+    wl = _named("hyena_b8_h768_n4096_bf16")
     y, _ = run_1d(wl)
-    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, wl.N, per_row, seed=1)
+    assert_close(y, oracle_full(wl), "bf16", wl.name + " (full)", scale=row_scale_1d(wl))
+
+
+def test_named_gated_rows_full():
+    """The gated workload at full size: 512 whole rows (seeded draw of (b, h))
+    against the oracle, plus sampled positions with uniform draws in every row."""
+    wl = _named("gated_b4_h1024_n16384_bf16")
+    y, _ = run_1d(wl)
+    rng = np.random.default_rng(77)
+    rows = rng.choice(wl.B * wl.H, size=512, replace=False)
+    bi, hi = rows // wl.H, rows % wl.H
+    # the chosen rows as one [1, 512, N] workload with their own filters
+    ref = oracle.causal_conv1d(wl.u[bi, hi][None], wl.k[hi], w=wl.w[bi, hi][None], v=wl.v[bi, hi][None])[0]
+    sub = wlmod.Workload1D("rows", 1, 512, wl.N, wl.dtype, True, wl.u[bi, hi][None], wl.k[hi], None,
+                           wl.v[bi, hi][None], wl.w[bi, hi][None])
+    assert_close(y[bi, hi], ref, "bf16", wl.name + " (512 rows)", gate=wl.v[bi, hi],
+                 scale=row_scale_1d(sub)[0])
+    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, wl.N, 8, seed=1)
     ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D, w=wl.w, v=wl.v)
-    assert_close(y[b, h, t], ref, wl.dtype, wl.name, gate=None if wl.v is None else wl.v[b, h, t],
+    assert_close(y[b, h, t], ref, wl.dtype, wl.name + " (sampled)", gate=wl.v[b, h, t],
                  scale=row_scale_1d(wl, b, h))
 
 
-# ------------------------------------------------------------------ 2-D
-def run_2d(wl):
+def test_named_long_sampled():
+    wl = _named("long_b2_h64_n1048576_f32")
+    y, _ = run_1d(wl)
+    b, h, t = wlmod.sample_points_1d(wl.B, wl.H, wl.N, 96, seed=1)
+    ref = oracle.causal_conv1d_points(wl.u, wl.k, b, h, t, D=wl.D, w=wl.w, v=wl.v)
+    assert_close(y[b, h, t], ref, wl.dtype, wl.name, scale=row_scale_1d(wl, b, h))
+
+
+@pytest.mark.parametrize("N,kernel", [(2048, "tcgen05"), (4096, "tcgen05"), (16384, "auto")])  # umma, t2, P = 128
+def test_wait_limit_timeout_then_recovers(N, kernel):
+    """A wait limit of 0 makes the first bounded device wait of every CTA give
+    up: the launch drains its products, frees its tensor memory and reports
+    FFTCONV_ERR_TIMEOUT once; the same plan, back at the default limit, then
+    runs a normal launch that matches the oracle.  Nothing hangs or faults:
+    the products do complete, the wait just stops looking."""
     from fft_long_convolution_causal_b200 import binding
-    plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, wl.dtype)
+    wl = wlmod.make_1d(3, 3, N, dtype="bf16", gated=False, seed=5 * N, with_D=True)
+    plan = binding.Plan(wl.B, wl.H, wl.N, "bf16", kernel=kernel)
+    assert plan.path in ("fused_umma", "fused_t2", "fused_tc"), plan.path
+    khat = plan.kernel_spectrum(torch.from_numpy(wl.k).cuda())
+    u, D = to_dev(wl.u, "bf16"), torch.from_numpy(wl.D).cuda()
+    plan.set_wait_limit(0)
+    plan.fwd(u, khat, D=D)
+    assert plan.device_status() == 6  # FFTCONV_ERR_TIMEOUT, once
+    assert plan.device_status() == 0
+    plan.set_wait_limit()
+    y = plan.fwd(u, khat, D=D)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    assert_close(to_host(y), oracle_full(wl), "bf16", f"after timeout N={N}", scale=row_scale_1d(wl))
+
+
+def test_mma_flops_reported():
+    from fft_long_convolution_causal_b200 import binding
+    assert binding.Plan(2, 2, 1024, "f32").mma_flops == 0.0
+    assert binding.Plan(2, 2, 1 << 16, "f32").mma_flops == 0.0
+    # mma.sync kernel, 2N = 8192 (P = 32): 1536 m16n8k16 products per pair
+    assert binding.Plan(4, 3, 4096, "bf16", kernel="mma_sync").mma_flops == 2 * 3 * 1536 * 2 * 16 * 8 * 16
+
+
+# ------------------------------------------------------------------ 2-D
+def run_2d(wl, **plan_kw):
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, wl.dtype, **plan_kw)
     khat = plan.kernel_spectrum(torch.from_numpy(wl.k).cuda())
     y = plan.fwd(to_dev(wl.u, wl.dtype), khat)
     torch.cuda.synchronize()
@@ -229,11 +310,10 @@ def test_conv2d_small_kernel():
     assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "f32", "2d small kernel", scale=row_scale_2d(wl))
 
 
-def test_conv2d_tensor_core_groups(monkeypatch):
+def test_conv2d_tensor_core_groups():
     """2-D on the tensor cores with several workspace groups (the last one short)."""
-    monkeypatch.setenv("FFTCONV_GROUP_MB", "4")  # 4 pairs of 1 MiB per group: groups of 4, 2 (6 pairs)
     wl = wlmod.make_2d(4, 3, 256, 256, dtype="bf16", seed=31, Kh=12, Kw=20, sigma=64.0)
-    y = run_2d(wl)
+    y = run_2d(wl, group_bytes=4 << 20)  # 4 pairs of 1 MiB per group: groups of 4, 2 (6 pairs)
     idx = wlmod.sample_points_2d(wl.B, wl.C, wl.Hs, wl.Ws, 2048, seed=31)
     ref = oracle.causal_conv2d_points(wl.u, wl.k, *idx)
     assert_close(y[idx], ref, "bf16", "2d tc groups", scale=row_scale_2d(wl, idx[0], idx[1]))

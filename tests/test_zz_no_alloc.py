@@ -6,7 +6,10 @@ this entry point; its scratch is a fixed device array inside the library.  It
 must give the same result as fftconv_fwd with a caller workspace.  The test
 calls it twice in a row on different inputs (the array keeps the previous
 call's contents, which must not leak into the next result) and compares each
-call with fftconv_fwd on the same input, within the parity tolerance.
+call with fftconv_fwd on the same input, within the parity tolerance, and the
+first call also with the fp64 oracle on sampled outputs.  One case has more
+row pairs than the static array holds at once and a short last group (10
+pairs of 2 MiB in groups of 8), a split that only this entry point makes.
 
 The file is named to be collected last, and it needs nothing from the other
 tests, so it passes alone in a fresh process as well as after them.
@@ -17,6 +20,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from fft_long_convolution_causal_b200 import workloads as wlmod
 from parity import assert_close, row_scale_1d, to_dev, to_host
 
@@ -35,11 +39,10 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("N,dtype,gated", [(1 << 16, "f32", False), (1 << 15, "bf16", True),
-                                           (1 << 20, "f32", False)])
-def test_static_workspace_matches_fftconv_fwd(lib, N, dtype, gated):
+@pytest.mark.parametrize("N,dtype,gated,B,H", [(1 << 16, "f32", False, 3, 2), (1 << 15, "bf16", True, 3, 2),
+                                               (1 << 20, "f32", False, 3, 2), (1 << 17, "f32", False, 3, 5)])
+def test_static_workspace_matches_fftconv_fwd(lib, N, dtype, gated, B, H):
     from fft_long_convolution_causal_b200 import binding
-    B, H = 3, 2
     plan = binding.Plan(B, H, N, dtype, gated=gated)
     assert plan.path == "multipass"
     first = wlmod.make_1d(B, H, N, dtype=dtype, gated=gated, seed=N, alpha=1e-4)
@@ -59,6 +62,11 @@ def test_static_workspace_matches_fftconv_fwd(lib, N, dtype, gated):
         assert np.all(np.isfinite(a)), f"call {call}: unwritten outputs"
         assert_close(a, b, dtype, f"static workspace call {call} N={N} {dtype}",
                      gate=wl.v if gated else None, scale=row_scale_1d(wl))
+        if call == 0:
+            bi, hi, ti = wlmod.sample_points_1d(B, H, N, 48, seed=N)
+            ref = oracle.causal_conv1d_points(wl.u, wl.k, bi, hi, ti, D=wl.D, w=wl.w, v=wl.v)
+            assert_close(a[bi, hi, ti], ref, dtype, f"static workspace vs oracle N={N} {dtype}",
+                         gate=wl.v[bi, hi, ti] if gated else None, scale=row_scale_1d(wl, bi, hi))
 
 
 def test_static_workspace_rejects_non_multipass_plans(lib):
