@@ -10,6 +10,8 @@ Definitions (see fftconv_oracle.c for the page citations):
   x = u (ungated) or u*w (gated, then y *= v).  This is
   irfft(rfft(x,2N) * rfft(k,2N))[:N] (+ D x) evaluated as the direct sum.
 * ``causal_conv1d_dynamic``: the same with one filter per batch row, k [B,H,L].
+* ``ssm_kernel``: filters of a diagonal state-space model, k = Re(sum c lam^t);
+  the convolution itself is causal_conv1d (or _points) with that k.
 * ``causal_conv1d_bwd``: the gradients du (dv, dw), dk, dD of that y for an
   upstream gradient dy, by the chain rule written as direct sums.
 * ``causal_conv2d``: y[b,c,i,j] = sum_{p<=i,q<=j} k[c,p,q] u[b,c,i-p,j-q].
@@ -36,6 +38,7 @@ def bind(path):
     lib.oracle_causal_conv1d_points.argtypes = [_i64] * 4 + [_f64p] * 5 + [_i64] + [_i64p] * 3 + [_f64p]
     lib.oracle_causal_conv1d_bwd.argtypes = [_i64] * 4 + [_f64p] * 11
     lib.oracle_causal_conv1d_dynamic.argtypes = [_i64] * 4 + [_f64p] * 6
+    lib.oracle_ssm_kernel.argtypes = [_i64] * 3 + [_f64p] * 5
     lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
     lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
     lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
@@ -127,6 +130,20 @@ def causal_conv1d_dynamic(u, k, D=None, w=None, v=None) -> np.ndarray:
     return y
 
 
+def ssm_kernel(lam, c, L) -> np.ndarray:
+    """fp64 filters of a diagonal state-space model: k[h,t] = Re(sum_j c[h,j]
+    lam[h,j]^t) for t < L; lam, c complex [H, d].  Returns [H, L]."""
+    lam = np.ascontiguousarray(np.asarray(lam, dtype=np.complex128))
+    c = np.ascontiguousarray(np.asarray(c, dtype=np.complex128))
+    if lam.ndim != 2 or lam.shape != c.shape:
+        raise ValueError("lam and c must be [H, d]")
+    H, d = lam.shape
+    parts = [np.ascontiguousarray(a) for a in (lam.real, lam.imag, c.real, c.imag)]
+    k = np.empty((H, int(L)))
+    _load().oracle_ssm_kernel(H, d, int(L), *[_p(a) for a in parts], _p(k))
+    return k
+
+
 def causal_conv1d_bwd(u, k, dy, D=None, w=None, v=None) -> dict:
     """fp64 gradients of y = causal_conv1d(u, k, D, w, v) for the upstream
     gradient dy [B,H,N]: du (and dv, dw when gated) [B,H,N], dk [H,L],
@@ -208,5 +225,5 @@ def dft_causal_conv2d(x, k) -> np.ndarray:
     return y
 
 
-__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "causal_conv2d", "causal_conv2d_points",
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "ssm_kernel", "causal_conv2d", "causal_conv2d_points",
            "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

@@ -223,6 +223,34 @@ void oracle_causal_conv1d_dynamic(int64_t B, int64_t H, int64_t N, int64_t L,
     }
 }
 
+/*
+ * Filters of a diagonal state-space model, the setting of "FlashConv"
+ * (Mechanism: state-space sequence convolutions, with the state passed
+ * between chunks past the on-chip length): each channel's filter is
+ *   k[h][t] = Re( sum_j c[h][j] lam[h][j]^t ),  t < L,
+ * with complex lam (|lam| < 1) and c (the input and output maps folded into
+ * c).  lam^t = |lam|^t (cos t.arg(lam) + i sin t.arg(lam)), in fp64.
+ * lam, c: [H][d] as separate real / imaginary arrays; k: [H][L].
+ */
+void oracle_ssm_kernel(int64_t H, int64_t d, int64_t L, const double* lam_re, const double* lam_im,
+                       const double* c_re, const double* c_im, double* k)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t h = 0; h < H; ++h) {
+        for (int64_t t = 0; t < L; ++t) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < d; ++j) {
+                double lr = lam_re[h * d + j], li = lam_im[h * d + j];
+                double mag = pow(sqrt(lr * lr + li * li), (double)t);
+                double ang = (double)t * atan2(li, lr);
+                double pr = mag * cos(ang), pi = mag * sin(ang);
+                acc += c_re[h * d + j] * pr - c_im[h * d + j] * pi;
+            }
+            k[h * L + t] = acc;
+        }
+    }
+}
+
 /* One output of the 2-D causal convolution of image (b,c) at (i,j). */
 static double conv2d_point(int64_t Ws, int64_t Kh, int64_t Kw, const double* ui,
                            const double* kc, int64_t i, int64_t j)

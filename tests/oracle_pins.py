@@ -345,10 +345,42 @@ def check_dynamic_kernels():
     assert changed[1, 0] and changed.sum() == 1
 
 
+def check_ssm_kernel():
+    """State-space filters: numpy's complex power (the library routine); the
+    conjugate-pair closed form 2 |c| |lam|^t cos(t arg lam + arg c); and the
+    state-space recursion itself -- s_j[t] = lam_j s_j[t-1] + x[t],
+    y[t] = Re(sum_j c_j s_j[t]) + D x[t], run in fp64 -- equal to the causal
+    convolution oracle with the materialised filter (the state-space view a
+    chunked computation passes between chunks)."""
+    r = _rng(65)
+    H, d, L = 2, 4, 300
+    lam = (r.uniform(0.9, 0.999, (H, d)) * np.exp(1j * r.uniform(-1.0, 1.0, (H, d))))
+    c = r.standard_normal((H, d)) + 1j * r.standard_normal((H, d))
+    k = oracle.ssm_kernel(lam, c, L)
+    t = np.arange(L)
+    want = np.real(np.sum(c[:, :, None] * lam[:, :, None] ** t[None, None, :], axis=1))
+    assert np.allclose(k, want, rtol=1e-11, atol=1e-11)
+    lam1 = np.array([[0.97 * np.exp(0.3j), 0.97 * np.exp(-0.3j)]])
+    c1 = np.array([[0.5 - 0.25j, 0.5 + 0.25j]])
+    want1 = 2 * abs(c1[0, 0]) * 0.97 ** t * np.cos(0.3 * t + np.angle(c1[0, 0]))
+    assert np.allclose(oracle.ssm_kernel(lam1, c1, L)[0], want1, rtol=1e-11, atol=1e-12)
+    B, N = 2, 300
+    x = r.standard_normal((B, H, N))
+    D = r.standard_normal(H)
+    y = oracle.causal_conv1d(x, k, D=D)
+    s = np.zeros((B, H, d), dtype=np.complex128)
+    rec = np.empty((B, H, N))
+    for tt in range(N):
+        s = lam[None] * s + x[:, :, tt:tt + 1]
+        rec[:, :, tt] = np.real(np.sum(c[None] * s, axis=2)) + D[None] * x[:, :, tt]
+    assert np.allclose(y, rec, rtol=1e-9, atol=1e-9)
+
+
 ALL_CHECKS = [
     check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
     check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
     check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
+    check_ssm_kernel,
 ]

@@ -51,6 +51,10 @@ MUTANTS = {
                                "        for (int64_t t = 0; t < N; ++t)\n            y[r * N + t] = conv1d_point",
                                "        const double* kr = k + h * L;\n        const double* Dh = D ? D + h : NULL;\n"
                                "        for (int64_t t = 0; t < N; ++t)\n            y[r * N + t] = conv1d_point"),
+    "ssm_power_sign": ("double ang = (double)t * atan2(li, lr);", "double ang = -(double)t * atan2(li, lr);"),
+    "ssm_drop_imag_part": ("acc += c_re[h * d + j] * pr - c_im[h * d + j] * pi;", "acc += c_re[h * d + j] * pr;"),
+    "ssm_power_off_by_one": ("double mag = pow(sqrt(lr * lr + li * li), (double)t);",
+                             "double mag = pow(sqrt(lr * lr + li * li), (double)(t + 1));"),
 }
 
 
