@@ -10,6 +10,8 @@ Definitions (see fftconv_oracle.c for the page citations):
   x = u (ungated) or u*w (gated, then y *= v).  This is
   irfft(rfft(x,2N) * rfft(k,2N))[:N] (+ D x) evaluated as the direct sum.
 * ``causal_conv1d_dynamic``: the same with one filter per batch row, k [B,H,L].
+* ``freq_sparse_conv1d``: the formula with the filter's spectrum zeroed on
+  blocks of frequencies (numpy FFT as the library step).
 * ``ssm_kernel``: filters of a diagonal state-space model, k = Re(sum c lam^t);
   the convolution itself is causal_conv1d (or _points) with that k.
 * ``causal_conv1d_bwd``: the gradients du (dv, dw), dk, dD of that y for an
@@ -144,6 +146,29 @@ def ssm_kernel(lam, c, L) -> np.ndarray:
     return k
 
 
+def freq_sparse_conv1d(u, k, keep, D=None) -> np.ndarray:
+    """Frequency-sparse causal convolution ("FlashFFTConv", abstract): the
+    defining formula with the filter's spectrum (skip term included) zeroed on
+    blocks of frequencies,
+        y = Re(iDFT_M(DFT_M(pad u) . (DFT_M(pad k) + D) . m))[:N],  M = 2N,
+    m[f] = keep[f mod G] for a block mask keep of G entries (f = k1 + G k2:
+    the outer frequency digit k1 of the split M = G x (M / G)).  numpy's FFT is
+    the library step; fp64.  u [B,H,N], k [H,L], keep [G] bool."""
+    u = np.asarray(u, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    keep = np.asarray(keep, dtype=bool)
+    B, H, N = u.shape
+    M = 2 * N
+    if M % keep.size:
+        raise ValueError("the mask length must divide 2N")
+    m = keep[np.arange(M) % keep.size].astype(np.float64)
+    K = np.fft.fft(k, M, axis=-1)
+    if D is not None:
+        K = K + np.asarray(D, dtype=np.float64)[:, None]
+    Y = np.fft.fft(u, M, axis=-1) * (K * m)[None]
+    return np.real(np.fft.ifft(Y, axis=-1))[..., :N]
+
+
 def causal_conv1d_bwd(u, k, dy, D=None, w=None, v=None) -> dict:
     """fp64 gradients of y = causal_conv1d(u, k, D, w, v) for the upstream
     gradient dy [B,H,N]: du (and dv, dw when gated) [B,H,N], dk [H,L],
@@ -225,5 +250,5 @@ def dft_causal_conv2d(x, k) -> np.ndarray:
     return y
 
 
-__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "ssm_kernel", "causal_conv2d", "causal_conv2d_points",
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "ssm_kernel", "freq_sparse_conv1d", "causal_conv2d", "causal_conv2d_points",
            "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

@@ -376,11 +376,41 @@ def check_ssm_kernel():
     assert np.allclose(y, rec, rtol=1e-9, atol=1e-9)
 
 
+def check_freq_sparse():
+    """Frequency-sparse form: an all-true mask gives the direct sum; a masked
+    case equals the same formula written with explicit O(M^2) DFT matrices
+    (no FFT library); a Hermitian-symmetric mask keeps the result real and
+    linear in u."""
+    r = _rng(66)
+    B, H, N, L = 2, 2, 32, 20
+    u = r.standard_normal((B, H, N))
+    k = r.standard_normal((H, L))
+    D = r.standard_normal(H)
+    G = 8
+    full = oracle.freq_sparse_conv1d(u, k, np.ones(G, bool), D=D)
+    assert np.allclose(full, oracle.causal_conv1d(u, k, D=D), rtol=1e-11, atol=1e-11)
+    keep = np.array([1, 0, 1, 1, 0, 1, 1, 0], bool)  # keep[j] == keep[(G - j) % G]
+    assert all(keep[j] == keep[(G - j) % G] for j in range(G))
+    y = oracle.freq_sparse_conv1d(u, k, keep, D=D)
+    M = 2 * N
+    f = np.arange(M)
+    F = np.exp(-2j * np.pi * np.outer(f, f) / M)            # explicit DFT matrix
+    up = np.zeros((B, H, M)); up[..., :N] = u
+    kp = np.zeros((H, M)); kp[:, :L] = k
+    Kf = (F @ kp.T).T + D[:, None]
+    Yf = np.einsum("fm,bhm->bhf", F, up) * (Kf * keep[f % G])[None]
+    want = np.einsum("nf,bhf->bhn", np.conj(F), Yf)[..., :N] / M
+    assert np.allclose(want.imag, 0, atol=1e-9)
+    assert np.allclose(y, want.real, rtol=1e-10, atol=1e-10)
+    y2 = oracle.freq_sparse_conv1d(2.0 * u, k, keep, D=D)
+    assert np.allclose(y2, 2.0 * y, rtol=1e-12, atol=1e-12)
+
+
 ALL_CHECKS = [
     check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
     check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
     check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
-    check_ssm_kernel,
+    check_ssm_kernel, check_freq_sparse,
 ]
