@@ -43,6 +43,13 @@ _SIGS = {
     "fftconv_plan_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint32]),
     "fftconv_spectrum_conjugate": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
     "fftconv_fwd_dynamic": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp]),
+    "fftconv_ssm_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int64]),
+    "fftconv_ssm_spectrum": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv_spectrum_blocks": (ctypes.c_int, [_vp]),
+    "fftconv_spectrum_sparsify": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp]),
+    "fftconv_partial_plan_create": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int64]),
     "fftconv_bwd_workspace_bytes": (ctypes.c_size_t, [_vp]),
     "fftconv_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]),
@@ -264,6 +271,22 @@ class Plan(_PlanBase):
                                             _ptr(y), _stream(stream)), "fftconv_fwd_dynamic")
         return y
 
+    @property
+    def spectrum_blocks(self) -> int:
+        """Outer frequency blocks a frequency-sparse mask has (0: not a multi-pass plan)."""
+        return int(self.lib.fftconv_spectrum_blocks(self._handle))
+
+    def sparsify(self, khat: torch.Tensor, keep, stream=None):
+        """Frequency-sparse: zero khat on the outer frequency rows k1 with keep[k1] false (None: dense)."""
+        if keep is None:
+            _check(self.lib.fftconv_spectrum_sparsify(self._handle, _ptr(khat), None, 0, _stream(stream)),
+                   "fftconv_spectrum_sparsify")
+            return khat
+        arr = (ctypes.c_uint8 * len(keep))(*[1 if x else 0 for x in keep])
+        _check(self.lib.fftconv_spectrum_sparsify(self._handle, _ptr(khat), ctypes.cast(arr, ctypes.c_void_p),
+                                                  len(keep), _stream(stream)), "fftconv_spectrum_sparsify")
+        return khat
+
     def spectrum_conjugate(self, khat: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """conj(khat) in the plan's layout: the spectrum of the correlation with k."""
         if out is None:
@@ -339,6 +362,66 @@ class Plan2D(_PlanBase):
         workspace = self._ws(workspace)
         _check(self.lib.fftconv2d_fwd(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace),
                                       _stream(stream)), "fftconv2d_fwd")
+        return y
+
+
+class PartialPlan(Plan):
+    """Partial convolution, filters of at most L_max taps:
+    fftconv_partial_plan_create(B, H, N, dtype, gated, L_max); kernel_spectrum
+    and fwd as a 1-D plan."""
+
+    def __init__(self, B: int, H: int, N: int, dtype: str = "f32", gated: bool = False, L_max: int = 1024):
+        self.lib = load_library()
+        self.B, self.H, self.N, self.dtype, self.gated = B, H, N, dtype, bool(gated)
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv_partial_plan_create(ctypes.byref(h), B, H, N, DTYPES[dtype], int(bool(gated)),
+                                                    int(L_max)), "fftconv_partial_plan_create")
+        self._handle = h
+        self._workspace = None
+
+
+class SSMPlan(_PlanBase):
+    """Chunked state passing: fftconv_ssm_plan_create(B, H, N, dtype, d_state, chunk)."""
+
+    def __init__(self, B: int, H: int, N: int, dtype: str = "f32", d_state: int = 16, chunk: int = 8192):
+        self.lib = load_library()
+        self.B, self.H, self.N, self.dtype, self.d, self.chunk = B, H, N, dtype, d_state, chunk
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv_ssm_plan_create(ctypes.byref(h), B, H, N, DTYPES[dtype], d_state, chunk),
+               "fftconv_ssm_plan_create")
+        self._handle = h
+        self._workspace = None
+
+    def set_filters(self, lam: torch.Tensor, c: torch.Tensor, khat: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+        """k[h,t] = Re(sum_j c[h,j] lam[h,j]^t); lam, c complex [H, d] (any device)."""
+        shape = (self.H, self.d)
+        if tuple(lam.shape) != shape or tuple(c.shape) != shape:
+            raise ValueError(f"lam and c must be {shape}")
+        parts = [t.real.to(torch.float32).contiguous().cuda() for t in (lam, c)] + \
+                [t.imag.to(torch.float32).contiguous().cuda() for t in (lam, c)]
+        lr, cr, li, ci = parts
+        if khat is None:
+            khat = self.new_spectrum()
+        ws = self._ws(None)
+        _check(self.lib.fftconv_ssm_spectrum(self._handle, _ptr(lr), _ptr(li), _ptr(cr), _ptr(ci), _ptr(khat),
+                                             _ptr(ws), _stream(stream)), "fftconv_ssm_spectrum")
+        self._keep = parts  # alive until the launch has read them
+        return khat
+
+    def fwd(self, u: torch.Tensor, khat: torch.Tensor, D: Optional[torch.Tensor] = None,
+            y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        shape = (self.B, self.H, self.N)
+        _need(u, "u", shape, self.torch_dtype)
+        if D is not None:
+            _need(D, "D", (self.H,), torch.float32)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        ws = self._ws(None)
+        _check(self.lib.fftconv_fwd(self._handle, _ptr(u), None, None, _ptr(khat), _ptr(D), _ptr(y), _ptr(ws),
+                                    _stream(stream)), "fftconv_fwd")
         return y
 
 

@@ -71,7 +71,7 @@ template <int LOG2M, typename IO, bool GATED>
 __global__ void __launch_bounds__(FusedG<LOG2M>::T)
 fused_fwd_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __restrict__ w,
                const float2* __restrict__ khat, const float* __restrict__ D, IO* __restrict__ y,
-               const float2* __restrict__ tw, int B, int H) {
+               const float2* __restrict__ tw, int B, int H, int kdiv) {
     using G = FusedG<LOG2M>;
     using Lay = typename G::Lay;
     constexpr int M = G::L, N = M / 2, NS = G::Plan::kStages;
@@ -92,9 +92,12 @@ fused_fwd_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __r
     __syncthreads();
     smem_stages<G, 1, NS, false>(smem, tid, tw);
 
-    // pointwise product with (Khat + D/M), fused into the first inverse stage
-    const float dm = D ? D[h] * (1.0f / M) : 0.f;
-    const float2* __restrict__ kh = khat + (size_t)h * M;
+    // pointwise product with (Khat + D/M), fused into the first inverse stage;
+    // kdiv consecutive row channels share one spectrum and skip weight (the
+    // chunks of one channel in the chunked state-passing path; 1 otherwise)
+    const int hk = h / kdiv;
+    const float dm = D ? D[hk] * (1.0f / M) : 0.f;
+    const float2* __restrict__ kh = khat + (size_t)hk * M;
     stage<G, 0, true, R0, R0, true>(
         tid, tw,
         [&](int i, int) {
@@ -290,6 +293,62 @@ fused_dyn_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __r
         [&](int n, int, float2 z) { store_pair<IO, GATED>(y, v, row0, row1, has1, n, z); });
 }
 
+// Partial convolutions ("FlashFFTConv", abstract: partial convolutions, a
+// filter shorter than the sequence, computed by skipping blocks of the
+// decomposition): for L <= T the row is cut into chunks of T and chunk c is
+// computed by overlap-save on a transform of 2T = M points over the window
+// x[cT - T, cT + T) (zeros before the row start).  The circular convolution
+// with the zero-padded k[:L] wraps only into outputs n < L - 1 of the window,
+// so its upper half n in [T, 2T) is exactly y[cT, cT + T): the cost is
+// O(N log T) on chip instead of O(N log N) through memory.  One CTA per (pair
+// of batch rows, channel x chunk); every chunk of a channel shares its
+// spectrum.
+template <int LOG2M, typename IO, bool GATED>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+fused_part_simt(const IO* __restrict__ u, const IO* __restrict__ v, const IO* __restrict__ w,
+                const float2* __restrict__ khat, const float* __restrict__ D, IO* __restrict__ y,
+                const float2* __restrict__ tw, int B, int H, int nc) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, T = M / 2, NS = G::Plan::kStages;
+    static_assert(NS >= 2, "transform too short");
+    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, h = blockIdx.y / nc, c = blockIdx.y % nc;
+    const int b0 = 2 * blockIdx.x;
+    const bool has1 = b0 + 1 < B;
+    const size_t NR = (size_t)nc * T;  // row length
+    const size_t row0 = ((size_t)b0 * H + h) * NR;
+    const size_t row1 = ((size_t)(b0 + 1) * H + h) * NR;
+    const int64_t start = (int64_t)c * T - T;
+    auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    stage<G, 0, false, R0, R0, false>(
+        tid, tw,
+        [&](int n, int) {
+            const int64_t pos = start + n;
+            return pos < 0 ? make_float2(0.f, 0.f) : load_pair<IO, GATED>(u, w, row0, row1, has1, (size_t)pos);
+        },
+        sts);
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(smem, tid, tw);
+    const float dm = D ? D[h] * (1.0f / M) : 0.f;
+    const float2* __restrict__ kh = khat + (size_t)h * M;
+    stage<G, 0, true, R0, R0, true>(
+        tid, tw,
+        [&](int i, int) {
+            float2 kk = __ldg(&kh[i]);
+            kk.x += dm;
+            return cmul(smem[Lay::at(i, 0)], kk);
+        },
+        sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, true>(smem, tid, tw);
+    stage<G, NS - 1, true, RL, RL, false>(tid, tw, lds, [&](int n, int, float2 z) {
+        if (n >= T) store_pair<IO, GATED>(y, v, row0, row1, has1, (size_t)(start + n), z);
+    });
+}
+
 template <int LOG2M>
 static size_t fused_smem() { return FusedG<LOG2M>::Lay::kWords * sizeof(float2); }
 
@@ -306,7 +365,7 @@ static cudaError_t fused_fwd_go(const fftconv_plan_s& p, const void* u, const vo
     ensure_smem(kern, smem);
     dim3 grid((p.B + 1) / 2, p.H);
     kern<<<grid, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)v, (const IO*)w, khat, D, (IO*)y,
-                                               p.tw.wL, p.B, p.H);
+                                               p.tw.wL, p.B, p.H, p.kdiv);
     return cudaGetLastError();
 }
 
@@ -378,6 +437,24 @@ static cudaError_t kgrad_dt(const fftconv_plan_s& p, const void* u, const void* 
 
 bool kgrad_supported(int log2M) { return log2M >= 7 && log2M <= 14; }
 
+// frequency-sparse plans: zero the spectrum rows k1 (all k2) the mask drops;
+// the multi-pass spectrum is [H][k1 N1][k2 N2]
+__global__ void zero_spectrum_rows(float2* __restrict__ khat, const uint8_t* __restrict__ keep, int N1, int N2,
+                                   size_t total) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const int k1 = (int)((i / N2) % N1);
+        if (!keep[k1]) khat[i] = make_float2(0.f, 0.f);
+    }
+}
+
+cudaError_t launch_zero_spectrum_rows(const fftconv_plan_s& p, void* khat, cudaStream_t s) {
+    const size_t total = (size_t)p.H << p.log2M;
+    const size_t blocks = (total + 255) / 256;
+    zero_spectrum_rows<<<(unsigned)(blocks < 8192 ? blocks : 8192), 256, 0, s>>>(
+        (float2*)khat, p.d_keep, 1 << p.log2N1, 1 << p.log2N2, total);
+    return cudaGetLastError();
+}
+
 template <int LOG2M, typename IO, bool GATED>
 static cudaError_t dyn_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
                           int L, const float* D, void* y, cudaStream_t s) {
@@ -401,6 +478,38 @@ static cudaError_t dyn_dt(const fftconv_plan_s& p, const void* u, const void* v,
 }
 
 bool dyn_supported(int log2M) { return log2M >= 7 && log2M <= 13; }
+
+template <int LOG2M, typename IO, bool GATED>
+static cudaError_t part_go(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float2* khat,
+                           const float* D, void* y, cudaStream_t s) {
+    auto kern = fused_part_simt<LOG2M, IO, GATED>;
+    const size_t smem = fused_smem<LOG2M>();
+    ensure_smem(kern, smem);
+    dim3 grid((p.B + 1) / 2, (unsigned)(p.H * p.nchunks));
+    kern<<<grid, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)v, (const IO*)w, khat, D, (IO*)y,
+                                               p.chunk->tw.wL, p.B, p.H, (int)p.nchunks);
+    return cudaGetLastError();
+}
+
+template <int LOG2M>
+static cudaError_t part_dt(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float2* khat,
+                           const float* D, void* y, cudaStream_t s) {
+    if (p.dtype == FFTCONV_BF16)
+        return p.gated ? part_go<LOG2M, __nv_bfloat16, true>(p, u, v, w, khat, D, y, s)
+                       : part_go<LOG2M, __nv_bfloat16, false>(p, u, v, w, khat, D, y, s);
+    return p.gated ? part_go<LOG2M, float, true>(p, u, v, w, khat, D, y, s)
+                   : part_go<LOG2M, float, false>(p, u, v, w, khat, D, y, s);
+}
+
+cudaError_t launch_partial_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                               const float2* khat, const float* D, void* y, cudaStream_t s) {
+    switch (p.chunk->log2M) {
+#define FFTC_P(X) case X: return part_dt<X>(p, u, v, w, khat, D, y, s);
+        FFTC_P(7) FFTC_P(8) FFTC_P(9) FFTC_P(10) FFTC_P(11) FFTC_P(12) FFTC_P(13) FFTC_P(14)
+#undef FFTC_P
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_dyn_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
                            int64_t L, const float* D, void* y, cudaStream_t s) {
@@ -483,7 +592,7 @@ template <int LOG2N1, int LOG2N2, typename IO, bool GATED, int MODE>
 __global__ void __launch_bounds__(ColG<LOG2N1>::T)
 mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __restrict__ k, int L,
          float2* __restrict__ work, const float2* __restrict__ twC, const float2* __restrict__ lo,
-         const float2* __restrict__ hi, int log2S, int B, int H, int64_t first) {
+         const float2* __restrict__ hi, int log2S, int B, int H, int64_t first, const uint8_t* __restrict__ keep) {
     using G = ColG<LOG2N1>;
     using Lay = typename G::Lay;
     constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2, LOG2M = LOG2N1 + LOG2N2;
@@ -526,7 +635,8 @@ mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __rest
         const uint32_t n2 = (uint32_t)(n2_0 + c);
         if (r == 0) step = twiddle_M(lo, hi, n2 * (uint32_t)(N1 / RL), LOG2M, log2S);
         tw = (r % kTwRun == 0) ? twiddle_M(lo, hi, n2 * (uint32_t)k1, LOG2M, log2S) : cmul(tw, step);
-        out[(size_t)k1 * N2 + n2] = cmul(z, tw);
+        // frequency-sparse plans: rows k1 whose spectrum is zeroed are never read again
+        if (!keep || keep[k1]) out[(size_t)k1 * N2 + n2] = cmul(z, tw);
     });
 }
 
@@ -537,7 +647,7 @@ template <int LOG2N1, int LOG2N2, int MODE>
 __global__ void __launch_bounds__(RowG<LOG2N2>::T, RowG<LOG2N2>::T <= 256 ? 3 : 1)
 mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __restrict__ khat_out,
          const float* __restrict__ D, const float2* __restrict__ twR, const float2* __restrict__ lo,
-         const float2* __restrict__ hi, int log2S, int H, int64_t first) {
+         const float2* __restrict__ hi, int log2S, int H, int64_t first, const uint8_t* __restrict__ keep) {
     using G = RowG<LOG2N2>;
     using Lay = typename G::Lay;
     constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2, LOG2M = LOG2N1 + LOG2N2;
@@ -548,6 +658,13 @@ mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __r
     constexpr int RC = G::C;                    // rows k1 of this CTA: k1_0 .. k1_0 + RC - 1
     const int k1_0 = blockIdx.x * RC;
     const int64_t P = first + blockIdx.y;
+    if (MODE == 0 && keep) {
+        // frequency-sparse plans: a CTA whose rows all have a zeroed spectrum has no work
+        bool any = false;
+#pragma unroll
+        for (int c = 0; c < RC; ++c) any |= keep[k1_0 + c] != 0;
+        if (!any) return;
+    }
     float2* __restrict__ rows = work + ((size_t)blockIdx.y * N1 + k1_0) * N2;
     auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
     auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
@@ -588,7 +705,7 @@ mp_pass2(float2* __restrict__ work, const float2* __restrict__ khat, float2* __r
 template <int LOG2N1, int LOG2N2, typename IO, bool GATED>
 __global__ void __launch_bounds__(ColG<LOG2N1>::T)
 mp_pass3(const float2* __restrict__ work, const IO* __restrict__ v, IO* __restrict__ y,
-         const float2* __restrict__ twC, int B, int H, int64_t first) {
+         const float2* __restrict__ twC, int B, int H, int64_t first, const uint8_t* __restrict__ keep) {
     using G = ColG<LOG2N1>;
     using Lay = typename G::Lay;
     constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2;
@@ -602,7 +719,11 @@ mp_pass3(const float2* __restrict__ work, const IO* __restrict__ v, IO* __restri
     auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
     auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
     stage<G, 0, true, R0, R0, false>(
-        tid, twC, [&](int k1, int c) { return in[(size_t)k1 * N2 + n2_0 + c]; }, sts);
+        tid, twC,
+        [&](int k1, int c) {
+            return (!keep || keep[k1]) ? in[(size_t)k1 * N2 + n2_0 + c] : make_float2(0.f, 0.f);
+        },
+        sts);
     __syncthreads();
     smem_stages<G, 1, NS - 1, true>(smem, tid, twC);
     const int h = (int)(P % H);
@@ -630,11 +751,11 @@ static cudaError_t mp_fwd_go(const fftconv_plan_s& p, const void* u, const void*
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
         k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
                                                                p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S, p.B,
-                                                               p.H, first);
+                                                               p.H, first, p.d_keep);
         k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
-                                                    p.log2S, p.H, first);
+                                                    p.log2S, p.H, first, p.d_keep);
         k3<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
-                                                               p.H, first);
+                                                               p.H, first, p.d_keep);
     }
     return cudaGetLastError();
 }
@@ -662,9 +783,10 @@ static cudaError_t mp_spec_go(const fftconv_plan_s& p, const float* k, int64_t L
     for (int64_t first = 0; first < p.H; first += p.group) {
         const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
         k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>(nullptr, nullptr, k, (int)L, work, p.tw.wC,
-                                                               p.tw.wLo, p.tw.wHi, p.log2S, p.B, p.H, first);
+                                                               p.tw.wLo, p.tw.wHi, p.log2S, p.B, p.H, first,
+                                                               nullptr);
         k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, nullptr, khat, nullptr, p.tw.wL, p.tw.wLo, p.tw.wHi,
-                                                    p.log2S, p.H, first);
+                                                    p.log2S, p.H, first, nullptr);
     }
     return cudaGetLastError();
 }

@@ -32,15 +32,16 @@
 // bf16 pairs and writes the next stage's A operand back into the same lane:
 // no transposes and no shared-memory round trip between A, B and C.
 //
-// Roles (320 threads, one CTA per SM, all 512 TMEM columns):
-//   warps 0-7  epilogues (warp e: TMEM lanes 32 (e % 4) .., column half e / 4)
-//   warp 8     issues every MMA (one lane) and commits to mbarriers
-//   warp 9     stages the input rows with cp.async
-// A unit is two row pairs of one channel (slot 0 and slot 1, 256 TMEM
-// columns each); while the epilogue warps work on one slot the tensor core
-// runs the other slot's product.  Every wait is bounded; a wait that gives
-// up stops the CTA, the issuer drains its products before TMEM is freed, and
-// the plan's status word is set.
+// Roles (384 threads, one CTA per SM, all 512 TMEM columns): two
+// independent pipelines ("slots", 256 TMEM columns and their own shared
+// memory each), every slot with
+//   4 epilogue warps (warp e: TMEM lanes 32 (e % 4) .., both column halves),
+//   1 warp that issues its MMAs (one lane) and commits to its mbarriers,
+//   1 warp that stages its input rows with cp.async,
+// working through its own sequence of row pairs, so while one slot's warps
+// run an epilogue the tensor core runs the other slot's product.  Every wait
+// is bounded; a wait that gives up stops the CTA, each issuer drains its
+// products before TMEM is freed, and the plan's status word is set.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -61,19 +62,21 @@ constexpr int kP = 128, kQ = 64, kM = 8192, kN = 4096;
 constexpr uint32_t kOffGP = 0;            // outer DFT matrix, [m 128][k 256] K-major core matrices, 64 KiB
 constexpr uint32_t kOffFQ = 65536;        // inner DFT matrix, [n 128][k 128] K-major, 32 KiB
 constexpr uint32_t kOffX = 98304;         // input planes of slot s at + 16 KiB s: [p 64][n 128] MN-major
-constexpr uint32_t kOffV = 131072;        // stage-D operand of the unit, [k 256][n 128] MN-major, 64 KiB
+constexpr uint32_t kOffV = 131072;        // stage-D operand of slot s at + 32 KiB s: [k 256][n 64] MN-major
 constexpr uint32_t kSmemBytes = 196608;
 
 // core-matrix strides of each operand (bytes)
 constexpr uint32_t kGPm = 4096, kGPk = 128;   // GP: row group (8 m) / column group (8 k)
 constexpr uint32_t kFQn = 2048, kFQk = 128;   // FQ: 8 n / 8 k
 constexpr uint32_t kXp = 2048, kXn = 128;     // X: 8 p / 8 n
-constexpr uint32_t kVk = 2048, kVn = 128;     // V: 8 k / 8 n
+constexpr uint32_t kVk = 1024, kVn = 128;     // V: 8 k / 8 n
 
-constexpr int kEpiWarps = 8, kIssuer = 8, kLoader = 9, kThreads = 320;
+// roles: warps 4 s .. 4 s + 3 epilogues of slot s, warp 8 + s its MMA issuer,
+// warp 10 + s its loader
+constexpr int kGroupWarps = 4, kThreads = 384;
 
-struct Bars {
-    uint64_t xfull[2], xempty[2], dA[2], dX[2], afull[2], dD, drain;
+struct SlotBars {
+    uint64_t xfull, xempty, dA, dX, dD, afull, drain;
 };
 
 __device__ __forceinline__ uint32_t lanes(int quarter) { return (uint32_t)(32 * quarter) << 16; }
@@ -84,42 +87,43 @@ __device__ __forceinline__ uint32_t mn_off(int k, int n, uint32_t rk, uint32_t c
     return (uint32_t)(k >> 3) * rk + (uint32_t)(n >> 3) * cn + (uint32_t)(k & 7) * 16u + (uint32_t)(n & 7) * 2u;
 }
 
+// a descriptor advanced by a compile-time byte offset (the start address field
+// is the low 14 bits of address / 16; every operand ends below 256 KiB)
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 __global__ void __launch_bounds__(kThreads, 1)
 fused_fwd_t2(const __nv_bfloat16* __restrict__ u, const uint4* __restrict__ khat, const float* __restrict__ D,
              __nv_bfloat16* __restrict__ y, const uint4* __restrict__ mats, const uint2* __restrict__ twid,
              int* __restrict__ err, int B, int H, uint32_t wait_limit) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(8) Bars s_bar;
-    __shared__ int s_drained;
+    __shared__ __align__(8) SlotBars s_bar[2];
+    __shared__ int s_drained[2];
     __shared__ volatile int s_abort;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t sbase = tc::smem_u32(smem);
-    const int npp = (B + 1) / 2;            // row pairs per channel
-    const int nu = (npp + 1) / 2;           // units per channel
-    const int units = nu * H;
+    const int npp = (B + 1) / 2;   // row pairs per channel
+    const int pairs = npp * H;
     auto bar = [&](const uint64_t& b) { return tc::smem_u32(&b); };
 
-    // ---- set-up: constant matrices into shared memory, barriers, TMEM
-    for (int i = tid; i < (int)(kOffX / 16); i += kThreads) {
-        const uint4 val = __ldg(&mats[i]);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(sbase + 16u * i), "r"(val.x), "r"(val.y),
-                     "r"(val.z), "r"(val.w)
-                     : "memory");
-    }
+    // ---- set-up: constant matrices into shared memory (all copies in flight at
+    // once), barriers, TMEM
+    for (int i = tid; i < (int)(kOffX / 16); i += kThreads) tc::cp_async16(sbase + 16u * i, mats + i, 16);
+    tc::cp_async_commit();
+    tc::cp_async_wait_all();
     um::fence_proxy_async();
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            um::mbar_init(bar(s_bar.xfull[s]), 1);
-            um::mbar_init(bar(s_bar.xempty[s]), 1);
-            um::mbar_init(bar(s_bar.dA[s]), 1);
-            um::mbar_init(bar(s_bar.dX[s]), 1);
-            um::mbar_init(bar(s_bar.afull[s]), kEpiWarps);
+            um::mbar_init(bar(s_bar[s].xfull), 1);
+            um::mbar_init(bar(s_bar[s].xempty), 1);
+            um::mbar_init(bar(s_bar[s].dA), 1);
+            um::mbar_init(bar(s_bar[s].dX), 1);
+            um::mbar_init(bar(s_bar[s].dD), 1);
+            um::mbar_init(bar(s_bar[s].afull), kGroupWarps);
+            um::mbar_init(bar(s_bar[s].drain), 1);
+            s_drained[s] = 1;
         }
-        um::mbar_init(bar(s_bar.dD), 1);
-        um::mbar_init(bar(s_bar.drain), 1);
         s_abort = 0;
-        s_drained = 1;
     }
     if (warp == 0) {
         um::tmem_alloc(tc::smem_u32(&s_tmem), 512);
@@ -130,265 +134,265 @@ fused_fwd_t2(const __nv_bfloat16* __restrict__ u, const uint4* __restrict__ khat
     um::fence_after();
     const uint32_t tmem = s_tmem;
 
-    // a bounded wait; on give-up the CTA stops (every role polls the flag)
-    auto wait = [&](uint32_t b, uint32_t& parity) -> bool {
-        const bool ok = !s_abort && um::mbar_wait(b, parity, wait_limit);
-        parity ^= 1u;
+    // a bounded wait on barrier b with the expected phase parity in *par; on
+    // give-up the CTA stops (every role polls the flag)
+    auto wait = [&](uint32_t b, uint32_t& par) -> bool {
+        const bool ok = !s_abort && um::mbar_wait(b, par, wait_limit);
+        par ^= 1u;
         if (!ok) s_abort = 1;
         return ok;
     };
+    // the pairs of slot s: q = blockIdx.x + (2 i + s) gridDim.x
+    const int slot = warp < 8 ? (warp >> 2) : (warp < 10 ? warp - 8 : warp - 10);
+    const int q0 = blockIdx.x + slot * (int)gridDim.x, qstep = 2 * (int)gridDim.x;
+    SlotBars& sb = s_bar[slot];
+    const uint32_t tslot = tmem + 256u * (uint32_t)slot;           // Ra = + 0, Rb = + 128
+    const uint32_t xs = sbase + kOffX + 16384u * (uint32_t)slot;
+    const uint32_t vs = sbase + kOffV + 32768u * (uint32_t)slot;
 
-    if (warp == kIssuer) {
-        // ======================= MMA issuer
+    if (warp >= 8 && warp < 10) {
+        // ======================= MMA issuer of slot s
         if (lane == 0) {
             const uint32_t idA128 = um::idesc_bf16(128, 128) | um::kAmn | um::kBmn;
             const uint32_t idA64 = um::idesc_bf16(128, 64) | um::kAmn | um::kBmn;
             const uint32_t idBC = um::idesc_bf16(128, 128);
-            const uint32_t idD = um::idesc_bf16(128, 128) | um::kBmn;
-            uint32_t px[2] = {0u, 0u}, pa[2] = {0u, 0u};
-            auto stage_a = [&](int s) -> bool {
-                if (!wait(bar(s_bar.xfull[s]), px[s])) return false;
+            const uint32_t idD = um::idesc_bf16(128, 64) | um::kBmn;
+            const uint64_t gpA = um::sdesc(sbase + kOffGP, kGPm, kGPk);   // MN-major view for stage A
+            const uint64_t gpD = um::sdesc(sbase + kOffGP, kGPk, kGPm);   // K-major for stage D
+            const uint64_t xd = um::sdesc(xs, kXp, kXn);
+            const uint64_t fq = um::sdesc(sbase + kOffFQ, kFQk, kFQn);
+            const uint64_t vd = um::sdesc(vs, kVk, kVn);
+            uint32_t px = 0u, pa = 0u;
+            auto stage_a = [&]() -> bool {
+                if (!wait(bar(sb.xfull), px)) return false;
                 um::fence_after();
-                const uint32_t d = tmem + 256u * s, xs = sbase + kOffX + 16384u * s;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {  // cos view x [x_re | x_im]
-                    const uint64_t a = um::sdesc(sbase + kOffGP + ks * 2 * kGPm, kGPm, kGPk);
-                    um::mma_ss(d, a, um::sdesc(xs + ks * 2 * kXp, kXp, kXn), idA128, ks > 0);
-                }
+                for (int ks = 0; ks < 4; ++ks)  // cos view x [x_re | x_im]
+                    um::mma_ss(tslot, dadd(gpA, ks * 2 * kGPm), dadd(xd, ks * 2 * kXp), idA128, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {  // sin view: + sin x_im -> Re, - sin x_re -> Im
-                    const uint64_t a = um::sdesc(sbase + kOffGP + 2048u + ks * 2 * kGPm, kGPm, kGPk);
-                    um::mma_ss(d, a, um::sdesc(xs + 1024u + ks * 2 * kXp, kXp, kXn), idA64, 1);
-                    um::mma_ss(d + 64u, a, um::sdesc(xs + ks * 2 * kXp, kXp, kXn), idA64 | um::kNegA, 1);
+                    const uint64_t a = dadd(gpA, 2048u + ks * 2 * kGPm);
+                    um::mma_ss(tslot, a, dadd(xd, 1024u + ks * 2 * kXp), idA64, 1);
+                    um::mma_ss(tslot + 64u, a, dadd(xd, ks * 2 * kXp), idA64 | um::kNegA, 1);
                 }
-                um::mma_commit(bar(s_bar.dA[s]));
-                um::mma_commit(bar(s_bar.xempty[s]));
+                um::mma_commit(bar(sb.dA));
+                um::mma_commit(bar(sb.xempty));
                 return true;
             };
-            // B (src Ra -> dst Rb) or C (Rb -> Ra) of slot s
-            auto stage_bc = [&](int s, bool isC) -> bool {
-                if (!wait(bar(s_bar.afull[s]), pa[s])) return false;
+            // B (Ra -> Rb) or C (Rb -> Ra), once the epilogue has written the operand
+            auto stage_bc = [&](bool isC) -> bool {
+                if (!wait(bar(sb.afull), pa)) return false;
                 um::fence_after();
-                const uint32_t base = tmem + 256u * s;
-                const uint32_t src = base + (isC ? 128u : 0u), dst = base + (isC ? 0u : 128u);
+                const uint32_t src = tslot + (isC ? 128u : 0u), dst = tslot + (isC ? 0u : 128u);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    um::mma_ts(dst, src + 8u * ks, um::sdesc(sbase + kOffFQ + ks * 2 * kFQk, kFQk, kFQn), idBC, ks > 0);
-                um::mma_commit(bar(s_bar.dX[s]));
+                for (int ks = 0; ks < 8; ++ks) um::mma_ts(dst, src + 8u * ks, dadd(fq, ks * 2 * kFQk), idBC, ks > 0);
+                um::mma_commit(bar(sb.dX));
                 return true;
             };
             bool ok = true;
-            int i = 0;
-            for (int un = blockIdx.x; un < units && ok; un += gridDim.x, ++i) {
-                const bool two = 2 * (un % nu) + 1 < npp;
-                if (i == 0) {
-                    ok = stage_a(0) && (!two || stage_a(1));
-                    if (!ok) break;
-                }
-                ok = stage_bc(0, false) && (!two || stage_bc(1, false)) && stage_bc(0, true) &&
-                     (!two || stage_bc(1, true));
-                if (!ok) break;
-                // D: both pairs of the unit side by side (N = 128), into slot 0's Rb
-                ok = wait(bar(s_bar.afull[0]), pa[0]) && (!two || wait(bar(s_bar.afull[1]), pa[1]));
-                if (!ok) break;
+            for (int q = q0; q < pairs && ok; q += qstep) {
+                if (q == q0 && !(ok = stage_a())) break;
+                if (!(ok = stage_bc(false) && stage_bc(true))) break;
+                // D once epilogue C has filled V: rows p (Re) and 64 + p (Im), N = 64 q, into Rb
+                if (!(ok = wait(bar(sb.afull), pa))) break;
                 um::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 16; ++ks)
-                    um::mma_ss(tmem + 128u, um::sdesc(sbase + kOffGP + ks * 2 * kGPk, kGPk, kGPm),
-                               um::sdesc(sbase + kOffV + ks * 2 * kVk, kVk, kVn), idD, ks > 0);
-                um::mma_commit(bar(s_bar.dD));
-                // the next unit's stage A (its rows are staged by now or soon)
-                const int nx = un + gridDim.x;
-                if (nx < units) {
-                    const bool two2 = 2 * (nx % nu) + 1 < npp;
-                    ok = stage_a(0) && (!two2 || stage_a(1));
-                }
+                    um::mma_ss(tslot + 128u, dadd(gpD, ks * 2 * kGPk), dadd(vd, ks * 2 * kVk), idD, ks > 0);
+                um::mma_commit(bar(sb.dD));
+                // the next pair's stage A (Ra is free: epilogue C has read it)
+                if (q + qstep < pairs && !(ok = stage_a())) break;
             }
             // drain: every product issued is complete before TMEM is freed
-            um::mma_commit(bar(s_bar.drain));
-            s_drained = um::mbar_wait(bar(s_bar.drain), 0u) ? 1 : 0;
-            if (!ok || !s_drained) atomicExch(err, 1);
+            um::mma_commit(bar(sb.drain));
+            s_drained[slot] = um::mbar_wait(bar(sb.drain), 0u) ? 1 : 0;
+            if (!ok || !s_drained[slot]) atomicExch(err, 1);
         }
         __syncwarp();
-    } else if (warp == kLoader) {
-        // ======================= input rows of a unit into the two slots' planes
-        uint32_t pe[2] = {1u, 1u};  // a fresh barrier's previous phase counts as complete
-        for (int un = blockIdx.x; un < units; un += gridDim.x) {
-            const int h = un / nu, pp0 = 2 * (un % nu);
-            const bool two = pp0 + 1 < npp;
-            bool ok = true;
-            for (int s = 0; s < (two ? 2 : 1) && ok; ++s) ok = wait(bar(s_bar.xempty[s]), pe[s]);
-            if (!ok) break;
-            for (int s = 0; s < (two ? 2 : 1); ++s) {
-                const int b0 = 2 * (pp0 + s);
-                const uint32_t xs = sbase + kOffX + 16384u * s;
+    } else if (warp >= 10) {
+        // ======================= input rows of slot s's pairs
+        uint32_t pe = 1u;  // a fresh barrier's previous phase counts as complete
+        for (int q = q0; q < pairs; q += qstep) {
+            if (!wait(bar(sb.xempty), pe)) break;
+            const int h = q / npp, b0 = 2 * (q % npp);
 #pragma unroll 4
-                for (int it = 0; it < 32; ++it) {
-                    // lane -> (p mod 8, 8-q chunk): 64-byte global runs, 8 bank groups per store
-                    const int plane = it >> 4, pg = (it >> 1) & 7, qc = (lane >> 3) + 4 * (it & 1);
-                    const int p = 8 * pg + (lane & 7);
-                    const int b = b0 + plane;
-                    const bool has = b < B;
-                    const size_t off = ((size_t)(has ? b : b0) * H + h) * kN + (size_t)(kQ * p + 8 * qc);
-                    tc::cp_async16(xs + mn_off(p, 64 * plane + 8 * qc, kXp, kXn), u + off, has ? 16 : 0);
-                }
+            for (int it = 0; it < 32; ++it) {
+                // lane -> (p mod 8, 8-q chunk): 64-byte global runs, 8 bank groups per store
+                const int plane = it >> 4, pg = (it >> 1) & 7, qc = (lane >> 3) + 4 * (it & 1);
+                const int p = 8 * pg + (lane & 7);
+                const int b = b0 + plane;
+                const bool has = b < B;
+                const size_t off = ((size_t)(has ? b : b0) * H + h) * kN + (size_t)(kQ * p + 8 * qc);
+                tc::cp_async16(xs + mn_off(p, 64 * plane + 8 * qc, kXp, kXn), u + off, has ? 16 : 0);
             }
             tc::cp_async_commit();
             tc::cp_async_wait_all();
             um::fence_proxy_async();
             __syncwarp();
-            if (lane == 0)
-                for (int s = 0; s < (two ? 2 : 1); ++s) um::mbar_arrive(bar(s_bar.xfull[s]));
+            if (lane == 0) um::mbar_arrive(bar(sb.xfull));
         }
         tc::cp_async_wait_all();
     } else {
-        // ======================= epilogue warps
-        const int quarter = warp & 3, ch = warp >> 2;
+        // ======================= epilogue warps of slot s: TMEM lanes 32 quarter .., both column halves
+        const int quarter = warp & 3;
         const int r = 32 * quarter + lane;  // TMEM lane: k_p in stages A-C
-        const uint32_t tl = tmem + lanes(quarter);
-        uint2 tw[16];  // (cos, sin) pairs of W_M^{q k_p}, q = 32 ch + 2 i, + 1
-#pragma unroll
-        for (int i = 0; i < 16; ++i) tw[i] = __ldg(&twid[(r * 2 + ch) * 16 + i]);
-        uint32_t pdA[2] = {0u, 0u}, pdX[2] = {0u, 0u}, pdD = 0u;
-        auto arrive = [&](int s) {
+        const uint32_t tl = tslot + lanes(quarter);
+        uint32_t pdA = 0u, pdX = 0u, pdD = 0u;
+        auto arrive = [&]() {
             um::fence_before();
             __syncwarp();
-            if (lane == 0) um::mbar_arrive(bar(s_bar.afull[s]));
+            if (lane == 0) um::mbar_arrive(bar(sb.afull));
         };
-        // read this thread's 32 Re and 32 Im accumulators of the half ch at column col
-        auto load = [&](uint32_t col, uint32_t (&re)[32], uint32_t (&im)[32]) {
-            um::ld32x32_x32(tl + col + 32u * ch, re);
-            um::ld32x32_x32(tl + col + 64u + 32u * ch, im);
+        // this thread's 32 Re and 32 Im accumulators of column half hf at column col
+        auto load = [&](uint32_t col, int hf, uint32_t (&re)[32], uint32_t (&im)[32]) {
+            um::ld32x32_x32(tl + col + 32u * hf, re);
+            um::ld32x32_x32(tl + col + 64u + 32u * hf, im);
             um::wait_ld<32>(re);
             um::wait_ld<32>(im);
         };
-        // the next stage's A operand, in this thread's own columns: Re pairs then Im pairs
-        auto store_a = [&](uint32_t col, const uint32_t (&ar)[16], const uint32_t (&ai)[16]) {
-            um::st32x32_x16(tl + col + 32u * ch, ar);
-            um::st32x32_x16(tl + col + 32u * ch + 16u, ai);
-            um::wait_st();
+        // the next stage's A operand in the thread's own columns: Re pairs then Im pairs
+        auto store_a = [&](uint32_t col, int hf, const uint32_t (&ar)[16], const uint32_t (&ai)[16]) {
+            um::st32x32_x16(tl + col + 32u * hf, ar);
+            um::st32x32_x16(tl + col + 32u * hf + 16u, ai);
         };
-        for (int un = blockIdx.x; un < units; un += gridDim.x) {
-            const int h = un / nu, pp0 = 2 * (un % nu);
-            const bool two = pp0 + 1 < npp;
-            const int ns = two ? 2 : 1;
+        auto fetch_tw = [&](int hf, uint2 (&tw)[16]) {
+            const uint2* t = twid + (r * 2 + hf) * 16;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tw[i] = __ldg(&t[i]);
+        };
+        // epilogue A / C: x W_M^{q k_p} on packed pairs
+        auto twiddle_half = [&](uint32_t col, int hf, uint32_t (&ar)[16], uint32_t (&ai)[16]) {
+            uint2 tw[16];
+            fetch_tw(hf, tw);
+            uint32_t re[32], im[32];
+            load(col, hf, re, im);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                ar[i] = tc::pack2(__uint_as_float(re[2 * i]), __uint_as_float(re[2 * i + 1]));
+                ai[i] = tc::pack2(__uint_as_float(im[2 * i]), __uint_as_float(im[2 * i + 1]));
+                tc::twiddle2<true>(ar[i], ai[i], tw[i]);
+            }
+        };
+        for (int q = q0; q < pairs; q += qstep) {
+            const int h = q / npp, b0 = 2 * (q % npp);
             bool ok = true;
-            // spectrum words of (h, k_p, half): 16 Re pairs, 16 negated-Im pairs
-            uint4 kv[8];
-            const uint4* kp = khat + ((size_t)(h * kP + r) * 2 + ch) * 8;
+            // spectrum words of (h, k_p): per half 16 Re pairs and 16 negated-Im pairs
+            uint4 kv[16];
+            {
+                const uint4* kp = khat + (size_t)(h * kP + r) * 16;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) kv[i] = __ldg(&kp[i]);
-            const float dmf = D ? D[h] * (1.0f / kM) : 0.f;
-            const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
-            // ---- epilogue A: x W_M^{q k_p} -> A operand of stage B (slot columns 0..63)
-            for (int s = 0; s < ns && ok; ++s) {
-                if (!(ok = wait(bar(s_bar.dA[s]), pdA[s]))) break;
-                um::fence_after();
-                uint32_t re[32], im[32], ar[16], ai[16];
-                load(256u * s, re, im);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    ar[i] = tc::pack2(__uint_as_float(re[2 * i]), __uint_as_float(re[2 * i + 1]));
-                    ai[i] = tc::pack2(__uint_as_float(im[2 * i]), __uint_as_float(im[2 * i + 1]));
-                    tc::twiddle2<true>(ar[i], ai[i], tw[i]);
-                }
-                store_a(256u * s, ar, ai);
-                arrive(s);
+                for (int i = 0; i < 16; ++i) kv[i] = __ldg(&kp[i]);
             }
-            if (!ok) break;
-            // ---- epilogue B: Z = conj(X (Khat + D/M)) -> A operand of stage C (columns 128..191)
-            for (int s = 0; s < ns && ok; ++s) {
-                if (!(ok = wait(bar(s_bar.dX[s]), pdX[s]))) break;
-                um::fence_after();
-                uint32_t re[32], im[32], ar[16], ai[16];
-                load(256u * s + 128u, re, im);
-                const uint32_t* kw = reinterpret_cast<const uint32_t*>(kv);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const __nv_bfloat162 xr = tc::as_b2(tc::pack2(__uint_as_float(re[2 * i]), __uint_as_float(re[2 * i + 1])));
-                    const __nv_bfloat162 xi = tc::as_b2(tc::pack2(__uint_as_float(im[2 * i]), __uint_as_float(im[2 * i + 1])));
-                    const __nv_bfloat162 kr = __hadd2(tc::as_b2(kw[i]), dm2), kin = tc::as_b2(kw[16 + i]);
-                    // Re Z = xr kr - xi ki;  -Im Z = -(xr ki + xi kr) = xr kin - xi kr
-                    ar[i] = tc::as_u(__hfma2(xr, kr, __hmul2(xi, kin)));
-                    ai[i] = tc::as_u(__hfma2(xr, kin, __hneg2(__hmul2(xi, kr))));
-                }
-                store_a(256u * s + 128u, ar, ai);
-                arrive(s);
+            const float dmf = D ? __ldg(&D[h]) * (1.0f / kM) : 0.f;
+            // ---- epilogue A: -> A operand of stage B (Ra columns 0..63)
+            if (!(ok = wait(bar(sb.dA), pdA))) break;
+            um::fence_after();
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t ar[16], ai[16];
+                twiddle_half(0u, hf, ar, ai);
+                store_a(0u, hf, ar, ai);
             }
-            if (!ok) break;
-            // ---- epilogue C: V = V0 W_M^{q k_p} -> stage-D operand in shared memory
-            for (int s = 0; s < ns && ok; ++s) {
-                if (!(ok = wait(bar(s_bar.dX[s]), pdX[s]))) break;
-                um::fence_after();
-                uint32_t re[32], im[32], vr[16], vi[16];
-                load(256u * s, re, im);
+            um::wait_st();
+            arrive();
+            // ---- epilogue B: Z = conj(X (Khat + D/M)) -> A operand of stage C (Rb columns 0..63)
+            if (!(ok = wait(bar(sb.dX), pdX))) break;
+            um::fence_after();
+            {
+                const __nv_bfloat162 dm2 = __floats2bfloat162_rn(dmf, dmf);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    vr[i] = tc::pack2(__uint_as_float(re[2 * i]), __uint_as_float(re[2 * i + 1]));
-                    vi[i] = tc::pack2(__uint_as_float(im[2 * i]), __uint_as_float(im[2 * i + 1]));
-                    tc::twiddle2<true>(vr[i], vi[i], tw[i]);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t re[32], im[32], ar[16], ai[16];
+                    load(128u, hf, re, im);
+                    const uint32_t* kw = reinterpret_cast<const uint32_t*>(kv + 8 * hf);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const __nv_bfloat162 xr =
+                            tc::as_b2(tc::pack2(__uint_as_float(re[2 * i]), __uint_as_float(re[2 * i + 1])));
+                        const __nv_bfloat162 xi =
+                            tc::as_b2(tc::pack2(__uint_as_float(im[2 * i]), __uint_as_float(im[2 * i + 1])));
+                        const __nv_bfloat162 kr = __hadd2(tc::as_b2(kw[i]), dm2), kin = tc::as_b2(kw[16 + i]);
+                        // Re Z = xr kr - xi ki;  -Im Z = -(xr ki + xi kr) = xr kin - xi kr
+                        ar[i] = tc::as_u(__hfma2(xr, kr, __hmul2(xi, kin)));
+                        ai[i] = tc::as_u(__hfma2(xr, kin, __hneg2(__hmul2(xi, kr))));
+                    }
+                    store_a(128u, hf, ar, ai);
                 }
-                // rows k = k_p (Re) and 128 + k_p (Im), columns n = 64 s + q
+            }
+            um::wait_st();
+            arrive();
+            // ---- epilogue C: V = V0 W_M^{q k_p} -> stage-D operand: rows k_p (Re), 128 + k_p (Im)
+            if (!(ok = wait(bar(sb.dX), pdX))) break;
+            um::fence_after();
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t vr[16], vi[16];
+                twiddle_half(0u, hf, vr, vi);
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
-                    const int n = 64 * s + 32 * ch + 8 * c8;
-                    const uint32_t ar = sbase + kOffV + mn_off(r, n, kVk, kVn);
-                    const uint32_t ai = sbase + kOffV + mn_off(128 + r, n, kVk, kVn);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(ar), "r"(vr[4 * c8]),
-                                 "r"(vr[4 * c8 + 1]), "r"(vr[4 * c8 + 2]), "r"(vr[4 * c8 + 3])
+                    const int n = 32 * hf + 8 * c8;
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(vs + mn_off(r, n, kVk, kVn)),
+                                 "r"(vr[4 * c8]), "r"(vr[4 * c8 + 1]), "r"(vr[4 * c8 + 2]), "r"(vr[4 * c8 + 3])
                                  : "memory");
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(ai), "r"(vi[4 * c8]),
-                                 "r"(vi[4 * c8 + 1]), "r"(vi[4 * c8 + 2]), "r"(vi[4 * c8 + 3])
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(vs + mn_off(128 + r, n, kVk, kVn)),
+                                 "r"(vi[4 * c8]), "r"(vi[4 * c8 + 1]), "r"(vi[4 * c8 + 2]), "r"(vi[4 * c8 + 3])
                                  : "memory");
                 }
-                um::fence_proxy_async();
-                arrive(s);
             }
-            if (!ok) break;
-            // ---- epilogue D: rows p (Re, lanes 0..63) and 64 + p (Im) of pair ch, q = 0..63
-            if (!(ok = wait(bar(s_bar.dD), pdD))) break;
+            um::fence_proxy_async();
+            arrive();
+            // ---- epilogue D: lane p (Re, row b0) or 64 + p (Im, row b0 + 1), q = 0..63.  The
+            // warp's 32 rows (contiguous in y) are staged in its own 4 KiB of the slot's V
+            // (free once D is complete), 16-byte chunks swizzled by row, then written out
+            // in whole 512-byte runs
+            if (!(ok = wait(bar(sb.dD), pdD))) break;
             um::fence_after();
             {
                 uint32_t v0[32], v1[32];
-                um::ld32x32_x32(tl + 128u + 64u * ch, v0);
-                um::ld32x32_x32(tl + 128u + 64u * ch + 32u, v1);
+                um::ld32x32_x32(tl + 128u, v0);
+                um::ld32x32_x32(tl + 160u, v1);
                 um::wait_ld<32>(v0);
                 um::wait_ld<32>(v1);
-                const int b = 2 * (pp0 + ch) + (quarter >> 1);
-                if (ch < ns && b < B) {
-                    const int p = r & 63;
-                    uint4* dst = reinterpret_cast<uint4*>(y + ((size_t)b * H + h) * kN + (size_t)kQ * p);
+                const int plane = quarter >> 1, p0 = 32 * (quarter & 1);
+                const uint32_t wbase = vs + (uint32_t)quarter * 4096u;
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 o;
-                        o.x = tc::pack2(__uint_as_float(v0[8 * c8]), __uint_as_float(v0[8 * c8 + 1]));
-                        o.y = tc::pack2(__uint_as_float(v0[8 * c8 + 2]), __uint_as_float(v0[8 * c8 + 3]));
-                        o.z = tc::pack2(__uint_as_float(v0[8 * c8 + 4]), __uint_as_float(v0[8 * c8 + 5]));
-                        o.w = tc::pack2(__uint_as_float(v0[8 * c8 + 6]), __uint_as_float(v0[8 * c8 + 7]));
-                        dst[c8] = o;
-                    }
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint32_t* vv = c8 < 4 ? v0 + 8 * c8 : v1 + 8 * (c8 - 4);
+                    const uint32_t w0 = tc::pack2(__uint_as_float(vv[0]), __uint_as_float(vv[1]));
+                    const uint32_t w1 = tc::pack2(__uint_as_float(vv[2]), __uint_as_float(vv[3]));
+                    const uint32_t w2 = tc::pack2(__uint_as_float(vv[4]), __uint_as_float(vv[5]));
+                    const uint32_t w3 = tc::pack2(__uint_as_float(vv[6]), __uint_as_float(vv[7]));
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                     wbase + (uint32_t)lane * 128u + 16u * (uint32_t)(c8 ^ (lane & 7))),
+                                 "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                                 : "memory");
+                }
+                __syncwarp();
+                const int b = b0 + plane;
+                if (b < B) {
+                    __nv_bfloat16* dst = y + ((size_t)b * H + h) * kN + (size_t)kQ * p0;
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 o;
-                        o.x = tc::pack2(__uint_as_float(v1[8 * c8]), __uint_as_float(v1[8 * c8 + 1]));
-                        o.y = tc::pack2(__uint_as_float(v1[8 * c8 + 2]), __uint_as_float(v1[8 * c8 + 3]));
-                        o.z = tc::pack2(__uint_as_float(v1[8 * c8 + 4]), __uint_as_float(v1[8 * c8 + 5]));
-                        o.w = tc::pack2(__uint_as_float(v1[8 * c8 + 6]), __uint_as_float(v1[8 * c8 + 7]));
-                        dst[4 + c8] = o;
+                    for (int m = 0; m < 8; ++m) {
+                        const int j = lane + 32 * m, rr = j >> 3, c = j & 7;
+                        uint4 val;
+                        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                                     : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                     : "r"(wbase + (uint32_t)rr * 128u + 16u * (uint32_t)(c ^ (rr & 7))));
+                        *reinterpret_cast<uint4*>(dst + (size_t)kQ * rr + 8 * c) = val;
                     }
                 }
+                __syncwarp();
             }
-            // Rb of slot 0 is rewritten by the next unit's stage B only after that
-            // unit's epilogue A, which this warp reaches after these reads
-            um::fence_before();
+            // Rb and V are rewritten by the next pair's stage B and epilogue C only
+            // after its epilogue A, which every warp of the group reaches after these reads
         }
     }
-    // every wait above is bounded and the issuer has drained its products; if
-    // even the drain gave up, TMEM stays allocated rather than freed under a
+    // every wait above is bounded and the issuers have drained their products;
+    // if even a drain gave up, TMEM stays allocated rather than freed under a
     // running product (the status word is set)
     um::fence_before();
     __syncthreads();
-    if (warp == 0 && s_drained) {
+    if (warp == 0 && s_drained[0] && s_drained[1]) {
         um::fence_after();
         um::tmem_dealloc(tmem, 512);
     }
@@ -498,8 +502,8 @@ cudaError_t launch_t2_fwd(const fftconv_plan_s& p, const void* u, const void* kh
         cudaGetLastError();
         if (sms <= 0) sms = 1;
     }
-    const int npp = (p.B + 1) / 2, units = ((npp + 1) / 2) * p.H;
-    dim3 grid(units < sms ? units : sms);
+    const int pairs = ((p.B + 1) / 2) * p.H;  // each CTA walks its pairs alternately on its two slots
+    dim3 grid(pairs < sms ? pairs : sms);
     kern<<<grid, t2::kThreads, t2::kSmemBytes, s>>>((const __nv_bfloat16*)u, (const uint4*)khat, D,
                                                     (__nv_bfloat16*)y, p.t2_mats, p.t2_twid, p.d_err, p.B, p.H,
                                                     p.wait_limit);

@@ -172,8 +172,11 @@ fftconv_status fftconv_plan_create_ex(fftconv_plan_t* out, int B, int H, int64_t
     const int64_t M = int64_t(1) << p->log2M;
     size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0, offT2[2] = {0, 0};
     const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && o.kernel != FFTCONV_KERNEL_SIMT;
-    if (use_tc && o.kernel == FFTCONV_KERNEL_TCGEN05 && fftc::t2_supported(p->log2M, p->gated)) {
-        // two-stage tcgen05 kernel, data in tensor memory between the stages
+    if (use_tc && (o.kernel == FFTCONV_KERNEL_AUTO || o.kernel == FFTCONV_KERNEL_TCGEN05) &&
+        fftc::t2_supported(p->log2M, p->gated)) {
+        // two-stage tcgen05 kernel, data in tensor memory between the stages (the
+        // fastest measured at 2N = 8192: 79.8 us against 88.8 us for the mma.sync
+        // kernel on the Hyena-style workload, same box)
         p->path = fftc::PATH_FUSED_TC;
         p->t2 = true;
         fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the SIMT spectrum transform
@@ -320,8 +323,154 @@ fftconv_status fftconv_plan_destroy(fftconv_plan_t p) {
     if (!p) return FFTCONV_OK;
     cudaError_t e = cudaSuccess;
     if (p->d_tables) e = cudaFree(p->d_tables);
+    if (p->d_ssm && cudaFree(p->d_ssm) != cudaSuccess) e = cudaErrorUnknown;
+    if (p->d_keep && cudaFree(p->d_keep) != cudaSuccess) e = cudaErrorUnknown;
+    if (p->chunk && fftconv_plan_destroy(p->chunk) != FFTCONV_OK) e = cudaErrorUnknown;
     delete p;
     return e == cudaSuccess ? FFTCONV_OK : FFTCONV_ERR_CUDA;
+}
+
+fftconv_status fftconv_ssm_plan_create(fftconv_plan_t* out, int B, int H, int64_t N, fftconv_dtype dtype,
+                                       int d_state, int64_t chunk) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
+    if (d_state < 1 || d_state > FFTCONV_SSM_MAX_STATE) return FFTCONV_ERR_INVALID_ARG;
+    if (!is_pow2(chunk) || chunk < FFTCONV_SSM_MIN_CHUNK || chunk > FFTCONV_SSM_MAX_CHUNK) return FFTCONV_ERR_UNSUPPORTED;
+    if (N < chunk || N % chunk != 0 || N / chunk > 65535) return FFTCONV_ERR_UNSUPPORTED;
+    const int64_t nc = N / chunk;
+    if ((int64_t)H * nc > 65535) return FFTCONV_ERR_UNSUPPORTED;
+    fftconv_plan_options o = defaults();
+    o.kernel = FFTCONV_KERNEL_SIMT;
+    fftconv_plan_t ch = nullptr;
+    fftconv_status st = fftconv_plan_create_ex(&ch, B, (int)(H * nc), chunk, dtype, 0, &o);
+    if (st != FFTCONV_OK) return st;
+    if (ch->path != fftc::PATH_FUSED) {
+        fftconv_plan_destroy(ch);
+        return FFTCONV_ERR_UNSUPPORTED;
+    }
+    ch->kdiv = (int)nc;
+    fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
+    if (!p) {
+        fftconv_plan_destroy(ch);
+        return FFTCONV_ERR_OOM;
+    }
+    p->kind = 3;
+    p->path = fftc::PATH_SSM;
+    p->B = B;
+    p->H = H;
+    p->N = N;
+    p->dtype = dtype;
+    p->pairs = (int64_t)((B + 1) / 2) * H;
+    p->chunk = ch;
+    p->d_state = d_state;
+    p->T = chunk;
+    p->nchunks = nc;
+    p->device = ch->device;
+    p->d_err = ch->d_err;
+    if (cudaMalloc(&p->d_ssm, fftc::ssm_block_bytes(H, d_state, chunk)) != cudaSuccess) {
+        cudaGetLastError();
+        p->d_ssm = nullptr;
+        fftconv_plan_destroy(p);
+        return FFTCONV_ERR_OOM;
+    }
+    p->spectrum_bytes = (size_t)H * 2 * chunk * sizeof(float2);
+    p->workspace_bytes = fftc::ssm_workspace_bytes(*p);
+    *out = p;
+    return FFTCONV_OK;
+}
+
+int fftconv_spectrum_blocks(fftconv_plan_t p) {
+    return (p && p->kind == 1 && p->path == fftc::PATH_MULTIPASS) ? (1 << p->log2N1) : 0;
+}
+
+fftconv_status fftconv_spectrum_sparsify(fftconv_plan_t p, void* khat, const uint8_t* keep, int nblocks,
+                                         void* stream) {
+    if (!p || !khat || !aligned16(khat)) return FFTCONV_ERR_INVALID_ARG;
+    if (p->kind != 1 || p->path != fftc::PATH_MULTIPASS) return FFTCONV_ERR_UNSUPPORTED;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!keep) {  // dense again (the spectrum must be recomputed to undo the zeroing)
+        if (nblocks != 0) return FFTCONV_ERR_INVALID_ARG;
+        if (p->d_keep) {
+            if (cudaStreamSynchronize(s) != cudaSuccess || cudaFree(p->d_keep) != cudaSuccess) {
+                cudaGetLastError();
+                return FFTCONV_ERR_CUDA;
+            }
+            p->d_keep = nullptr;
+        }
+        return FFTCONV_OK;
+    }
+    const int G = 1 << p->log2N1;
+    if (nblocks != G) return FFTCONV_ERR_INVALID_ARG;
+    for (int j = 0; j < G; ++j)  // Hermitian symmetry keeps the packed rows apart
+        if ((keep[j] != 0) != (keep[(G - j) % G] != 0)) return FFTCONV_ERR_INVALID_ARG;
+    if (!p->d_keep && cudaMalloc(&p->d_keep, (size_t)G) != cudaSuccess) {
+        cudaGetLastError();
+        p->d_keep = nullptr;
+        return FFTCONV_ERR_OOM;
+    }
+    std::vector<uint8_t> flags(G);
+    for (int j = 0; j < G; ++j) flags[j] = keep[j] ? 1 : 0;
+    if (cudaMemcpyAsync(p->d_keep, flags.data(), (size_t)G, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return FFTCONV_ERR_CUDA;
+    }
+    return cuda_status(fftc::launch_zero_spectrum_rows(*p, khat, s));
+}
+
+fftconv_status fftconv_partial_plan_create(fftconv_plan_t* out, int B, int H, int64_t N, fftconv_dtype dtype,
+                                           int gated, int64_t L_max) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || L_max < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
+    int64_t T = 64;
+    while (T < L_max) T <<= 1;
+    if (T > FFTCONV_PARTIAL_MAX_CHUNK || N < T || N % T != 0 || N / T > 65535) return FFTCONV_ERR_UNSUPPORTED;
+    const int64_t nc = N / T;
+    if ((int64_t)H * nc > 65535) return FFTCONV_ERR_UNSUPPORTED;
+    fftconv_plan_options o = defaults();
+    o.kernel = FFTCONV_KERNEL_SIMT;
+    fftconv_plan_t ch = nullptr;  // the tables of the 2T-point transform
+    fftconv_status st = fftconv_plan_create_ex(&ch, 1, H, T, dtype, 0, &o);
+    if (st != FFTCONV_OK) return st;
+    if (ch->path != fftc::PATH_FUSED) {
+        fftconv_plan_destroy(ch);
+        return FFTCONV_ERR_UNSUPPORTED;
+    }
+    fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
+    if (!p) {
+        fftconv_plan_destroy(ch);
+        return FFTCONV_ERR_OOM;
+    }
+    p->kind = 4;
+    p->path = fftc::PATH_PARTIAL;
+    p->B = B;
+    p->H = H;
+    p->N = N;
+    p->dtype = dtype;
+    p->gated = gated ? 1 : 0;
+    p->pairs = (int64_t)((B + 1) / 2) * H;
+    p->chunk = ch;
+    p->T = T;
+    p->nchunks = nc;
+    p->device = ch->device;
+    p->d_err = ch->d_err;
+    p->spectrum_bytes = (size_t)H * 2 * T * sizeof(float2);
+    p->workspace_bytes = 0;
+    *out = p;
+    return FFTCONV_OK;
+}
+
+fftconv_status fftconv_ssm_spectrum(fftconv_plan_t p, const float* lam_re, const float* lam_im, const float* c_re,
+                                    const float* c_im, void* khat, void* work, void* stream) {
+    if (!p || p->kind != 3 || !lam_re || !lam_im || !c_re || !c_im || !khat || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(khat) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    const cudaError_t e = fftc::launch_ssm_setup(*p, lam_re, lam_im, c_re, c_im, khat, work, (cudaStream_t)stream);
+    if (e == cudaSuccess) p->spectrum_ready = true;
+    return cuda_status(e);
 }
 
 size_t fftconv_spectrum_bytes(fftconv_plan_t p) { return p ? p->spectrum_bytes : 0; }
@@ -334,12 +483,22 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
         case fftc::PATH_FUSED_TC: return p->t2 ? "fused_t2" : (p->umma ? "fused_umma" : "fused_tc");
         case fftc::PATH_MULTIPASS: return "multipass";
         case fftc::PATH_2D: return p->tc2d ? "2d_tc" : "2d";
+        case fftc::PATH_SSM: return "ssm_chunked";
+        case fftc::PATH_PARTIAL: return "partial_chunked";
     }
     return "unknown";
 }
 
 fftconv_status fftconv_kernel_spectrum(fftconv_plan_t p, const float* k, int64_t L, void* khat, void* work,
                                        void* stream) {
+    if (p && p->kind == 4) {
+        // partial plans: the 2T-point spectrum of k[:L], L <= T
+        if (!k || !khat || L < 1 || L > p->T || !aligned16(k) || !aligned16(khat)) return FFTCONV_ERR_INVALID_ARG;
+        if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+        const cudaError_t e = fftc::launch_fused_spectrum(*p->chunk, k, L, (float2*)khat, (cudaStream_t)stream);
+        if (e == cudaSuccess) p->spectrum_ready = true;
+        return cuda_status(e);
+    }
     if (!p || p->kind != 1 || !k || !khat || L < 1 || L > p->N) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(khat)) return FFTCONV_ERR_INVALID_ARG;
     if (p->workspace_bytes && (!work || !aligned16(work))) return FFTCONV_ERR_INVALID_ARG;
@@ -360,7 +519,7 @@ fftconv_status fftconv_kernel_spectrum(fftconv_plan_t p, const float* k, int64_t
 
 fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const void* w, const void* khat,
                            const float* D, void* y, void* work, void* stream) {
-    if (!p || p->kind != 1 || !u || !khat || !y) return FFTCONV_ERR_INVALID_ARG;
+    if (!p || (p->kind != 1 && p->kind != 3 && p->kind != 4) || !u || !khat || !y) return FFTCONV_ERR_INVALID_ARG;
     if (p->gated ? (!v || !w) : (v || w)) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || (v && !aligned16(v)) || (w && !aligned16(w)) ||
         (D && !aligned16(D)))
@@ -371,7 +530,11 @@ fftconv_status fftconv_fwd(fftconv_plan_t p, const void* u, const void* v, const
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (p->t2)
+    if (p->kind == 3)
+        e = fftc::launch_ssm_fwd(*p, u, khat, D, y, work, s);
+    else if (p->kind == 4)
+        e = fftc::launch_partial_fwd(*p, u, v, w, (const float2*)khat, D, y, s);
+    else if (p->t2)
         e = fftc::launch_t2_fwd(*p, u, khat, D, y, s);
     else if (p->path == fftc::PATH_FUSED_TC)
         e = p->umma ? fftc::launch_umma_fwd(*p, u, v, w, khat, D, y, s) : fftc::launch_tc_fwd(*p, u, v, w, khat, D, y, s);

@@ -11,7 +11,7 @@
 
 namespace fftc {
 
-enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2, PATH_FUSED_TC = 3 };
+enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2, PATH_FUSED_TC = 3, PATH_SSM = 4, PATH_PARTIAL = 5 };
 
 // Twiddle tables of one plan (device pointers into one allocation).  wL / wC
 // are per-stage tables of the row / column transforms (StageTwiddles layout);
@@ -45,7 +45,7 @@ struct C2TcTables {
 }  // namespace fftc
 
 struct fftconv_plan_s {
-    int kind = 1;          // 1: 1-D, 2: 2-D
+    int kind = 1;          // 1: 1-D, 2: 2-D, 3: state-space filters, chunked, 4: partial, chunked
     int path = 0;          // fftc::Path
     int B = 0, H = 0;      // 1-D batch, channels (2-D: B images, H = C channels)
     int64_t N = 0;         // 1-D sequence length
@@ -75,6 +75,14 @@ struct fftconv_plan_s {
     int device = 0;
     int kernel = 0;                 // fftconv_kernel the caller asked for at creation
     uint32_t wait_limit = 1u << 16; // probes per bounded device wait (fftconv_plan_set_wait_limit)
+    int kdiv = 1;                   // fused SIMT forward: row channels per spectrum channel
+    // chunked state-passing plans (kind 3): the chunk plan and the filters' state-space model
+    fftconv_plan_s* chunk = nullptr;  // fused plan of B x (H * nchunks) x T rows
+    int d_state = 0;                  // states per channel
+    int64_t T = 0, nchunks = 0;       // chunk length, chunks per row
+    void* d_ssm = nullptr;            // plan-owned: lam, c, the power table (see conv1d_ssm.cu)
+    bool ssm_ready = false;
+    uint8_t* d_keep = nullptr;        // frequency-sparse multi-pass plans: keep flag per outer row k1
 };
 
 namespace fftc {
@@ -97,6 +105,21 @@ cudaError_t launch_t2_fwd(const fftconv_plan_s& p, const void* u, const void* kh
 bool dyn_supported(int log2M);
 cudaError_t launch_dyn_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w, const float* k,
                            int64_t L, const float* D, void* y, cudaStream_t s);
+
+// Chunked state passing for filters of a diagonal state-space model.
+size_t ssm_block_bytes(int H, int d, int64_t T);
+size_t ssm_workspace_bytes(const fftconv_plan_s& p);
+cudaError_t launch_ssm_setup(const fftconv_plan_s& p, const float* lr, const float* li, const float* cr,
+                             const float* ci, void* khat, void* work, cudaStream_t s);
+cudaError_t launch_ssm_fwd(const fftconv_plan_s& p, const void* u, const void* khat, const float* D, void* y,
+                           void* work, cudaStream_t s);
+
+// Frequency-sparse multi-pass plans: zero the dropped spectrum rows.
+cudaError_t launch_zero_spectrum_rows(const fftconv_plan_s& p, void* khat, cudaStream_t s);
+
+// Partial convolutions (L <= T), overlap-save in chunks of T on the fused fp32 kernel.
+cudaError_t launch_partial_fwd(const fftconv_plan_s& p, const void* u, const void* v, const void* w,
+                               const float2* khat, const float* D, void* y, cudaStream_t s);
 
 // Tensor-core flops of one forward call (0 for SIMT paths).
 double plan_mma_flops(const fftconv_plan_s& p);

@@ -155,9 +155,11 @@ FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
 
 /* Name of the execution path the plan chose: "fused" (fp32 on-chip),
  * "fused_tc" (bf16 on-chip, 2N <= 32768, warp-level mma.sync tensor cores),
- * "fused_umma" (the same factorisation on tcgen05 tensor cores, 2N = 4096 or
- * 8192), "fused_t2" (two-stage tcgen05 kernel, data held in tensor memory
- * between the stages, 2N = 8192), "multipass", "2d", "2d_tc". */
+ * "fused_umma" (the same factorisation on tcgen05 tensor cores, 2N = 4096,
+ * or 8192 gated, with FFTCONV_KERNEL_TCGEN05), "fused_t2" (two-stage tcgen05
+ * kernel, data held in tensor memory between the stages: the default for
+ * ungated bf16 at 2N = 8192), "multipass", "2d", "2d_tc", "partial_chunked",
+ * "ssm_chunked". */
 FFTCONV_API const char* fftconv_plan_path(fftconv_plan_t plan);
 
 /* Tensor-core floating-point operations (2 per multiply-add, as executed,
@@ -211,6 +213,73 @@ FFTCONV_API fftconv_status fftconv_fwd(fftconv_plan_t plan, const void* u, const
  */
 FFTCONV_API fftconv_status fftconv_fwd_dynamic(fftconv_plan_t plan, const void* u, const void* v, const void* w,
                                                const float* k, int64_t L, const float* D, void* y, void* stream);
+
+/*
+ * Frequency-sparse convolutions ("FlashFFTConv", abstract: frequency-sparse
+ * convolutions, computed by skipping blocks of the matrix decomposition), on
+ * multi-pass plans (2N >= 32768).  The transform splits 2N = G x (2N / G)
+ * with frequency f = k1 + G k2; keep[k1] = 0 zeroes the spectrum (skip term
+ * included) at every frequency of outer digit k1, and the kernels skip those
+ * rows: pass 1 stores nothing for them, pass 2 skips CTAs whose rows are all
+ * dropped, pass 3 reads zeros.  The result is
+ *     y = Re(iDFT(DFT(pad x) . (DFT(pad k) + D) . m))[:N],  m[f] = keep[f mod G].
+ * keep: host array of nblocks = fftconv_spectrum_blocks(plan) = G flags,
+ * Hermitian-symmetric (keep[j] == keep[(G - j) mod G], else
+ * FFTCONV_ERR_INVALID_ARG: the two packed rows would mix).  Zeroes the rows
+ * of khat (the output of fftconv_kernel_spectrum on this plan) and records
+ * the mask in the plan (a G-byte device array the plan owns); keep = NULL,
+ * nblocks = 0 makes the plan dense again (recompute khat).  Synchronises the
+ * stream.  FFTCONV_ERR_UNSUPPORTED for other plans.
+ */
+FFTCONV_API int fftconv_spectrum_blocks(fftconv_plan_t plan);
+FFTCONV_API fftconv_status fftconv_spectrum_sparsify(fftconv_plan_t plan, void* khat, const uint8_t* keep,
+                                                     int nblocks, void* stream);
+
+/*
+ * Partial convolutions: a filter of at most L_max taps, much shorter than the
+ * rows ("FlashFFTConv", abstract: partial convolutions, computed by skipping
+ * blocks of the matrix decomposition).  The row is cut into chunks of T (the
+ * power of two >= max(L_max, 64), at most FFTCONV_PARTIAL_MAX_CHUNK, dividing
+ * N); chunk c is the upper half of a 2T-point circular convolution over the
+ * window [cT - T, cT + T), which equals y there exactly because the filter
+ * is no longer than T.  Work and traffic scale with N log T and every chunk
+ * runs on chip, whatever N.  Same calls as a 1-D plan: fftconv_kernel_spectrum
+ * (1 <= L <= T taps; khat of fftconv_spectrum_bytes) and fftconv_fwd (gated
+ * or not, D optional; no workspace).  Path name "partial_chunked".
+ */
+#define FFTCONV_PARTIAL_MAX_CHUNK 8192
+FFTCONV_API fftconv_status fftconv_partial_plan_create(fftconv_plan_t* plan, int B, int H, int64_t N,
+                                                       fftconv_dtype dtype, int gated, int64_t L_max);
+
+/*
+ * Filters of a diagonal state-space model, computed in chunks with the state
+ * passed between them ("FlashConv", Mechanism: chunk convolutions past the
+ * on-chip length with the state-space boundary state propagated between
+ * chunks).  Channel h's filter is
+ *     k[h][t] = Re( sum_{j < d} c[h][j] lam[h][j]^t ),   t < N,  |lam| < 1,
+ * and the forward is the causal convolution of the header's first formula
+ * with that k (ungated).  A row is split into chunks of T (a power of two in
+ * [FFTCONV_SSM_MIN_CHUNK, FFTCONV_SSM_MAX_CHUNK] dividing N): each chunk is
+ * convolved on chip with k[:T] (the fp32 fused kernel) and the contribution
+ * of all earlier input, Re(sum_j c_j lam_j^t S_j), is added from the d
+ * states S entering the chunk, which a scan carries from chunk to chunk.
+ * The plan owns the chunk plan and a small table (lam, c, lam^(32 i));
+ * khat (fftconv_spectrum_bytes) and the workspace (fftconv_workspace_bytes)
+ * are the caller's.  Path name "ssm_chunked".
+ */
+#define FFTCONV_SSM_MAX_STATE 64
+#define FFTCONV_SSM_MIN_CHUNK 64
+#define FFTCONV_SSM_MAX_CHUNK 8192
+FFTCONV_API fftconv_status fftconv_ssm_plan_create(fftconv_plan_t* plan, int B, int H, int64_t N,
+                                                   fftconv_dtype dtype, int d_state, int64_t chunk);
+
+/* Set the filters: lam and c are [H][d] fp32 device arrays (real and
+ * imaginary parts separately).  Materialises k[:T], writes khat and keeps
+ * lam, c and their power table in the plan.  Then fftconv_fwd(plan, u, NULL,
+ * NULL, khat, D, y, workspace, stream) runs the chunked convolution. */
+FFTCONV_API fftconv_status fftconv_ssm_spectrum(fftconv_plan_t plan, const float* lam_re, const float* lam_im,
+                                                const float* c_re, const float* c_im, void* khat, void* workspace,
+                                                void* stream);
 
 /*
  * 2-D kernel spectrum: khat <- DFT_{2Hs x 2Ws}(k[c] zero-padded) / (4 Hs Ws)
