@@ -17,6 +17,7 @@ Definitions (see fftconv_oracle.c for the page citations):
 * ``causal_conv1d_bwd``: the gradients du (dv, dw), dk, dD of that y for an
   upstream gradient dy, by the chain rule written as direct sums.
 * ``causal_conv2d``: y[b,c,i,j] = sum_{p<=i,q<=j} k[c,p,q] u[b,c,i-p,j-q].
+* ``causal_conv2d_offset``: the same convolution, crop window moved by (oy, ox).
 * ``dft_causal_conv1d`` / ``dft_causal_conv2d``: the same results through an
   explicit O(M^2) DFT product (tiny sizes only), the independent second route.
 """
@@ -42,6 +43,7 @@ def bind(path):
     lib.oracle_causal_conv1d_dynamic.argtypes = [_i64] * 4 + [_f64p] * 6
     lib.oracle_ssm_kernel.argtypes = [_i64] * 3 + [_f64p] * 5
     lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
+    lib.oracle_causal_conv2d_offset.argtypes = [_i64] * 8 + [_f64p] * 3
     lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
     lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
     lib.oracle_dft_causal_conv2d.argtypes = [_i64] * 4 + [_f64p] * 3
@@ -210,6 +212,18 @@ def causal_conv2d(u, k) -> np.ndarray:
     return y
 
 
+def causal_conv2d_offset(u, k, oy, ox) -> np.ndarray:
+    """fp64 2-D oracle, crop window [oy, oy+Hs) x [ox, ox+Ws) of the full linear
+    convolution (0, 0: the first-quadrant crop; Hs/2, Ws/2: the centred one)."""
+    u, k = _check_2d(u, k)
+    B, C, Hs, Ws = u.shape
+    if not (0 <= oy <= Hs and 0 <= ox <= Ws):
+        raise ValueError("offset outside [0, Hs] x [0, Ws]")
+    y = np.empty_like(u)
+    _load().oracle_causal_conv2d_offset(B, C, Hs, Ws, k.shape[1], k.shape[2], int(oy), int(ox), _p(u), _p(k), _p(y))
+    return y
+
+
 def causal_conv2d_points(u, k, b_idx, c_idx, i_idx, j_idx) -> np.ndarray:
     """fp64 2-D oracle at sampled pixels."""
     u, k = _check_2d(u, k)
@@ -250,5 +264,5 @@ def dft_causal_conv2d(x, k) -> np.ndarray:
     return y
 
 
-__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "ssm_kernel", "freq_sparse_conv1d", "causal_conv2d", "causal_conv2d_points",
+__all__ = ["causal_conv1d", "causal_conv1d_points", "causal_conv1d_bwd", "causal_conv1d_dynamic", "ssm_kernel", "freq_sparse_conv1d", "causal_conv2d", "causal_conv2d_points", "causal_conv2d_offset",
            "dft_causal_conv1d", "dft_causal_conv2d", "num_threads"]

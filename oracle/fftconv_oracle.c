@@ -280,6 +280,40 @@ void oracle_causal_conv2d(int64_t B, int64_t C, int64_t Hs, int64_t Ws, int64_t 
     }
 }
 
+/*
+ * 2-D with a crop offset: the window [oy, oy + Hs) x [ox, ox + Ws) of the full
+ * (2Hs - 1) x (2Ws - 1) linear convolution instead of its first quadrant
+ * (oy = Hs/2, ox = Ws/2 is the centred "same" reading of a kernel anchored at
+ * its middle).  y[i][j] = sum_{p,q} k[p][q] u[i + oy - p][j + ox - q] over the
+ * indices inside both arrays.  0 <= oy <= Hs, 0 <= ox <= Ws.
+ */
+void oracle_causal_conv2d_offset(int64_t B, int64_t C, int64_t Hs, int64_t Ws, int64_t Kh, int64_t Kw,
+                                 int64_t oy, int64_t ox, const double* u, const double* k, double* y)
+{
+    int64_t imgs = B * C;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < imgs; ++r) {
+        int64_t c = r % C;
+        const double* ui = u + r * Hs * Ws;
+        const double* kc = k + c * Kh * Kw;
+        for (int64_t i = 0; i < Hs; ++i)
+            for (int64_t j = 0; j < Ws; ++j) {
+                int64_t fi = i + oy, fj = j + ox;
+                double acc = 0.0;
+                for (int64_t p = 0; p < Kh; ++p) {
+                    int64_t a = fi - p;
+                    if (a < 0 || a >= Hs) continue;
+                    for (int64_t q = 0; q < Kw; ++q) {
+                        int64_t bq = fj - q;
+                        if (bq < 0 || bq >= Ws) continue;
+                        acc += kc[p * Kw + q] * ui[a * Ws + bq];
+                    }
+                }
+                y[r * Hs * Ws + i * Ws + j] = acc;
+            }
+    }
+}
+
 /* Sampled 2-D oracle: out[n] = y[bi[n], ci[n], ii[n], jj[n]]. */
 void oracle_causal_conv2d_points(int64_t B, int64_t C, int64_t Hs, int64_t Ws, int64_t Kh,
                                  int64_t Kw, const double* u, const double* k, int64_t n_pts,

@@ -406,11 +406,29 @@ def check_freq_sparse():
     assert np.allclose(y2, 2.0 * y, rtol=1e-12, atol=1e-12)
 
 
+def check_conv2d_offset():
+    """Crop offsets: (0, 0) is the first-quadrant oracle; any offset is the
+    window of scipy.signal.convolve2d's full linear convolution."""
+    r = _rng(67)
+    u = r.standard_normal((2, 2, 12, 10))
+    k = r.standard_normal((2, 7, 10))
+    assert np.array_equal(oracle.causal_conv2d_offset(u, k, 0, 0), oracle.causal_conv2d(u, k))
+    for oy, ox in ((6, 5), (12, 10), (3, 0), (0, 8)):
+        y = oracle.causal_conv2d_offset(u, k, oy, ox)
+        for b in range(2):
+            for c in range(2):
+                full = scipy.signal.convolve2d(u[b, c], k[c], mode="full")
+                want = np.zeros((12, 10))
+                win = full[oy:oy + 12, ox:ox + 10]
+                want[:win.shape[0], :win.shape[1]] = win
+                assert np.allclose(y[b, c], want, rtol=1e-12, atol=1e-12), (oy, ox)
+
+
 ALL_CHECKS = [
     check_golden_1d, check_golden_2d, check_fft_formula_1d, check_numpy_convolve_1d,
     check_dft_route_1d, check_delta_identities, check_linearity_commutativity,
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
     check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
-    check_ssm_kernel, check_freq_sparse,
+    check_ssm_kernel, check_freq_sparse, check_conv2d_offset,
 ]

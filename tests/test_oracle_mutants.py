@@ -55,6 +55,8 @@ MUTANTS = {
     "ssm_drop_imag_part": ("acc += c_re[h * d + j] * pr - c_im[h * d + j] * pi;", "acc += c_re[h * d + j] * pr;"),
     "ssm_power_off_by_one": ("double mag = pow(sqrt(lr * lr + li * li), (double)t);",
                              "double mag = pow(sqrt(lr * lr + li * li), (double)(t + 1));"),
+    "conv2d_offset_ignored": ("int64_t fi = i + oy, fj = j + ox;", "int64_t fi = i, fj = j + ox;"),
+    "conv2d_offset_clip": ("if (a < 0 || a >= Hs) continue;", "if (a < 0 || a >= Hs - 1) continue;"),
 }
 
 
