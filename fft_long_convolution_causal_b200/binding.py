@@ -66,6 +66,7 @@ _SIGS = {
     "fftconv_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv2d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
     "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "fftconv2d_fwd_offset": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int]),
     "fftconv_fwd_static_workspace": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv_static_workspace_bytes": (ctypes.c_size_t, []),
     "fftconv_device_status": (ctypes.c_int, [_vp, _vp]),
@@ -353,15 +354,18 @@ class Plan2D(_PlanBase):
         return khat
 
     def fwd(self, u: torch.Tensor, khat: torch.Tensor, y: Optional[torch.Tensor] = None,
-            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+            workspace: Optional[torch.Tensor] = None, stream=None, offset=(0, 0)) -> torch.Tensor:
+        """y = window [oy, oy+Hs) x [ox, ox+Ws) of the full linear convolution
+        (offset (0, 0): the first-quadrant crop; (Hs/2, Ws/2): the centred one)."""
         shape = (self.B, self.C, self.Hs, self.Ws)
         _need(u, "u", shape, self.torch_dtype)
         if y is None:
             y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
         _need(y, "y", shape, self.torch_dtype)
         workspace = self._ws(workspace)
-        _check(self.lib.fftconv2d_fwd(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace),
-                                      _stream(stream)), "fftconv2d_fwd")
+        oy, ox = (int(offset[0]), int(offset[1]))
+        _check(self.lib.fftconv2d_fwd_offset(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace),
+                                             _stream(stream), oy, ox), "fftconv2d_fwd_offset")
         return y
 
 

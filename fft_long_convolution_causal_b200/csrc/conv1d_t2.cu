@@ -63,7 +63,8 @@ constexpr uint32_t kOffGP = 0;            // outer DFT matrix, [m 128][k 256] K-
 constexpr uint32_t kOffFQ = 65536;        // inner DFT matrix, [n 128][k 128] K-major, 32 KiB
 constexpr uint32_t kOffX = 98304;         // input planes of slot s at + 16 KiB s: [p 64][n 128] MN-major
 constexpr uint32_t kOffV = 131072;        // stage-D operand of slot s at + 32 KiB s: [k 256][n 64] MN-major
-constexpr uint32_t kSmemBytes = 196608;
+constexpr uint32_t kOffTW = 196608;       // twiddle pairs of W_M^{q k_p}: [half 2][i 16][k_p 128] uint2, 32 KiB
+constexpr uint32_t kSmemBytes = 229376;
 
 // core-matrix strides of each operand (bytes)
 constexpr uint32_t kGPm = 4096, kGPk = 128;   // GP: row group (8 m) / column group (8 k)
@@ -109,6 +110,8 @@ fused_fwd_t2(const __nv_bfloat16* __restrict__ u, const uint4* __restrict__ khat
     // ---- set-up: constant matrices into shared memory (all copies in flight at
     // once), barriers, TMEM
     for (int i = tid; i < (int)(kOffX / 16); i += kThreads) tc::cp_async16(sbase + 16u * i, mats + i, 16);
+    for (int i = tid; i < 2048; i += kThreads)
+        tc::cp_async16(sbase + kOffTW + 16u * i, reinterpret_cast<const uint4*>(twid) + i, 16);
     tc::cp_async_commit();
     tc::cp_async_wait_all();
     um::fence_proxy_async();
@@ -255,10 +258,14 @@ fused_fwd_t2(const __nv_bfloat16* __restrict__ u, const uint4* __restrict__ khat
             um::st32x32_x16(tl + col + 32u * hf, ar);
             um::st32x32_x16(tl + col + 32u * hf + 16u, ai);
         };
+        // twiddles from shared memory: consecutive lanes read consecutive 8-byte words
         auto fetch_tw = [&](int hf, uint2 (&tw)[16]) {
-            const uint2* t = twid + (r * 2 + hf) * 16;
+            const uint32_t t = sbase + kOffTW + (uint32_t)((hf * 16) * 128 + r) * 8u;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) tw[i] = __ldg(&t[i]);
+            for (int i = 0; i < 16; ++i)
+                asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];\n"
+                             : "=r"(tw[i].x), "=r"(tw[i].y)
+                             : "r"(t + (uint32_t)i * 1024u));
         };
         // epilogue A / C: x W_M^{q k_p} on packed pairs
         auto twiddle_half = [&](uint32_t col, int hf, uint32_t (&ar)[16], uint32_t (&ai)[16]) {
@@ -471,12 +478,12 @@ bool t2_tables(std::vector<float2>& out, size_t off[2]) {
     size_t base = out.size();
     out.resize(base + img.size() / sizeof(float2));
     memcpy(&out[base], img.data(), img.size());
-    // twiddles: [k_p][half][i] -> (bf16x2 cos(q0, q0 + 1), bf16x2 sin(...)), q0 = 32 half + 2 i
+    // twiddles: [half][i][k_p] -> (bf16x2 cos(q0, q0 + 1), bf16x2 sin(...)), q0 = 32 half + 2 i
     off[1] = out.size();
     std::vector<Word32> tw;
-    for (int kp = 0; kp < kP; ++kp)
-        for (int hf = 0; hf < 2; ++hf)
-            for (int i = 0; i < 16; ++i) {
+    for (int hf = 0; hf < 2; ++hf)
+        for (int i = 0; i < 16; ++i)
+            for (int kp = 0; kp < kP; ++kp) {
                 double c0, s0, c1, s1;
                 const int q0 = 32 * hf + 2 * i;
                 cs_t2((int64_t)q0 * kp, kM, &c0, &s0);

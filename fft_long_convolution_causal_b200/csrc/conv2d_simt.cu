@@ -94,7 +94,7 @@ c2_pass1(const IO* __restrict__ u, const float* __restrict__ k, int Kh, int Kw, 
 template <int LOG2LC, int LOG2LR, int MODE, bool KB, bool KTC = false>
 __global__ void __launch_bounds__(Col2G<LOG2LC>::T)
 c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restrict__ khat_out,
-         const float2* __restrict__ twC, int npp, int64_t first) {
+         const float2* __restrict__ twC, int npp, int64_t first, int oy) {
     using G = Col2G<LOG2LC>;
     using Lay = typename G::Lay;
     constexpr int LC = 1 << LOG2LC, LR = 1 << LOG2LR, Hs = LC / 2;
@@ -151,8 +151,9 @@ c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restr
             sts);
         __syncthreads();
         smem_stages<G, 1, NS - 1, true>(smem, tid, twC);
-        stage<G, NS - 1, true, RL, RL / 2, false>(tid, twC, lds, [&](int i, int c, float2 z) {
-            img[(size_t)i * LR + kx0 + c] = z;
+        // rows oy .. oy + Hs - 1 of the inverse (the crop window; 0 .. Hs - 1 by default)
+        stage<G, NS - 1, true, RL, RL, false>(tid, twC, lds, [&](int i, int c, float2 z) {
+            if (i >= oy && i < oy + Hs) img[(size_t)(i - oy) * LR + kx0 + c] = z;
         });
     }
 }
@@ -161,7 +162,7 @@ c2_pass2(float2* __restrict__ work, const void* __restrict__ khat, void* __restr
 template <int LOG2LR, int RB, typename IO>
 __global__ void __launch_bounds__(Row2G<LOG2LR, RB>::T)
 c2_pass3(const float2* __restrict__ work, IO* __restrict__ y, const float2* __restrict__ twR, int B, int C,
-         int Hs, int64_t first) {
+         int Hs, int64_t first, int ox) {
     using G = Row2G<LOG2LR, RB>;
     using Lay = typename G::Lay;
     constexpr int LR = 1 << LOG2LR, Ws = LR / 2;
@@ -182,8 +183,10 @@ c2_pass3(const float2* __restrict__ work, IO* __restrict__ y, const float2* __re
     const int ch = (int)(P / npp), b0 = (int)(P % npp) * 2;
     const bool has1 = b0 + 1 < B;
     const size_t img0 = ((size_t)b0 * C + ch) * Hs * Ws, img1 = ((size_t)(b0 + 1) * C + ch) * Hs * Ws;
-    stage<G, NS - 1, true, RL, RL / 2, false>(tid, twR, lds, [&](int j, int r, float2 z) {
-        const size_t off = (size_t)(i0 + r) * Ws + j;
+    // columns ox .. ox + Ws - 1 of the inverse (the crop window; 0 .. Ws - 1 by default)
+    stage<G, NS - 1, true, RL, RL, false>(tid, twR, lds, [&](int j, int r, float2 z) {
+        if (j < ox || j >= ox + Ws) return;
+        const size_t off = (size_t)(i0 + r) * Ws + (j - ox);
         y[img0 + off] = from_f<IO>(z.x);
         if (has1) y[img1 + off] = from_f<IO>(z.y);
     });
@@ -191,7 +194,7 @@ c2_pass3(const float2* __restrict__ work, IO* __restrict__ y, const float2* __re
 
 template <int LOG2LC, int LOG2LR, typename IO>
 static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float2* khat, void* y, float2* work,
-                             cudaStream_t s) {
+                             cudaStream_t s, int oy, int ox) {
     constexpr int Hs = (1 << LOG2LC) / 2;
     constexpr int RB = rows_per_cta<LOG2LR>(Hs);
     constexpr int LR = 1 << LOG2LR;
@@ -214,17 +217,17 @@ static cudaError_t c2_fwd_go(const fftconv_plan_s& p, const void* u, const float
                                                                  p.H, Hs, first);
         }
         if (p.tc2d) {
-            const cudaError_t e = launch_c2tc_cols(p, work, khat, g, first, s);
+            const cudaError_t e = launch_c2tc_cols(p, work, khat, g, first, s, oy);
             if (e != cudaSuccess) return e;
         } else {
             k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, khat, nullptr, p.tw.wC, (p.B + 1) / 2,
-                                                                    first);
+                                                                    first, oy);
         }
         if (tc_rows) {
-            const cudaError_t e = launch_c2tc_rows_inv(p, work, y, g, first, s);
+            const cudaError_t e = launch_c2tc_rows_inv(p, work, y, g, first, s, ox);
             if (e != cudaSuccess) return e;
         } else {
-            k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first);
+            k3<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(work, (IO*)y, p.tw.wL, p.B, p.H, Hs, first, ox);
         }
     }
     return cudaGetLastError();
@@ -249,7 +252,7 @@ static cudaError_t c2_spec_go(const fftconv_plan_s& p, const float* k, int Kh, i
         const int g = (int)((p.H - first) < p.group ? (p.H - first) : p.group);
         k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(nullptr, k, Kh, Kw, work, p.tw.wL, p.B, p.H, Hs,
                                                              first);
-        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, nullptr, khat, p.tw.wC, 1, first);
+        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(work, nullptr, khat, p.tw.wC, 1, first, 0);
     }
     return cudaGetLastError();
 }
@@ -262,12 +265,12 @@ static int ilog2_host(int x) {
 
 template <int LOG2LC>
 static cudaError_t c2_fwd_w(const fftconv_plan_s& p, const void* u, const float2* khat, void* y, float2* work,
-                            cudaStream_t s) {
+                            cudaStream_t s, int oy, int ox) {
     const bool bf = p.dtype == FFTCONV_BF16;
     switch (ilog2_host(p.Ws)) {
 #define FFTC_C(LW) \
-    case LW: return bf ? c2_fwd_go<LOG2LC, LW + 1, __nv_bfloat16>(p, u, khat, y, work, s) \
-                       : c2_fwd_go<LOG2LC, LW + 1, float>(p, u, khat, y, work, s);
+    case LW: return bf ? c2_fwd_go<LOG2LC, LW + 1, __nv_bfloat16>(p, u, khat, y, work, s, oy, ox) \
+                       : c2_fwd_go<LOG2LC, LW + 1, float>(p, u, khat, y, work, s, oy, ox);
         FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
 #undef FFTC_C
         default: return cudaErrorInvalidValue;
@@ -319,13 +322,13 @@ bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_
 }
 
 cudaError_t launch_conv2d_fwd(const fftconv_plan_s& p, const void* u, const float2* khat, void* y, float2* work,
-                              cudaStream_t s) {
+                              cudaStream_t s, int oy, int ox) {
     switch (ilog2_host(p.Hs)) {
-        case 4: return c2_fwd_w<5>(p, u, khat, y, work, s);
-        case 5: return c2_fwd_w<6>(p, u, khat, y, work, s);
-        case 6: return c2_fwd_w<7>(p, u, khat, y, work, s);
-        case 7: return c2_fwd_w<8>(p, u, khat, y, work, s);
-        case 8: return c2_fwd_w<9>(p, u, khat, y, work, s);
+        case 4: return c2_fwd_w<5>(p, u, khat, y, work, s, oy, ox);
+        case 5: return c2_fwd_w<6>(p, u, khat, y, work, s, oy, ox);
+        case 6: return c2_fwd_w<7>(p, u, khat, y, work, s, oy, ox);
+        case 7: return c2_fwd_w<8>(p, u, khat, y, work, s, oy, ox);
+        case 8: return c2_fwd_w<9>(p, u, khat, y, work, s, oy, ox);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -50,7 +50,7 @@ constexpr size_t kW1Bytes = 512 * 1024;
 
 template <int LOG2LR, bool BW>
 __global__ void __launch_bounds__(128, 4)
-c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables tb, int npp, int64_t first) {
+c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables tb, int npp, int64_t first, int oy) {
     constexpr int LR = 1 << LOG2LR, Hs = 256;
     __shared__ __align__(128) uint8_t smem[2 * kC2Cols * 512];  // re, im planes: row = column, 256 i
     __shared__ __align__(16) float2 otile[Hs * kC2Cols];        // results, rows i, before the coalesced store
@@ -173,18 +173,21 @@ c2tc_cols(float2* __restrict__ work, const uint4* __restrict__ khat, C2TcTables 
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) cmma2z(acr[u], aci[u], xr[u], xi[u], f16[0], f16[2], f16[1]);
-        // z[i] = Z_even[i] + W_512^{-i} Z_odd[i] (fp32) into the output tile
+        // z[i] = Z_even[i] + W_512^{-i} Z_odd[i] (fp32) into the output tile.  With a
+        // crop offset oy the output row is i - oy, and for i < oy the row 256 + i of
+        // the 512-point inverse: z[i + 256] = Z_even[i] - W_512^{-i} Z_odd[i]
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 w = tz[j][e];
-                const float orr = acr[1][j][e], oi = aci[1][j][e];
+                const int i = 16 * (8 * j + 2 * t + (e & 1)) + g + 8 * (e >> 1);
+                const float sg = i < oy ? -1.f : 1.f;
+                const float orr = sg * acr[1][j][e], oi = sg * aci[1][j][e];
                 // W_512^{-i} = cos + i sin of 2 pi i / 512
                 const float zr = acr[0][j][e] + fmaf(orr, w.x, -oi * w.y);
                 const float zi = aci[0][j][e] + fmaf(oi, w.x, orr * w.y);
-                const int i = 16 * (8 * j + 2 * t + (e & 1)) + g + 8 * (e >> 1);
-                otile[c2_outpos(i, col)] = make_float2(zr, zi);
+                otile[c2_outpos((i - oy) & (Hs - 1), col)] = make_float2(zr, zi);
             }
     }
     __syncthreads();
@@ -356,7 +359,7 @@ c2tc_rows_fwd(const __nv_bfloat16* __restrict__ u, float2* __restrict__ work, C2
 constexpr int kC2RowsI = 8;  // rows per work item
 __global__ void __launch_bounds__(128, 4)
 c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2TcTables tb, int B, int C,
-              int64_t first, int items) {
+              int64_t first, int items, int ox) {
     constexpr int Hs = 256, Ws = 256, LR = 512, RBLK = Hs / kC2RowsI;
     // two staging buffers of planes (row r, 256 k'): [parity][re, im]; then y planes (row r, 256 j) [image]
     __shared__ __align__(128) uint8_t smem[2 * 4 * kC2RowsI * 512 + 2 * kC2RowsI * 512];
@@ -430,14 +433,18 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
             }
 #pragma unroll
             for (int v = 0; v < 2; ++v) cmma2z(acr[v], aci[v], xr[v], xi[v], f16[0], f16[2], f16[1]);
-            // z[j] = Z_even[j] + W_512^{-j} Z_odd[j]: re -> image b0, im -> image b0 + 1
+            // z[j] = Z_even[j] + W_512^{-j} Z_odd[j]: re -> image b0, im -> image b0 + 1;
+            // with a crop offset ox, columns j < ox carry z[256 + j] (the minus sign)
+            // and the store below rotates the columns by ox
             float zr[2][4], zi[2][4];
 #pragma unroll
             for (int n = 0; n < 2; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 w = tz[n][e];
-                    const float orr = acr[1][n][e], oi = aci[1][n][e];
+                    const int jx = 16 * (8 * n + 2 * (lane & 3) + (e & 1)) + (lane >> 2) + 8 * (e >> 1);
+                    const float sg = jx < ox ? -1.f : 1.f;
+                    const float orr = sg * acr[1][n][e], oi = sg * aci[1][n][e];
                     zr[n][e] = acr[0][n][e] + fmaf(orr, w.x, -oi * w.y);
                     zi[n][e] = aci[0][n][e] + fmaf(oi, w.x, orr * w.y);
                 }
@@ -461,7 +468,8 @@ c2tc_rows_inv(const float2* __restrict__ work, __nv_bfloat16* __restrict__ y, C2
             asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
                          : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
                          : "r"(plane_addr(im ? y1p : y0p, r, chunk)));
-            *reinterpret_cast<uint4*>(y + (im ? img1 : img0) + (size_t)(i0 + r) * Ws + chunk * 8) = val;
+            const int oc = (chunk - ox / 8) & (Ws / 8 - 1);  // ox is a multiple of 8
+            *reinterpret_cast<uint4*>(y + (im ? img1 : img0) + (size_t)(i0 + r) * Ws + oc * 8) = val;
         }
         // the next item's wait + barrier orders these reads before the y planes are rewritten
     }
@@ -534,18 +542,18 @@ bool c2tc_tables(std::vector<float2>& out, size_t off[4]) {
 
 template <int LOG2LR>
 static cudaError_t c2tc_go(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
-                           cudaStream_t s) {
+                           cudaStream_t s, int oy) {
     constexpr int LR = 1 << LOG2LR;
     if constexpr (LOG2LR == 9) {
         // all passes on the tensor cores: the bf16 workspace
         if (c2tc_rows_supported(p)) {
             tc::c2tc_cols<LOG2LR, true><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc,
-                                                                                 (p.B + 1) / 2, first);
+                                                                                 (p.B + 1) / 2, first, oy);
             return cudaGetLastError();
         }
     }
     tc::c2tc_cols<LOG2LR, false><<<dim3(LR / tc::kC2Cols, g), 128, 0, s>>>(work, (const uint4*)khat, p.c2tc, (p.B + 1) / 2,
-                                                                     first);
+                                                                     first, oy);
     return cudaGetLastError();
 }
 
@@ -567,7 +575,7 @@ cudaError_t launch_c2tc_rows_fwd(const fftconv_plan_s& p, const void* u, float2*
 }
 
 cudaError_t launch_c2tc_rows_inv(const fftconv_plan_s& p, const float2* work, void* y, int g, int64_t first,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, int ox) {
     static int resident = 0;  // persistent grid, as for the forward row pass
     if (resident == 0) {
         int per_sm = 0, sms = 0, dev = 0;
@@ -578,18 +586,18 @@ cudaError_t launch_c2tc_rows_inv(const fftconv_plan_s& p, const float2* work, vo
     }
     const int items = (256 / tc::kC2RowsI) * g;
     tc::c2tc_rows_inv<<<items < resident ? items : resident, 128, 0, s>>>(work, (__nv_bfloat16*)y, p.c2tc, p.B, p.H,
-                                                                          first, items);
+                                                                          first, items, ox);
     return cudaGetLastError();
 }
 
 cudaError_t launch_c2tc_cols(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
-                             cudaStream_t s) {
+                             cudaStream_t s, int oy) {
     switch (p.Ws) {
-        case 16: return c2tc_go<5>(p, work, khat, g, first, s);
-        case 32: return c2tc_go<6>(p, work, khat, g, first, s);
-        case 64: return c2tc_go<7>(p, work, khat, g, first, s);
-        case 128: return c2tc_go<8>(p, work, khat, g, first, s);
-        case 256: return c2tc_go<9>(p, work, khat, g, first, s);
+        case 16: return c2tc_go<5>(p, work, khat, g, first, s, oy);
+        case 32: return c2tc_go<6>(p, work, khat, g, first, s, oy);
+        case 64: return c2tc_go<7>(p, work, khat, g, first, s, oy);
+        case 128: return c2tc_go<8>(p, work, khat, g, first, s, oy);
+        case 256: return c2tc_go<9>(p, work, khat, g, first, s, oy);
         default: return cudaErrorInvalidValue;
     }
 }

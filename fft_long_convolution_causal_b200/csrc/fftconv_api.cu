@@ -172,11 +172,9 @@ fftconv_status fftconv_plan_create_ex(fftconv_plan_t* out, int B, int H, int64_t
     const int64_t M = int64_t(1) << p->log2M;
     size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0, offT2[2] = {0, 0};
     const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && o.kernel != FFTCONV_KERNEL_SIMT;
-    if (use_tc && (o.kernel == FFTCONV_KERNEL_AUTO || o.kernel == FFTCONV_KERNEL_TCGEN05) &&
-        fftc::t2_supported(p->log2M, p->gated)) {
-        // two-stage tcgen05 kernel, data in tensor memory between the stages (the
-        // fastest measured at 2N = 8192: 79.8 us against 88.8 us for the mma.sync
-        // kernel on the Hyena-style workload, same box)
+    if (use_tc && o.kernel == FFTCONV_KERNEL_TCGEN05 && fftc::t2_supported(p->log2M, p->gated)) {
+        // two-stage tcgen05 kernel, data in tensor memory between the stages: on
+        // request (the mma.sync kernel is still the faster one at 2N = 8192)
         p->path = fftc::PATH_FUSED_TC;
         p->t2 = true;
         fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the SIMT spectrum transform
@@ -571,13 +569,19 @@ fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t p, const float* k, int K
 }
 
 fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work, void* stream) {
+    return fftconv2d_fwd_offset(p, u, khat, y, work, stream, 0, 0);
+}
+
+fftconv_status fftconv2d_fwd_offset(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work,
+                                    void* stream, int oy, int ox) {
     if (!p || p->kind != 2 || !u || !khat || !y || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (oy < 0 || ox < 0 || oy > p->Hs || ox > p->Ws || (oy % 8) || (ox % 8)) return FFTCONV_ERR_INVALID_ARG;
     if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
     if (y == u) return FFTCONV_ERR_INVALID_ARG;
     if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
     if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
     return cuda_status(
-        fftc::launch_conv2d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream));
+        fftc::launch_conv2d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream, oy, ox));
 }
 
 fftconv_status fftconv_plan_set_wait_limit(fftconv_plan_t p, uint32_t probes) {

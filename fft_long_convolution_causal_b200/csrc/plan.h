@@ -156,18 +156,18 @@ cudaError_t launch_multipass_fwd(const fftconv_plan_s& p, const void* u, const v
 bool c2tc_supported(int Hs, int Ws, int dtype);
 bool c2tc_tables(std::vector<float2>& out, size_t off[4]);
 cudaError_t launch_c2tc_cols(const fftconv_plan_s& p, float2* work, const void* khat, int g, int64_t first,
-                             cudaStream_t s);
+                             cudaStream_t s, int oy);
 // the row passes too, for 256 x 256 images
 bool c2tc_rows_supported(const fftconv_plan_s& p);
 cudaError_t launch_c2tc_rows_fwd(const fftconv_plan_s& p, const void* u, float2* work, int g, int64_t first,
                                  cudaStream_t s);
 cudaError_t launch_c2tc_rows_inv(const fftconv_plan_s& p, const float2* work, void* y, int g, int64_t first,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int ox);
 
 // 2-D path (row DFT -> column DFT, product, inverse column DFT -> row iDFT).
 cudaError_t launch_conv2d_spectrum(const fftconv_plan_s& p, const float* k, int Kh, int Kw,
                                    float2* khat, float2* work, cudaStream_t s);
 cudaError_t launch_conv2d_fwd(const fftconv_plan_s& p, const void* u, const float2* khat, void* y,
-                              float2* work, cudaStream_t s);
+                              float2* work, cudaStream_t s, int oy = 0, int ox = 0);
 
 }  // namespace fftc

@@ -157,8 +157,8 @@ FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
  * "fused_tc" (bf16 on-chip, 2N <= 32768, warp-level mma.sync tensor cores),
  * "fused_umma" (the same factorisation on tcgen05 tensor cores, 2N = 4096,
  * or 8192 gated, with FFTCONV_KERNEL_TCGEN05), "fused_t2" (two-stage tcgen05
- * kernel, data held in tensor memory between the stages: the default for
- * ungated bf16 at 2N = 8192), "multipass", "2d", "2d_tc", "partial_chunked",
+ * kernel, data held in tensor memory between the stages, ungated bf16 at
+ * 2N = 8192 with FFTCONV_KERNEL_TCGEN05), "multipass", "2d", "2d_tc", "partial_chunked",
  * "ssm_chunked". */
 FFTCONV_API const char* fftconv_plan_path(fftconv_plan_t plan);
 
@@ -299,6 +299,21 @@ FFTCONV_API fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t plan, const 
  */
 FFTCONV_API fftconv_status fftconv2d_fwd(fftconv_plan_t plan, const void* u, const void* khat, void* y,
                              void* workspace, void* stream);
+
+/*
+ * 2-D forward with a crop offset: y[b,c,i,j] = full[i + oy][j + ox], the
+ * window [oy, oy + Hs) x [ox, ox + Ws) of the full (2Hs - 1) x (2Ws - 1)
+ * linear convolution full[r][s] = sum_{p,q} k[c,p,q] u[b,c,r-p,s-q] (indices
+ * inside both arrays).  (0, 0) is fftconv2d_fwd's first-quadrant crop;
+ * (Hs/2, Ws/2) the centred reading of a kernel anchored at its middle (the
+ * pages' zero-padded convolution does not say which window).  0 <= oy <= Hs,
+ * 0 <= ox <= Ws, both multiples of 8 (else FFTCONV_ERR_INVALID_ARG).  The
+ * transform of length 2Hs x 2Ws holds the full convolution without
+ * wrap-around, so only the last inverse passes change: they keep rows
+ * oy.. and columns ox.. instead of 0...
+ */
+FFTCONV_API fftconv_status fftconv2d_fwd_offset(fftconv_plan_t plan, const void* u, const void* khat, void* y,
+                                                void* workspace, void* stream, int oy, int ox);
 
 /*
  * Conjugate spectrum: khat_conj <- conj(khat) in the plan's layout, the

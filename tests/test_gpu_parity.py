@@ -58,8 +58,6 @@ def test_fused_full_compare(N, dtype):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
     y, plan = run_1d(wl)
     want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 16384) else "fused"
-    if dtype == "bf16" and N == 4096:
-        want = "fused_t2"  # the two-stage tcgen05 kernel is the default at 2N = 8192
     assert plan.path == want
     assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}", scale=row_scale_1d(wl))
 
@@ -330,6 +328,24 @@ def test_conv2d_tensor_core_columns(Ws, Kh, Kw):
     assert binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, "bf16").path == "2d_tc"
     y = run_2d(wl)
     assert_close(y, oracle.causal_conv2d(wl.u, wl.k), "bf16", f"2d tc 256x{Ws} k{Kh}x{Kw}", scale=row_scale_2d(wl))
+
+
+@pytest.mark.parametrize("Hs,Ws,dtype,Kh,Kw", [(16, 16, "f32", 16, 16), (64, 32, "bf16", 40, 32),
+                                              (256, 256, "bf16", 256, 256), (256, 64, "bf16", 100, 64)])
+@pytest.mark.parametrize("frac", [(0.5, 0.5), (1.0, 1.0), (0.5, 0.0), (0.0, 0.25)])
+def test_conv2d_crop_offset(Hs, Ws, dtype, Kh, Kw, frac):
+    """Crop windows other than the first quadrant (fftconv2d_fwd_offset): the
+    centred reading (Hs/2, Ws/2), the far window, and one-sided shifts, on
+    the SIMT passes and on the tensor-core passes (256 rows, bf16); every
+    output against the oracle's window of the full linear convolution."""
+    oy, ox = 8 * int(Hs * frac[0] / 8), 8 * int(Ws * frac[1] / 8)  # offsets are multiples of 8
+    from fft_long_convolution_causal_b200 import binding
+    wl = wlmod.make_2d(3, 2, Hs, Ws, dtype=dtype, seed=Hs + Ws + oy + ox, Kh=Kh, Kw=Kw, sigma=Hs / 4)
+    plan = binding.Plan2D(wl.B, wl.C, wl.Hs, wl.Ws, dtype)
+    khat = plan.kernel_spectrum(torch.from_numpy(wl.k).cuda())
+    y = to_host(plan.fwd(to_dev(wl.u, dtype), khat, offset=(oy, ox)))
+    want = oracle.causal_conv2d_offset(wl.u, wl.k, oy, ox)
+    assert_close(y, want, dtype, f"2d offset {Hs}x{Ws} {dtype} ({oy},{ox}) path={plan.path}", scale=row_scale_2d(wl))
 
 
 def test_conv2d_named_sampled():
