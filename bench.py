@@ -33,6 +33,11 @@ output copy.
 
 cpu_baseline (rank 0, N=1): the CPU fp64 oracle, as it stands, on a bounded
 uniform sample of the same workload's outputs.
+
+variants (N=1): the skipped-work forms on the long workload's shape, each
+timed against the dense multi-pass plan on the same inputs (partial
+convolution, frequency-sparse filter, state-space filters with chunked state
+passing).
 """
 import argparse
 import hashlib
@@ -84,6 +89,8 @@ def parse():
                     help="kernel family the plans may use (the library's choice by default)")
     ap.add_argument("--no-per-config", action="store_true", help="headline workload only")
     ap.add_argument("--per-config-steps", type=int, default=10)
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the partial / frequency-sparse / state-passing comparisons")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json's entry for --config from an ncu raw CSV and exit")
     ap.add_argument("--traffic-command", default="", help="the capture command, stored with the record")
@@ -511,6 +518,92 @@ def measure(wl, args, torch, steps, warmup, pg=None, world=1, clocks=False, e2e=
     return res
 
 
+def _time_fn(fn, steps, warmup, torch, flush):
+    """Mean device ms of fn() over `steps` calls, L2 flushed between calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
+def variants(torch, steps=5):
+    """Skipped-work variants of the long workload's shape (B=2, H=64, N=2^20,
+    fp32), each timed against the dense multi-pass plan on the same inputs:
+    a partial convolution (4096-tap filters, chunked on chip), a
+    frequency-sparse filter (half of the outer-digit pairs dropped) and the
+    state-space filters with chunked state passing (d = 16)."""
+    from fft_long_convolution_causal_b200 import binding
+    B, H, N = 2, 64, 1 << 20
+    dev = torch.device("cuda")
+    g = torch.Generator(device="cpu").manual_seed(7)
+    u = torch.randn(B, H, N, generator=g).to(dev)
+    D = torch.randn(H, generator=g).to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    out = {}
+
+    def pair(name, fn_variant, fn_dense, note):
+        tv = _time_fn(fn_variant, steps, 3, torch, flush)
+        td = _time_fn(fn_dense, steps, 3, torch, flush)
+        out[name] = {"ms_variant": round(tv, 4), "ms_dense": round(td, 4), "speedup": round(td / tv, 3),
+                     "note": note}
+
+    dense = binding.Plan(B, H, N, "f32")
+    ws = dense.new_workspace()
+    y = torch.empty_like(u)
+    # partial: 4096 taps
+    L = 4096
+    k = (torch.randn(H, L, generator=g) * torch.exp(-1e-3 * torch.arange(L, dtype=torch.float32))).to(dev)
+    part = binding.PartialPlan(B, H, N, "f32", L_max=L)
+    kp = part.kernel_spectrum(k)
+    kd = dense.kernel_spectrum(k)
+    pair("partial_l4096", lambda: part.fwd(u, kp, D=D, y=y), lambda: dense.fwd(u, kd, D=D, y=y, workspace=ws),
+         "filters of 4096 taps: chunked partial plan vs the dense 2N-point multi-pass plan")
+    del part, kp
+    # frequency-sparse: half of the outer-digit pairs dropped (Hermitian-symmetric mask)
+    kfull = (torch.randn(H, N, generator=g) * torch.exp(-1e-5 * torch.arange(N, dtype=torch.float32))).to(dev)
+    sp = binding.Plan(B, H, N, "f32")
+    ks = sp.kernel_spectrum(kfull)
+    G = sp.spectrum_blocks
+    keep = np.ones(G, bool)
+    for j in range(1, G // 2 + 1):
+        if j % 2 == 1:
+            keep[j] = keep[(G - j) % G] = False
+    sp.sparsify(ks, keep)
+    kd = dense.kernel_spectrum(kfull, khat=kd)
+    pair("freq_sparse_half", lambda: sp.fwd(u, ks, D=D, y=y, workspace=ws),
+         lambda: dense.fwd(u, kd, D=D, y=y, workspace=ws),
+         f"{int((~keep).sum())} of {G} outer-digit blocks dropped vs the same plan dense")
+    del sp, ks
+    # chunked state passing: d = 16 poles per channel
+    d = 16
+    mag = 1.0 - torch.rand(H, d, generator=g) * 1e-3
+    ang = torch.rand(H, d, generator=g) * 0.1
+    lam = torch.polar(mag, ang)
+    c = torch.complex(torch.randn(H, d, generator=g), torch.randn(H, d, generator=g)) * 0.1
+    ssm = binding.SSMPlan(B, H, N, "f32", d_state=d, chunk=8192)
+    kss = ssm.set_filters(lam, c)
+    tt = torch.arange(N, dtype=torch.float64, device=dev)
+    kmat = torch.zeros(H, N, dtype=torch.float64, device=dev)
+    lam64, c64 = lam.to(torch.complex128).to(dev), c.to(torch.complex128).to(dev)
+    for j in range(d):  # the same filters materialised (fp64) for the dense plan
+        kmat += (c64[:, j:j + 1] * torch.exp(tt[None, :] * torch.log(lam64[:, j:j + 1]))).real
+    kd = dense.kernel_spectrum(kmat.to(torch.float32), khat=kd)
+    del kmat, tt
+    pair("ssm_chunked_d16", lambda: ssm.fwd(u, kss, D=D, y=y), lambda: dense.fwd(u, kd, D=D, y=y, workspace=ws),
+         "diagonal state-space filters, chunks of 8192 with the state passed vs the dense plan on the same filters")
+    del ssm, kss, dense, ws, u, y
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     if args.record_traffic:
@@ -545,6 +638,9 @@ def main():
                           config_name=name)
             del w2
             per_config[name] = res
+    var = None
+    if world == 1 and not args.no_variants and not args.channels:
+        var = variants(torch)
     if pg:
         pg.barrier()
         pg.destroy_process_group()
@@ -559,6 +655,8 @@ def main():
             "ms_per_step_min": head["ms_per_step_min"], "ms_per_step_median": head["ms_per_step_median"]}
     if per_config is not None:
         line["per_config"] = per_config
+    if var is not None:
+        line["variants"] = var
     print(json.dumps(line))
     return 0
 

@@ -136,8 +136,10 @@ fused_spectrum_simt(const float* __restrict__ k, int L, float2* __restrict__ kha
 }
 
 // The spectrum in the layout of the two-stage tensor-core kernel (2N = 8192 =
-// 128 x 64, frequency k = k_p + 128 c): per channel, row k_p and column half
-// c / 32, 32 words: 16 bf16 pairs of Re (c, c + 1) then 16 of -Im, scaled 1/M.
+// 128 x 64, frequency k = k_p + 128 c): per channel, row k_p and column group
+// g = c / 16, 16 words: 8 bf16 pairs of Re (c, c + 1) then 8 of -Im, scaled
+// 1/M; stored as 16-byte quads [h][g][word / 4][k_p], so that consecutive rows
+// k_p of one quad are adjacent.
 __global__ void __launch_bounds__(FusedG<13>::T)
 t2_spectrum_simt(const float* __restrict__ k, int L, uint16_t* __restrict__ khat, const float2* __restrict__ tw) {
     using G = FusedG<13>;
@@ -156,10 +158,12 @@ t2_spectrum_simt(const float* __restrict__ k, int L, uint16_t* __restrict__ khat
     uint16_t* __restrict__ out = khat + (size_t)h * M * 2;
     stage<G, NS - 1, false, RL, RL, false>(tid, tw, lds, [&](int i, int, float2 z) {
         const int kp = i & 127, c = i >> 7;
-        const size_t word = ((size_t)kp * 2 + (c >> 5)) * 32 + ((c & 31) >> 1);
+        // 32-bit word index of word w (< 16) of group c / 16 of row kp
+        auto word = [&](int w) { return ((size_t)((c >> 4) * 4 + (w >> 2)) * 128 + kp) * 4 + (w & 3); };
+        const int w = (c & 15) >> 1;
         const __nv_bfloat16 re = __float2bfloat16_rn(z.x * (1.0f / M)), nim = __float2bfloat16_rn(-z.y * (1.0f / M));
-        out[2 * word + (c & 1)] = *reinterpret_cast<const uint16_t*>(&re);
-        out[2 * (word + 16) + (c & 1)] = *reinterpret_cast<const uint16_t*>(&nim);
+        out[2 * word(w) + (c & 1)] = *reinterpret_cast<const uint16_t*>(&re);
+        out[2 * word(w + 8) + (c & 1)] = *reinterpret_cast<const uint16_t*>(&nim);
     });
 }
 

@@ -172,9 +172,11 @@ fftconv_status fftconv_plan_create_ex(fftconv_plan_t* out, int B, int H, int64_t
     const int64_t M = int64_t(1) << p->log2M;
     size_t offL = 0, offC = 0, offLo = 0, offHi = 0, offTc[7] = {0, 0, 0, 0, 0, 0, 0}, offU = 0, offT2[2] = {0, 0};
     const bool use_tc = dtype == FFTCONV_BF16 && fftc::tc_supported(p->log2M) && o.kernel != FFTCONV_KERNEL_SIMT;
-    if (use_tc && o.kernel == FFTCONV_KERNEL_TCGEN05 && fftc::t2_supported(p->log2M, p->gated)) {
-        // two-stage tcgen05 kernel, data in tensor memory between the stages: on
-        // request (the mma.sync kernel is still the faster one at 2N = 8192)
+    if (use_tc && (o.kernel == FFTCONV_KERNEL_AUTO || o.kernel == FFTCONV_KERNEL_TCGEN05) &&
+        fftc::t2_supported(p->log2M, p->gated)) {
+        // two-stage tcgen05 kernel, data in tensor memory between the stages (the
+        // fastest measured at 2N = 8192: 72.4 us against 88.8-97 us for the
+        // mma.sync kernel on the Hyena-style workload)
         p->path = fftc::PATH_FUSED_TC;
         p->t2 = true;
         fftc::fused_tables(p->log2M, host, &offL);  // stage tables of the SIMT spectrum transform

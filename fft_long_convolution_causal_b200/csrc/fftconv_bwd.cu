@@ -25,13 +25,14 @@ namespace fftc {
 
 // flip the sign of the imaginary parts of a spectrum stored as 32-bit words:
 // kind 0: fp32 complex (odd words); 1: bf16 pairs, odd words Im (fragment
-// order); 2: bf16 pairs, words 16..31 of every 32 Im (two-stage layout)
+// order); 2: bf16 pairs in 16-byte quads [h][g][j][k_p], quads j = 2, 3 Im
+// (two-stage layout)
 __global__ void conj_words(const uint32_t* __restrict__ in, uint32_t* __restrict__ out, size_t n, int kind) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         uint32_t x = in[i];
         if (kind == 0 && (i & 1)) x ^= 0x80000000u;
         if (kind == 1 && (i & 1)) x ^= 0x80008000u;
-        if (kind == 2 && (i & 16)) x ^= 0x80008000u;
+        if (kind == 2 && ((i >> 9) & 2)) x ^= 0x80008000u;
         out[i] = x;
     }
 }

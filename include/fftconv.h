@@ -157,8 +157,8 @@ FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
  * "fused_tc" (bf16 on-chip, 2N <= 32768, warp-level mma.sync tensor cores),
  * "fused_umma" (the same factorisation on tcgen05 tensor cores, 2N = 4096,
  * or 8192 gated, with FFTCONV_KERNEL_TCGEN05), "fused_t2" (two-stage tcgen05
- * kernel, data held in tensor memory between the stages, ungated bf16 at
- * 2N = 8192 with FFTCONV_KERNEL_TCGEN05), "multipass", "2d", "2d_tc", "partial_chunked",
+ * kernel, data held in tensor memory between the stages: the default for
+ * ungated bf16 at 2N = 8192), "multipass", "2d", "2d_tc", "partial_chunked",
  * "ssm_chunked". */
 FFTCONV_API const char* fftconv_plan_path(fftconv_plan_t plan);
 

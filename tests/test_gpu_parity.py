@@ -58,6 +58,8 @@ def test_fused_full_compare(N, dtype):
     wl = wlmod.make_1d(3, 2, N, dtype=dtype, gated=False, seed=N, kernel="decay")
     y, plan = run_1d(wl)
     want = "fused_tc" if (dtype == "bf16" and 2048 <= N <= 16384) else "fused"
+    if dtype == "bf16" and N == 4096:
+        want = "fused_t2"  # the two-stage tcgen05 kernel is the default at 2N = 8192
     assert plan.path == want
     assert_close(y, oracle_full(wl), dtype, f"fused N={N} {dtype}", scale=row_scale_1d(wl))
 
@@ -116,10 +118,9 @@ def test_tcgen05_path(N, B, gated, with_D, L):
 @pytest.mark.parametrize("B,H,with_D,L", [(1, 3, True, None), (3, 4, True, None), (6, 5, False, None),
                                          (7, 2, True, 1000), (4, 300, True, None), (2, 1, False, 1)])
 def test_two_stage_kernel(B, H, with_D, L):
-    """The two-stage tcgen05 kernel (2N = 8192): units of two row pairs with
-    a missing last row (odd B), single-pair units (B = 6: pairs 0-1 and 2),
-    many units per CTA (H = 300), partial kernels, no skip term; every output
-    compared."""
+    """The two-stage tcgen05 kernel (2N = 8192): a missing last row (odd B),
+    CTAs whose second slot has no pair (few pairs), many pairs per slot
+    (H = 300), partial kernels, no skip term; every output compared."""
     wl = wlmod.make_1d(B, H, 4096, dtype="bf16", gated=False, seed=17 * B + H, with_D=with_D, L=L)
     y, plan = run_1d(wl, kernel="tcgen05")
     assert plan.path == "fused_t2"
