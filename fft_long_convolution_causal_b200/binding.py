@@ -67,6 +67,9 @@ _SIGS = {
     "fftconv2d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
     "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv2d_fwd_offset": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int]),
+    "fftconv2d_dynamic_plan_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "fftconv2d_fwd_dynamic": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
     "fftconv_fwd_static_workspace": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv_static_workspace_bytes": (ctypes.c_size_t, []),
     "fftconv_device_status": (ctypes.c_int, [_vp, _vp]),
@@ -366,6 +369,36 @@ class Plan2D(_PlanBase):
         oy, ox = (int(offset[0]), int(offset[1]))
         _check(self.lib.fftconv2d_fwd_offset(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace),
                                              _stream(stream), oy, ox), "fftconv2d_fwd_offset")
+        return y
+
+
+class Plan2DDynamic(_PlanBase):
+    """2-D plan with one filter per image: fftconv2d_dynamic_plan_create(B, C, Hs, Ws, dtype)."""
+
+    def __init__(self, B: int, C: int, Hs: int, Ws: int, dtype: str = "bf16"):
+        self.lib = load_library()
+        self.B, self.C, self.Hs, self.Ws, self.dtype = B, C, Hs, Ws, dtype
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv2d_dynamic_plan_create(ctypes.byref(h), B, C, Hs, Ws, DTYPES[dtype]),
+               "fftconv2d_dynamic_plan_create")
+        self._handle = h
+        self._workspace = None
+
+    def fwd(self, u: torch.Tensor, k: torch.Tensor, y: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """y[b, c] = first-quadrant crop of u[b, c] convolved with k[b, c] ([B, C, Kh, Kw] fp32)."""
+        shape = (self.B, self.C, self.Hs, self.Ws)
+        _need(u, "u", shape, self.torch_dtype)
+        if k.dim() != 4:
+            raise ValueError("k must be [B, C, Kh, Kw]")
+        _need(k, "k", (self.B, self.C, k.shape[2], k.shape[3]), torch.float32)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        _need(y, "y", shape, self.torch_dtype)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv2d_fwd_dynamic(self._handle, _ptr(u), _ptr(k), k.shape[2], k.shape[3], _ptr(y),
+                                              _ptr(workspace), _stream(stream)), "fftconv2d_fwd_dynamic")
         return y
 
 

@@ -570,6 +570,40 @@ fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t p, const float* k, int K
     return cuda_status(e);
 }
 
+fftconv_status fftconv2d_dynamic_plan_create(fftconv_plan_t* out, int B, int C, int Hs, int Ws,
+                                             fftconv_dtype dtype) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || C < 1 || (int64_t)B * C > (int64_t)1 << 30) return FFTCONV_ERR_INVALID_ARG;
+    fftconv_plan_t p = nullptr;
+    fftconv_status st = fftconv2d_plan_create_ex(&p, 1, B * C, Hs, Ws, dtype, nullptr);
+    if (st != FFTCONV_OK) return st;
+    p->dyn2d = true;
+    p->dynB = B;
+    p->dynC = C;
+    // workspace: [the images' spectra][the passes' workspace]
+    p->dyn_spectrum_offset = (p->spectrum_bytes + 255) & ~size_t(255);
+    p->workspace_bytes += p->dyn_spectrum_offset;
+    *out = p;
+    return FFTCONV_OK;
+}
+
+fftconv_status fftconv2d_fwd_dynamic(fftconv_plan_t p, const void* u, const float* k, int Kh, int Kw, void* y,
+                                     void* work, void* stream) {
+    if (!p || p->kind != 2 || !p->dyn2d || !u || !k || !y || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (Kh < 1 || Kw < 1 || Kh > p->Hs || Kw > p->Ws) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(k) || !aligned16(y) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (y == u) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    float2* khat = (float2*)work;
+    float2* rest = (float2*)((uint8_t*)work + p->dyn_spectrum_offset);
+    // every image's filter is a channel of the single-image batch: its spectrum, then the forward
+    cudaError_t e = fftc::launch_conv2d_spectrum(*p, k, Kh, Kw, khat, rest, s);
+    if (e == cudaSuccess) e = fftc::launch_conv2d_fwd(*p, u, khat, y, rest, s, 0, 0);
+    return cuda_status(e);
+}
+
 fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work, void* stream) {
     return fftconv2d_fwd_offset(p, u, khat, y, work, stream, 0, 0);
 }

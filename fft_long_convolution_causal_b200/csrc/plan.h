@@ -70,6 +70,12 @@ struct fftconv_plan_s {
     const void* umma_b = nullptr;   // tcgen05 path: B operand images of the DFT matrices
     int* d_err = nullptr;           // device status word: nonzero after a timed-out device wait
     bool tc2d = false;              // 2-D: column pass on the tensor cores (bf16, Hs = 256)
+    // 2-D plans with one filter per image: the images run as channels of a
+    // single-image batch (B = 1, C = B C of the caller), their spectra in the
+    // head of the workspace
+    bool dyn2d = false;
+    int dynB = 0, dynC = 0;
+    size_t dyn_spectrum_offset = 0;
     fftc::C2TcTables c2tc;
     bool spectrum_ready = false;
     int device = 0;

@@ -316,6 +316,26 @@ FFTCONV_API fftconv_status fftconv2d_fwd_offset(fftconv_plan_t plan, const void*
                                                 void* workspace, void* stream, int oy, int ox);
 
 /*
+ * 2-D forward with one filter per image (input-dependent kernels, "Native
+ * Multi-Dimensional Subquadratic Operators via Input Dependent Long
+ * Convolutions", abstract):
+ *     y[b,c,i,j] = sum_{p<=i, q<=j} k[b,c,p,q] u[b,c,i-p,j-q]
+ * (fftconv2d_fwd's crop).  Plans from fftconv2d_dynamic_plan_create (B, C,
+ * Hs, Ws, dtype as fftconv2d_plan_create); k is [B][C][Kh][Kw] fp32 on the
+ * device, 1 <= Kh <= Hs, 1 <= Kw <= Ws, transformed inside the call (no
+ * cached spectrum: fftconv2d_kernel_spectrum is not needed).  The images run
+ * as the channels of a single-image batch, so each transform carries one
+ * image (half of fftconv2d_fwd's packing of two).  workspace: device,
+ * fftconv_workspace_bytes(plan) bytes (the images' spectra, then the passes'
+ * workspace), 16-byte aligned.  FFTCONV_ERR_INVALID_ARG for plans of any
+ * other kind, or when the current device is not the plan's.
+ */
+FFTCONV_API fftconv_status fftconv2d_dynamic_plan_create(fftconv_plan_t* plan, int B, int C, int Hs, int Ws,
+                                                         fftconv_dtype dtype);
+FFTCONV_API fftconv_status fftconv2d_fwd_dynamic(fftconv_plan_t plan, const void* u, const float* k, int Kh, int Kw,
+                                                 void* y, void* workspace, void* stream);
+
+/*
  * Conjugate spectrum: khat_conj <- conj(khat) in the plan's layout, the
  * spectrum of the correlation with k (the backward pass's filter).  khat is
  * the output of fftconv_kernel_spectrum on this plan; khat_conj is a buffer of

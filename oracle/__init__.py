@@ -212,6 +212,30 @@ def causal_conv2d(u, k) -> np.ndarray:
     return y
 
 
+def causal_conv2d_dynamic(u, k) -> np.ndarray:
+    """fp64 2-D oracle with one filter per image ("Native Multi-Dimensional
+    Subquadratic Operators via Input Dependent Long Convolutions", abstract):
+    y[b, c] = first-quadrant crop of u[b, c] convolved with k[b, c]; k is
+    [B][C][Kh][Kw].  Every image is its own channel of a one-image batch."""
+    u = np.asarray(u, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    if u.ndim != 4 or k.ndim != 4 or k.shape[:2] != u.shape[:2]:
+        raise ValueError("u must be [B, C, Hs, Ws] and k [B, C, Kh, Kw]")
+    B, C, Hs, Ws = u.shape
+    y = causal_conv2d(u.reshape(1, B * C, Hs, Ws), k.reshape(B * C, k.shape[2], k.shape[3]))
+    return y.reshape(B, C, Hs, Ws)
+
+
+def causal_conv2d_dynamic_points(u, k, b_idx, c_idx, i_idx, j_idx) -> np.ndarray:
+    """causal_conv2d_dynamic at sampled pixels."""
+    u = np.asarray(u, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    B, C, Hs, Ws = u.shape
+    flat = np.asarray(b_idx, dtype=np.int64) * C + np.asarray(c_idx, dtype=np.int64)
+    return causal_conv2d_points(u.reshape(1, B * C, Hs, Ws), k.reshape(B * C, k.shape[2], k.shape[3]),
+                                np.zeros_like(flat), flat, i_idx, j_idx)
+
+
 def causal_conv2d_offset(u, k, oy, ox) -> np.ndarray:
     """fp64 2-D oracle, crop window [oy, oy+Hs) x [ox, ox+Ws) of the full linear
     convolution (0, 0: the first-quadrant crop; Hs/2, Ws/2: the centred one)."""

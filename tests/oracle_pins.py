@@ -406,6 +406,30 @@ def check_freq_sparse():
     assert np.allclose(y2, 2.0 * y, rtol=1e-12, atol=1e-12)
 
 
+def check_conv2d_dynamic():
+    """Per-image 2-D filters: filters equal across the batch give the
+    shared-filter oracle; every image is scipy.signal.convolve2d's full linear
+    convolution of its own image and filter, cropped to the first quadrant;
+    the sampled entry point matches the full one."""
+    from scipy.signal import convolve2d
+    r = _rng(68)
+    B, C, Hs, Ws, Kh, Kw = 3, 2, 8, 16, 5, 7
+    u = r.standard_normal((B, C, Hs, Ws))
+    kc = r.standard_normal((C, Kh, Kw))
+    same = oracle.causal_conv2d_dynamic(u, np.broadcast_to(kc, (B, C, Kh, Kw)))
+    assert np.allclose(same, oracle.causal_conv2d(u, kc), rtol=1e-12, atol=1e-12)
+    k = r.standard_normal((B, C, Kh, Kw))
+    y = oracle.causal_conv2d_dynamic(u, k)
+    for b in range(B):
+        for c in range(C):
+            want = convolve2d(u[b, c], k[b, c])[:Hs, :Ws]
+            assert np.allclose(y[b, c], want, rtol=1e-11, atol=1e-11), (b, c)
+    bi, ci = np.array([0, 2, 1, 2]), np.array([1, 0, 1, 1])
+    ii, jj = np.array([0, 7, 3, 5]), np.array([15, 0, 9, 4])
+    pts = oracle.causal_conv2d_dynamic_points(u, k, bi, ci, ii, jj)
+    assert np.allclose(pts, y[bi, ci, ii, jj], rtol=1e-12, atol=1e-12)
+
+
 def check_conv2d_offset():
     """Crop offsets: (0, 0) is the first-quadrant oracle; any offset is the
     window of scipy.signal.convolve2d's full linear convolution."""
@@ -430,5 +454,5 @@ ALL_CHECKS = [
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
     check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
-    check_ssm_kernel, check_freq_sparse, check_conv2d_offset,
+    check_ssm_kernel, check_freq_sparse, check_conv2d_offset, check_conv2d_dynamic,
 ]

@@ -1,5 +1,6 @@
 """GPU parity of the forward with input-dependent filters (one per batch row,
-transformed in the same launch) through the C ABI against the fp64 oracle."""
+transformed in the same launch; one per 2-D image, transformed in the same
+call) through the C ABI against the fp64 oracle."""
 import numpy as np
 import pytest
 import torch
@@ -75,3 +76,78 @@ def test_dynamic_refuses_long_sequences():
     with pytest.raises(binding.FFTConvError) as e:
         plan.fwd_dynamic(u, torch.zeros(2, 1, 8192, device="cuda"))
     assert e.value.status == 2
+
+
+def _filters_2d(B, C, Kh, Kw, sigma, seed):
+    """Per-image filters k[b,c,p,q] = N(0,1) exp(-(p^2 + q^2) / (2 sigma^2))."""
+    r = np.random.default_rng(seed)
+    p = np.arange(Kh, dtype=np.float64)[:, None]
+    q = np.arange(Kw, dtype=np.float64)[None, :]
+    win = np.exp(-(p * p + q * q) / (2.0 * sigma * sigma))
+    return (r.standard_normal((B, C, Kh, Kw)) * win[None, None]).astype(np.float32)
+
+
+def _scale_2d(u, k, b_idx=None, c_idx=None):
+    """Per-image scale RMS(u[b, c]) * ||k[b, c]|| (the 2-D analogue of the row scale)."""
+    s = np.sqrt(np.mean(u.astype(np.float64) ** 2, axis=(2, 3))) * np.sqrt(
+        np.sum(k.astype(np.float64) ** 2, axis=(2, 3)))
+    if b_idx is None:
+        return np.broadcast_to(s[:, :, None, None], u.shape)
+    return s[b_idx, c_idx]
+
+
+@pytest.mark.parametrize("B,C,Hs,Ws,dtype,Kh,Kw", [
+    (3, 2, 16, 16, "f32", 16, 16), (2, 3, 64, 32, "bf16", 40, 9), (1, 2, 128, 128, "f32", 128, 128),
+    (3, 2, 256, 64, "bf16", 100, 64), (2, 2, 256, 256, "bf16", 256, 256)])
+def test_dynamic_2d_full_compare(B, C, Hs, Ws, dtype, Kh, Kw):
+    """One filter per image (fftconv2d_fwd_dynamic): the SIMT passes and the
+    tensor-core passes (256 rows, bf16), odd and even B; every output
+    compared with the oracle's per-image convolution."""
+    from fft_long_convolution_causal_b200 import binding
+    wl = wlmod.make_2d(B, C, Hs, Ws, dtype=dtype, seed=Hs + 3 * Ws + B, sigma=Hs / 4)
+    k = _filters_2d(B, C, Kh, Kw, Hs / 4, seed=Hs * 7 + C)
+    plan = binding.Plan2DDynamic(B, C, Hs, Ws, dtype)
+    y = to_host(plan.fwd(to_dev(wl.u, dtype), torch.from_numpy(k).cuda()))
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    want = oracle.causal_conv2d_dynamic(wl.u, k)
+    assert_close(y, want, dtype, f"2d dynamic B={B} C={C} {Hs}x{Ws} {dtype} k{Kh}x{Kw}", scale=_scale_2d(wl.u, k))
+
+
+def test_dynamic_2d_filters_differ_per_image():
+    """Two images of one channel with different filters: each output follows
+    its own filter (a path that shared one filter per channel would fail)."""
+    from fft_long_convolution_causal_b200 import binding
+    wl = wlmod.make_2d(2, 1, 64, 64, dtype="f32", seed=5, sigma=16.0)
+    k = _filters_2d(2, 1, 8, 8, 16.0, seed=6)
+    k[1] *= -3.0
+    y = to_host(binding.Plan2DDynamic(2, 1, 64, 64, "f32").fwd(to_dev(wl.u, "f32"), torch.from_numpy(k).cuda()))
+    want = oracle.causal_conv2d_dynamic(wl.u, k)
+    assert_close(y, want, "f32", "2d dynamic, different filters", scale=_scale_2d(wl.u, k))
+    shared = oracle.causal_conv2d(wl.u, k[0])
+    assert np.max(np.abs(y[1] - shared[1])) > 1.0
+
+
+def test_dynamic_2d_sampled_at_named_size():
+    """Per-image filters at the 2-D workload's image size (256 x 256 bf16,
+    full-size filters), 2048 sampled pixels against the oracle."""
+    from fft_long_convolution_causal_b200 import binding
+    B, C = 4, 6
+    wl = wlmod.make_2d(B, C, 256, 256, dtype="bf16", seed=41, sigma=64.0)
+    k = _filters_2d(B, C, 256, 256, 64.0, seed=42)
+    y = to_host(binding.Plan2DDynamic(B, C, 256, 256, "bf16").fwd(to_dev(wl.u, "bf16"), torch.from_numpy(k).cuda()))
+    idx = wlmod.sample_points_2d(B, C, 256, 256, 2048, seed=43)
+    ref = oracle.causal_conv2d_dynamic_points(wl.u, k, *idx)
+    assert_close(y[idx], ref, "bf16", "2d dynamic 256x256 sampled", scale=_scale_2d(wl.u, k, idx[0], idx[1]))
+
+
+def test_dynamic_2d_rejects_other_plans():
+    from fft_long_convolution_causal_b200 import binding
+    plan = binding.Plan2D(2, 2, 16, 16, "f32")
+    lib = binding.load_library()
+    u = torch.zeros(2, 2, 16, 16, device="cuda")
+    k = torch.zeros(2, 2, 4, 4, device="cuda")
+    ws = plan.new_workspace()
+    st = lib.fftconv2d_fwd_dynamic(plan._handle, u.data_ptr(), k.data_ptr(), 4, 4, torch.empty_like(u).data_ptr(),
+                                   ws.data_ptr() if ws is not None else None, None)
+    assert st == 1  # FFTCONV_ERR_INVALID_ARG: not a plan with one filter per image
