@@ -45,6 +45,8 @@ def bind(path):
     lib.oracle_causal_conv2d.argtypes = [_i64] * 6 + [_f64p] * 3
     lib.oracle_causal_conv2d_offset.argtypes = [_i64] * 8 + [_f64p] * 3
     lib.oracle_causal_conv2d_points.argtypes = [_i64] * 6 + [_f64p] * 2 + [_i64] + [_i64p] * 4 + [_f64p]
+    lib.oracle_causal_conv3d.argtypes = [_i64] * 8 + [_f64p] * 3
+    lib.oracle_causal_conv3d_points.argtypes = [_i64] * 8 + [_f64p] * 2 + [_i64] + [_i64p] * 5 + [_f64p]
     lib.oracle_dft_causal_conv1d.argtypes = [_i64, _i64, _f64p, _f64p, _f64p]
     lib.oracle_dft_causal_conv2d.argtypes = [_i64] * 4 + [_f64p] * 3
     return lib
@@ -210,6 +212,43 @@ def causal_conv2d(u, k) -> np.ndarray:
     y = np.empty_like(u)
     _load().oracle_causal_conv2d(B, C, Hs, Ws, k.shape[1], k.shape[2], _p(u), _p(k), _p(y))
     return y
+
+
+def _check_3d(u, k):
+    u = _f64(u)
+    k = _f64(k)
+    if u.ndim != 5 or k.ndim != 4:
+        raise ValueError("u must be [B,C,Dd,Hs,Ws] and k [C,Kd,Kh,Kw]")
+    B, C, Dd, Hs, Ws = u.shape
+    if k.shape[0] != C or not (1 <= k.shape[1] <= Dd and 1 <= k.shape[2] <= Hs and 1 <= k.shape[3] <= Ws):
+        raise ValueError("k must be [C,Kd,Kh,Kw] with Kd <= Dd, Kh <= Hs, Kw <= Ws")
+    return u, k
+
+
+def causal_conv3d(u, k) -> np.ndarray:
+    """Full fp64 3-D oracle: the first-octant crop of the zero-padded linear
+    convolution (the 3-D analogue of [:N]), by direct sums."""
+    u, k = _check_3d(u, k)
+    B, C, Dd, Hs, Ws = u.shape
+    y = np.empty_like(u)
+    _load().oracle_causal_conv3d(B, C, Dd, Hs, Ws, k.shape[1], k.shape[2], k.shape[3], _p(u), _p(k), _p(y))
+    return y
+
+
+def causal_conv3d_points(u, k, b_idx, c_idx, d_idx, i_idx, j_idx) -> np.ndarray:
+    """fp64 3-D oracle at sampled voxels."""
+    u, k = _check_3d(u, k)
+    B, C, Dd, Hs, Ws = u.shape
+    idx = [np.ascontiguousarray(a, dtype=np.int64) for a in (b_idx, c_idx, d_idx, i_idx, j_idx)]
+    n = idx[0].size
+    if any(a.shape != (n,) for a in idx):
+        raise ValueError("index arrays must be 1-D and of equal length")
+    if n and any(a.min() < 0 or a.max() >= m for a, m in zip(idx, (B, C, Dd, Hs, Ws))):
+        raise ValueError("sample index out of range")
+    out = np.empty(n, dtype=np.float64)
+    _load().oracle_causal_conv3d_points(B, C, Dd, Hs, Ws, k.shape[1], k.shape[2], k.shape[3], _p(u), _p(k), n,
+                                        *[_ip(a) for a in idx], _p(out))
+    return out
 
 
 def causal_conv2d_dynamic(u, k) -> np.ndarray:

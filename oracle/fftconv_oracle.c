@@ -329,6 +329,58 @@ void oracle_causal_conv2d_points(int64_t B, int64_t C, int64_t Hs, int64_t Ws, i
     }
 }
 
+/*
+ * 3-D variant ("Native Multi-Dimensional Subquadratic Operators via Input
+ * Dependent Long Convolutions", abstract: the long convolution on native N-D
+ * geometry), the first-octant crop of the zero-padded linear convolution:
+ *     y[b,c,d,i,j] = sum_{e<=d, p<=i, q<=j} k[c,e,p,q] u[b,c,d-e,i-p,j-q],
+ * d < Dd, i < Hs, j < Ws; k is [C][Kd][Kh][Kw] (taps outside it are zero).
+ */
+static double conv3d_point(int64_t Hs, int64_t Ws, int64_t Kd, int64_t Kh, int64_t Kw, const double* u,
+                           const double* k, int64_t d, int64_t i, int64_t j)
+{
+    double acc = 0.0;
+    int64_t emax = d < Kd - 1 ? d : Kd - 1;
+    int64_t pmax = i < Kh - 1 ? i : Kh - 1;
+    int64_t qmax = j < Kw - 1 ? j : Kw - 1;
+    for (int64_t e = 0; e <= emax; ++e)
+        for (int64_t p = 0; p <= pmax; ++p)
+            for (int64_t q = 0; q <= qmax; ++q)
+                acc += k[(e * Kh + p) * Kw + q] * u[((d - e) * Hs + (i - p)) * Ws + (j - q)];
+    return acc;
+}
+
+void oracle_causal_conv3d(int64_t B, int64_t C, int64_t Dd, int64_t Hs, int64_t Ws, int64_t Kd, int64_t Kh,
+                          int64_t Kw, const double* u, const double* k, double* y)
+{
+    int64_t vol = Dd * Hs * Ws, vols = B * C;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < vols; ++r) {
+        int64_t c = r % C;
+        const double* ur = u + r * vol;
+        const double* kc = k + c * Kd * Kh * Kw;
+        for (int64_t d = 0; d < Dd; ++d)
+            for (int64_t i = 0; i < Hs; ++i)
+                for (int64_t j = 0; j < Ws; ++j)
+                    y[r * vol + (d * Hs + i) * Ws + j] = conv3d_point(Hs, Ws, Kd, Kh, Kw, ur, kc, d, i, j);
+    }
+}
+
+/* Sampled 3-D oracle: out[n] = y[bi[n], ci[n], di[n], ii[n], jj[n]]. */
+void oracle_causal_conv3d_points(int64_t B, int64_t C, int64_t Dd, int64_t Hs, int64_t Ws, int64_t Kd,
+                                 int64_t Kh, int64_t Kw, const double* u, const double* k, int64_t n_pts,
+                                 const int64_t* bi, const int64_t* ci, const int64_t* di, const int64_t* ii,
+                                 const int64_t* jj, double* out)
+{
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < n_pts; ++n) {
+        const double* ur = u + (bi[n] * C + ci[n]) * Dd * Hs * Ws;
+        const double* kc = k + ci[n] * Kd * Kh * Kw;
+        out[n] = conv3d_point(Hs, Ws, Kd, Kh, Kw, ur, kc, di[n], ii[n], jj[n]);
+    }
+}
+
 /* exp(-2*pi*i*m/M) for an integer m reduced mod M first, so the angle is exact. */
 static void unit_root(int64_t m, int64_t M, double* re, double* im)
 {

@@ -430,6 +430,39 @@ def check_conv2d_dynamic():
     assert np.allclose(pts, y[bi, ci, ii, jj], rtol=1e-12, atol=1e-12)
 
 
+def check_conv3d():
+    """3-D first-octant crop: scipy.signal.convolve's full N-D linear
+    convolution (direct method) cropped; one depth slice is the 2-D oracle;
+    a separable volume and filter give the product of three 1-D causal
+    convolutions; the delta filter returns u; the sampled entry point
+    matches the full one."""
+    from scipy.signal import convolve
+    r = _rng(69)
+    B, C, Dd, Hs, Ws, Kd, Kh, Kw = 2, 2, 4, 8, 16, 3, 5, 16
+    u = r.standard_normal((B, C, Dd, Hs, Ws))
+    k = r.standard_normal((C, Kd, Kh, Kw))
+    y = oracle.causal_conv3d(u, k)
+    for b in range(B):
+        for c in range(C):
+            want = convolve(u[b, c], k[c], method="direct")[:Dd, :Hs, :Ws]
+            assert np.allclose(y[b, c], want, rtol=1e-11, atol=1e-11), (b, c)
+    flat = oracle.causal_conv3d(u[:, :, :1], k[:, :1])
+    assert np.allclose(flat[:, :, 0], oracle.causal_conv2d(u[:, :, 0], k[:, 0]), rtol=1e-12, atol=1e-12)
+    a1, a2, a3 = r.standard_normal(Dd), r.standard_normal(Hs), r.standard_normal(Ws)
+    f1, f2, f3 = r.standard_normal(Kd), r.standard_normal(Kh), r.standard_normal(Kw)
+    us = np.einsum("d,i,j->dij", a1, a2, a3)[None, None]
+    ks = np.einsum("d,i,j->dij", f1, f2, f3)[None]
+    sep = np.einsum("d,i,j->dij", np.convolve(a1, f1)[:Dd], np.convolve(a2, f2)[:Hs], np.convolve(a3, f3)[:Ws])
+    assert np.allclose(oracle.causal_conv3d(us, ks)[0, 0], sep, rtol=1e-11, atol=1e-11)
+    delta = np.zeros((C, Kd, Kh, Kw))
+    delta[:, 0, 0, 0] = 1.0
+    assert np.array_equal(oracle.causal_conv3d(u, delta), u)
+    bi, ci, di = np.array([0, 1, 1]), np.array([1, 0, 1]), np.array([3, 0, 2])
+    ii, jj = np.array([7, 0, 4]), np.array([15, 3, 0])
+    pts = oracle.causal_conv3d_points(u, k, bi, ci, di, ii, jj)
+    assert np.allclose(pts, y[bi, ci, di, ii, jj], rtol=1e-12, atol=1e-12)
+
+
 def check_conv2d_offset():
     """Crop offsets: (0, 0) is the first-quadrant oracle; any offset is the
     window of scipy.signal.convolve2d's full linear convolution."""
@@ -454,5 +487,5 @@ ALL_CHECKS = [
     check_causality_shift, check_closed_forms, check_points_match_full_1d,
     check_conv2d_library, check_conv2d_separable_and_dft, check_points_match_full_2d,
     check_bwd_central_differences, check_bwd_numpy_correlate, check_bwd_delta_kernel, check_dynamic_kernels,
-    check_ssm_kernel, check_freq_sparse, check_conv2d_offset, check_conv2d_dynamic,
+    check_ssm_kernel, check_freq_sparse, check_conv2d_offset, check_conv2d_dynamic, check_conv3d,
 ]

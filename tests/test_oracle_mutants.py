@@ -57,6 +57,10 @@ MUTANTS = {
                              "double mag = pow(sqrt(lr * lr + li * li), (double)(t + 1));"),
     "conv2d_offset_ignored": ("int64_t fi = i + oy, fj = j + ox;", "int64_t fi = i, fj = j + ox;"),
     "conv2d_offset_clip": ("if (a < 0 || a >= Hs) continue;", "if (a < 0 || a >= Hs - 1) continue;"),
+    "conv3d_no_depth_shift": ("acc += k[(e * Kh + p) * Kw + q] * u[((d - e) * Hs + (i - p)) * Ws + (j - q)];",
+                              "acc += k[(e * Kh + p) * Kw + q] * u[(d * Hs + (i - p)) * Ws + (j - q)];"),
+    "conv3d_drop_last_depth_tap": ("int64_t emax = d < Kd - 1 ? d : Kd - 1;",
+                                   "int64_t emax = d < Kd - 2 ? d : Kd - 2;"),
 }
 
 
