@@ -67,6 +67,10 @@ _SIGS = {
     "fftconv2d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
     "fftconv2d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv2d_fwd_offset": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int]),
+    "fftconv3d_plan_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "fftconv3d_kernel_spectrum": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
+    "fftconv3d_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fftconv2d_dynamic_plan_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
                                                      ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "fftconv2d_fwd_dynamic": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]),
@@ -399,6 +403,46 @@ class Plan2DDynamic(_PlanBase):
         workspace = self._ws(workspace)
         _check(self.lib.fftconv2d_fwd_dynamic(self._handle, _ptr(u), _ptr(k), k.shape[2], k.shape[3], _ptr(y),
                                               _ptr(workspace), _stream(stream)), "fftconv2d_fwd_dynamic")
+        return y
+
+
+class Plan3D(_PlanBase):
+    """3-D plan: fftconv3d_plan_create(B, C, Dd, Hs, Ws, dtype)."""
+
+    def __init__(self, B: int, C: int, Dd: int, Hs: int, Ws: int, dtype: str = "f32"):
+        self.lib = load_library()
+        self.B, self.C, self.Dd, self.Hs, self.Ws, self.dtype = B, C, Dd, Hs, Ws, dtype
+        self.torch_dtype = TORCH_DTYPES[dtype]
+        h = ctypes.c_void_p()
+        _check(self.lib.fftconv3d_plan_create(ctypes.byref(h), B, C, Dd, Hs, Ws, DTYPES[dtype]),
+               "fftconv3d_plan_create")
+        self._handle = h
+        self._workspace = None
+
+    def kernel_spectrum(self, k: torch.Tensor, khat: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """khat <- spectrum of k [C, Kd, Kh, Kw] (fp32)."""
+        if k.dim() != 4:
+            raise ValueError("k must be [C, Kd, Kh, Kw]")
+        _need(k, "k", (self.C, k.shape[1], k.shape[2], k.shape[3]), torch.float32)
+        if khat is None:
+            khat = self.new_spectrum(k.device)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv3d_kernel_spectrum(self._handle, _ptr(k), k.shape[1], k.shape[2], k.shape[3],
+                                                  _ptr(khat), _ptr(workspace), _stream(stream)),
+               "fftconv3d_kernel_spectrum")
+        return khat
+
+    def fwd(self, u: torch.Tensor, khat: torch.Tensor, y: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        shape = (self.B, self.C, self.Dd, self.Hs, self.Ws)
+        _need(u, "u", shape, self.torch_dtype)
+        if y is None:
+            y = torch.empty(shape, dtype=self.torch_dtype, device=u.device)
+        _need(y, "y", shape, self.torch_dtype)
+        workspace = self._ws(workspace)
+        _check(self.lib.fftconv3d_fwd(self._handle, _ptr(u), _ptr(khat), _ptr(y), _ptr(workspace), _stream(stream)),
+               "fftconv3d_fwd")
         return y
 
 

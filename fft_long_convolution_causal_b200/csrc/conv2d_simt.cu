@@ -345,4 +345,263 @@ cudaError_t launch_conv2d_spectrum(const fftconv_plan_s& p, const float* k, int 
     }
 }
 
+// ====================================================================== 3-D
+// The 3-D causal convolution ("Native Multi-Dimensional Subquadratic
+// Operators via Input Dependent Long Convolutions", abstract: the long
+// convolution on native N-D geometry), first-octant crop of the zero-padded
+// linear convolution, over (2 Dd) x (2 Hs) x (2 Ws) points.  Every depth
+// slice of a volume is an image of a 2-D plan with C Dd channels (channel
+// c Dd + d), so the 2-D row and column passes serve unchanged:
+//   1. rows of every slice pair (c2_pass1)            -> W2 [slice pair][Hs][LR]
+//   2. columns, forward only (c2_pass2 MODE 1)         -> W3 [slice pair][LC][LR] = X2 / (LC LR)
+//   3. depth: DFT over d (Dd nonzero of LD = 2 Dd), product with K3, inverse,
+//      d < Dd kept, in place in W3 (c3_depth MODE 0)
+//   4. columns, inverse only, rows i < Hs kept (c3_colinv) -> W2
+//   5. rows, inverse, crop, store (c2_pass3)
+// The spectrum K3 = DFT3(pad k) / LD is built the same way (steps 1, 2 on the
+// filter slices, then c3_depth MODE 1); with step 2's 1 / (LC LR) the product
+// carries the whole 1 / (LD LC LR) of the inverse.
+
+// Inverse column DFT of full column spectra: spec[g][ky][kx] (LC x LR) -> rows
+// i < Hs of work[g] (Hs x LR).
+template <int LOG2LC, int LOG2LR>
+__global__ void __launch_bounds__(Col2G<LOG2LC>::T)
+c3_colinv(const float2* __restrict__ spec, float2* __restrict__ work, const float2* __restrict__ twC) {
+    using G = Col2G<LOG2LC>;
+    using Lay = typename G::Lay;
+    constexpr int LC = 1 << LOG2LC, LR = 1 << LOG2LR, Hs = LC / 2;
+    constexpr int NS = G::Plan::kStages;
+    constexpr int R0 = 1 << G::Plan::log2r(0), RL = 1 << G::Plan::log2r(NS - 1);
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x;
+    const int kx0 = blockIdx.x * kTile2d;
+    const float2* __restrict__ in = spec + (size_t)blockIdx.y * LC * LR;
+    float2* __restrict__ img = work + (size_t)blockIdx.y * Hs * LR;
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    stage<G, 0, true, R0, R0, false>(
+        tid, twC, [&](int ky, int c) { return in[(size_t)ky * LR + kx0 + c]; }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS - 1, true>(smem, tid, twC);
+    stage<G, NS - 1, true, RL, RL / 2, false>(tid, twC, lds, [&](int i, int c, float2 z) {
+        img[(size_t)i * LR + kx0 + c] = z;
+    });
+}
+
+// Depth pass over the slices of one volume ("set": channel c_rel of the
+// group, pair bp), 16 plane positions f0 .. f0 + 15 per CTA: slice d of the
+// set at work + c_rel cstride + bp plane + d dstride; the first nz of the LD
+// depth points are nonzero (the rest is the padding).
+//   MODE 0: forward DFT over d, product with K3[c][kd][f], inverse, d < LD/2 kept, in place;
+//   MODE 1: forward DFT over d times scale -> khat_out[c][kd][f].
+template <int LOG2LD, int MODE>
+__global__ void __launch_bounds__(Col2G<LOG2LD>::T)
+c3_depth(float2* __restrict__ work, const float2* __restrict__ khat3, float2* __restrict__ khat_out,
+         const float2* __restrict__ twD, int nz, int64_t plane, int64_t dstride, int64_t cstride, int npp,
+         int64_t first_c, float scale) {
+    using G = Col2G<LOG2LD>;
+    using Lay = typename G::Lay;
+    constexpr int LD = 1 << LOG2LD;
+    constexpr int NS = G::Plan::kStages;
+    constexpr int R0 = 1 << G::Plan::log2r(0), RL = 1 << G::Plan::log2r(NS - 1);
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x;
+    const int c_rel = blockIdx.y / npp, bp = blockIdx.y % npp;
+    float2* __restrict__ base = work + (size_t)c_rel * cstride + (size_t)bp * plane;
+    const size_t f0 = (size_t)blockIdx.x * kTile2d;
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, twD,
+        [&](int d, int c) { return d < nz ? base[(size_t)d * dstride + f0 + c] : make_float2(0.f, 0.f); }, sts);
+    __syncthreads();
+    if constexpr (MODE == 1) {
+        smem_stages<G, 1, NS - 1, false>(smem, tid, twD);
+        float2* __restrict__ out = khat_out + (size_t)(first_c + c_rel) * LD * plane;
+        stage<G, NS - 1, false, RL, RL, false>(tid, twD, lds, [&](int kd, int c, float2 z) {
+            out[(size_t)kd * plane + f0 + c] = cscale(z, scale);
+        });
+    } else {
+        smem_stages<G, 1, NS, false>(smem, tid, twD);
+        const float2* __restrict__ kh = khat3 + (size_t)(first_c + c_rel) * LD * plane;
+        stage<G, 0, true, R0, R0, true>(
+            tid, twD,
+            [&](int kd, int c) { return cmul(smem[Lay::at(kd, c)], __ldg(&kh[(size_t)kd * plane + f0 + c])); },
+            sts);
+        __syncthreads();
+        smem_stages<G, 1, NS - 1, true>(smem, tid, twD);
+        stage<G, NS - 1, true, RL, RL / 2, false>(tid, twD, lds, [&](int d, int c, float2 z) {
+            base[(size_t)d * dstride + f0 + c] = z;
+        });
+    }
+}
+
+template <int LOG2LD, int MODE>
+static cudaError_t c3_depth_go(const fftconv_plan_s& p, float2* work, const float2* khat3, float2* khat_out,
+                               int nz, int64_t plane, int64_t dstride, int64_t cstride, int npp, int64_t first_c,
+                               int sets, float scale, cudaStream_t s) {
+    auto kern = c3_depth<LOG2LD, MODE>;
+    const size_t sm = Col2G<LOG2LD>::Lay::kWords * sizeof(float2);
+    ensure_smem2(kern, sm);
+    kern<<<dim3((unsigned)(plane / kTile2d), sets), Col2G<LOG2LD>::T, sm, s>>>(
+        work, khat3, khat_out, p.tw3.wD, nz, plane, dstride, cstride, npp, first_c, scale);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t c3_depth_sw(const fftconv_plan_s& p, float2* work, const float2* khat3, float2* khat_out, int nz,
+                               int64_t plane, int64_t dstride, int64_t cstride, int npp, int64_t first_c, int sets,
+                               float scale, cudaStream_t s) {
+    switch (ilog2_host(p.Dd)) {
+#define FFTC_D(LD)                                                                                                \
+    case LD: return c3_depth_go<LD + 1, MODE>(p, work, khat3, khat_out, nz, plane, dstride, cstride, npp, first_c, \
+                                              sets, scale, s);
+        FFTC_D(4) FFTC_D(5) FFTC_D(6) FFTC_D(7) FFTC_D(8)
+#undef FFTC_D
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// the workspace of a group of gc channels: W2 then W3 (whole slice pairs)
+static void c3_split(const fftconv_plan_s& p, float2* work, float2** w2, float2** w3) {
+    const size_t LR = 2 * (size_t)p.Ws, LC = 2 * (size_t)p.Hs;
+    const size_t slices = (size_t)p.group * p.Dd * ((p.B + 1) / 2);
+    *w2 = work;
+    *w3 = work + slices * p.Hs * LR;
+    (void)LC;
+}
+
+template <int LOG2LC, int LOG2LR, typename IO>
+static cudaError_t c3_fwd_go(const fftconv_plan_s& p, const void* u, const float2* khat3, void* y, float2* work,
+                             cudaStream_t s) {
+    constexpr int Hs = (1 << LOG2LC) / 2;
+    constexpr int RB = rows_per_cta<LOG2LR>(Hs);
+    constexpr int LR = 1 << LOG2LR, LC = 1 << LOG2LC;
+    auto k1 = c2_pass1<LOG2LR, RB, IO, 0>;
+    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1, false>;
+    auto k4 = c3_colinv<LOG2LC, LOG2LR>;
+    auto k5 = c2_pass3<LOG2LR, RB, IO>;
+    const size_t sr = Row2G<LOG2LR, RB>::Lay::kWords * sizeof(float2);
+    const size_t sc = Col2G<LOG2LC>::Lay::kWords * sizeof(float2);
+    ensure_smem2(k1, sr);
+    ensure_smem2(k2, sc);
+    ensure_smem2(k4, sc);
+    ensure_smem2(k5, sr);
+    const int npp = (p.B + 1) / 2;
+    const int Cs = p.H * p.Dd;  // channels of the slice view
+    const int64_t plane = (int64_t)LC * LR;
+    float2 *w2, *w3;
+    c3_split(p, work, &w2, &w3);
+    for (int64_t c0 = 0; c0 < p.H; c0 += p.group) {
+        const int gc = (int)((p.H - c0) < p.group ? (p.H - c0) : p.group);
+        const int g = gc * p.Dd * npp;            // slice pairs of the group
+        const int64_t first = c0 * p.Dd * npp;    // their first index in the slice view
+        k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>((const IO*)u, nullptr, 0, 0, w2, p.tw.wL, p.B, Cs, Hs,
+                                                             first);
+        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(w2, nullptr, w3, p.tw.wC, 1, 0, 0);
+        cudaError_t e = c3_depth_sw<0>(p, w3, khat3, nullptr, p.Dd, plane, (int64_t)npp * plane,
+                                       (int64_t)p.Dd * npp * plane, npp, c0, gc * npp, 1.0f, s);
+        if (e != cudaSuccess) return e;
+        k4<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(w3, w2, p.tw.wC);
+        k5<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(w2, (IO*)y, p.tw.wL, p.B, Cs, Hs, first, 0);
+    }
+    return cudaGetLastError();
+}
+
+template <int LOG2LC, int LOG2LR>
+static cudaError_t c3_spec_go(const fftconv_plan_s& p, const float* k, int Kd, int Kh, int Kw, float2* khat3,
+                              float2* work, cudaStream_t s) {
+    constexpr int Hs = (1 << LOG2LC) / 2;
+    constexpr int RB = rows_per_cta<LOG2LR>(Hs);
+    constexpr int LR = 1 << LOG2LR, LC = 1 << LOG2LC;
+    auto k1 = c2_pass1<LOG2LR, RB, float, 1>;
+    auto k2 = c2_pass2<LOG2LC, LOG2LR, 1, false>;
+    const size_t sr = Row2G<LOG2LR, RB>::Lay::kWords * sizeof(float2);
+    const size_t sc = Col2G<LOG2LC>::Lay::kWords * sizeof(float2);
+    ensure_smem2(k1, sr);
+    ensure_smem2(k2, sc);
+    const int64_t plane = (int64_t)LC * LR;
+    const int LD = 2 * p.Dd;
+    float2 *w2, *w3;
+    c3_split(p, work, &w2, &w3);
+    for (int64_t c0 = 0; c0 < p.H; c0 += p.group) {
+        const int gc = (int)((p.H - c0) < p.group ? (p.H - c0) : p.group);
+        const int g = gc * Kd;  // filter slices of the group, as images [C Kd][Kh][Kw]
+        k1<<<dim3(Hs / RB, g), Row2G<LOG2LR, RB>::T, sr, s>>>(nullptr, k, Kh, Kw, w2, p.tw.wL, 1, p.H * Kd, Hs,
+                                                             c0 * Kd);
+        k2<<<dim3(LR / kTile2d, g), Col2G<LOG2LC>::T, sc, s>>>(w2, nullptr, w3, p.tw.wC, 1, 0, 0);
+        cudaError_t e = c3_depth_sw<1>(p, w3, nullptr, khat3, Kd, plane, plane, (int64_t)Kd * plane, 1, c0, gc,
+                                       (float)plane / (float)LD, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+template <int LOG2LC>
+static cudaError_t c3_fwd_w(const fftconv_plan_s& p, const void* u, const float2* khat3, void* y, float2* work,
+                            cudaStream_t s) {
+    const bool bf = p.dtype == FFTCONV_BF16;
+    switch (ilog2_host(p.Ws)) {
+#define FFTC_C(LW) \
+    case LW: return bf ? c3_fwd_go<LOG2LC, LW + 1, __nv_bfloat16>(p, u, khat3, y, work, s) \
+                       : c3_fwd_go<LOG2LC, LW + 1, float>(p, u, khat3, y, work, s);
+        FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
+#undef FFTC_C
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int LOG2LC>
+static cudaError_t c3_spec_w(const fftconv_plan_s& p, const float* k, int Kd, int Kh, int Kw, float2* khat3,
+                             float2* work, cudaStream_t s) {
+    switch (ilog2_host(p.Ws)) {
+#define FFTC_C(LW) case LW: return c3_spec_go<LOG2LC, LW + 1>(p, k, Kd, Kh, Kw, khat3, work, s);
+        FFTC_C(4) FFTC_C(5) FFTC_C(6) FFTC_C(7) FFTC_C(8)
+#undef FFTC_C
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int LOG2LD>
+static bool c3_depth_tables_go(std::vector<float2>& out, size_t* offD) {
+    *offD = out.size();
+    append_stage_twiddles<Col2G<LOG2LD>>(out);
+    return true;
+}
+
+bool conv3d_depth_tables(int Dd, std::vector<float2>& out, size_t* offD) {
+    switch (ilog2_host(Dd)) {
+        case 4: return c3_depth_tables_go<5>(out, offD);
+        case 5: return c3_depth_tables_go<6>(out, offD);
+        case 6: return c3_depth_tables_go<7>(out, offD);
+        case 7: return c3_depth_tables_go<8>(out, offD);
+        case 8: return c3_depth_tables_go<9>(out, offD);
+        default: return false;
+    }
+}
+
+cudaError_t launch_conv3d_fwd(const fftconv_plan_s& p, const void* u, const float2* khat3, void* y, float2* work,
+                              cudaStream_t s) {
+    switch (ilog2_host(p.Hs)) {
+        case 4: return c3_fwd_w<5>(p, u, khat3, y, work, s);
+        case 5: return c3_fwd_w<6>(p, u, khat3, y, work, s);
+        case 6: return c3_fwd_w<7>(p, u, khat3, y, work, s);
+        case 7: return c3_fwd_w<8>(p, u, khat3, y, work, s);
+        case 8: return c3_fwd_w<9>(p, u, khat3, y, work, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_conv3d_spectrum(const fftconv_plan_s& p, const float* k, int Kd, int Kh, int Kw, float2* khat3,
+                                   float2* work, cudaStream_t s) {
+    switch (ilog2_host(p.Hs)) {
+        case 4: return c3_spec_w<5>(p, k, Kd, Kh, Kw, khat3, work, s);
+        case 5: return c3_spec_w<6>(p, k, Kd, Kh, Kw, khat3, work, s);
+        case 6: return c3_spec_w<7>(p, k, Kd, Kh, Kw, khat3, work, s);
+        case 7: return c3_spec_w<8>(p, k, Kd, Kh, Kw, khat3, work, s);
+        case 8: return c3_spec_w<9>(p, k, Kd, Kh, Kw, khat3, work, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace fftc

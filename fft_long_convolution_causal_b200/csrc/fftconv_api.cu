@@ -485,6 +485,7 @@ const char* fftconv_plan_path(fftconv_plan_t p) {
         case fftc::PATH_2D: return p->tc2d ? "2d_tc" : "2d";
         case fftc::PATH_SSM: return "ssm_chunked";
         case fftc::PATH_PARTIAL: return "partial_chunked";
+        case fftc::PATH_3D: return "3d";
     }
     return "unknown";
 }
@@ -602,6 +603,75 @@ fftconv_status fftconv2d_fwd_dynamic(fftconv_plan_t p, const void* u, const floa
     cudaError_t e = fftc::launch_conv2d_spectrum(*p, k, Kh, Kw, khat, rest, s);
     if (e == cudaSuccess) e = fftc::launch_conv2d_fwd(*p, u, khat, y, rest, s, 0, 0);
     return cuda_status(e);
+}
+
+fftconv_status fftconv3d_plan_create(fftconv_plan_t* out, int B, int C, int Dd, int Hs, int Ws, fftconv_dtype dtype) {
+    if (!out) return FFTCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || C < 1 || (dtype != FFTCONV_F32 && dtype != FFTCONV_BF16)) return FFTCONV_ERR_INVALID_ARG;
+    if ((int64_t)C * Dd > (int64_t)1 << 30) return FFTCONV_ERR_INVALID_ARG;
+    auto side_ok = [](int x) { return is_pow2(x) && x >= FFTCONV3D_MIN_SIDE && x <= FFTCONV3D_MAX_SIDE; };
+    if (!side_ok(Dd) || !side_ok(Hs) || !side_ok(Ws)) return FFTCONV_ERR_UNSUPPORTED;
+    fftconv_plan_s* p = new (std::nothrow) fftconv_plan_s();
+    if (!p) return FFTCONV_ERR_OOM;
+    p->kind = 5;
+    p->path = fftc::PATH_3D;
+    p->B = B;
+    p->H = C;
+    p->Dd = Dd;
+    p->Hs = Hs;
+    p->Ws = Ws;
+    p->dtype = dtype;
+    p->pairs = (int64_t)((B + 1) / 2) * C;
+    cudaGetDevice(&p->device);
+    const int64_t LR = 2 * (int64_t)Ws, LC = 2 * (int64_t)Hs, LD = 2 * (int64_t)Dd;
+    std::vector<float2> host;
+    size_t offR = 0, offC = 0, offD = 0;
+    fftc::conv2d_tables(Hs, Ws, host, &offR, &offC);
+    fftc::conv3d_depth_tables(Dd, host, &offD);
+    const size_t offErr = append_status_word(host);
+    // workspace per channel: its slice pairs' row spectra (Hs x LR) and column spectra (LC x LR)
+    const size_t per_channel = (size_t)Dd * ((B + 1) / 2) * (size_t)(Hs + LC) * LR * sizeof(float2);
+    int64_t g = (int64_t)(group_bytes(defaults()) / per_channel);
+    if (g < 1) g = 1;
+    if (g > C) g = C;
+    p->group = (int)g;
+    p->spectrum_bytes = (size_t)C * LD * LC * LR * sizeof(float2);
+    p->workspace_bytes = (size_t)g * per_channel;
+    fftconv_status st = upload_tables(p, host);
+    if (st != FFTCONV_OK) {
+        delete p;
+        return st;
+    }
+    const float2* base = (const float2*)p->d_tables;
+    p->tw.wL = base + offR;
+    p->tw.wC = base + offC;
+    p->tw3.wD = base + offD;
+    p->d_err = (int*)(base + offErr);
+    *out = p;
+    return FFTCONV_OK;
+}
+
+fftconv_status fftconv3d_kernel_spectrum(fftconv_plan_t p, const float* k, int Kd, int Kh, int Kw, void* khat,
+                                         void* work, void* stream) {
+    if (!p || p->kind != 5 || !k || !khat || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (Kd < 1 || Kh < 1 || Kw < 1 || Kd > p->Dd || Kh > p->Hs || Kw > p->Ws) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(khat) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    cudaError_t e =
+        fftc::launch_conv3d_spectrum(*p, k, Kd, Kh, Kw, (float2*)khat, (float2*)work, (cudaStream_t)stream);
+    if (e == cudaSuccess) p->spectrum_ready = true;
+    return cuda_status(e);
+}
+
+fftconv_status fftconv3d_fwd(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work, void* stream) {
+    if (!p || p->kind != 5 || !u || !khat || !y || !work) return FFTCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(khat) || !aligned16(y) || !aligned16(work)) return FFTCONV_ERR_INVALID_ARG;
+    if (y == u) return FFTCONV_ERR_INVALID_ARG;
+    if (!on_plan_device(p)) return FFTCONV_ERR_INVALID_ARG;
+    if (!p->spectrum_ready) return FFTCONV_ERR_NOT_READY;
+    return cuda_status(
+        fftc::launch_conv3d_fwd(*p, u, (const float2*)khat, y, (float2*)work, (cudaStream_t)stream));
 }
 
 fftconv_status fftconv2d_fwd(fftconv_plan_t p, const void* u, const void* khat, void* y, void* work, void* stream) {

@@ -11,7 +11,8 @@
 
 namespace fftc {
 
-enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2, PATH_FUSED_TC = 3, PATH_SSM = 4, PATH_PARTIAL = 5 };
+enum Path { PATH_FUSED = 0, PATH_MULTIPASS = 1, PATH_2D = 2, PATH_FUSED_TC = 3, PATH_SSM = 4, PATH_PARTIAL = 5,
+            PATH_3D = 6 };
 
 // Twiddle tables of one plan (device pointers into one allocation).  wL / wC
 // are per-stage tables of the row / column transforms (StageTwiddles layout);
@@ -21,6 +22,11 @@ struct Tables {
     const float2* wC = nullptr;     // multipass: columns N1;  2-D: columns 2Hs
     const float2* wLo = nullptr;    // multipass: W_M^e for e < 2^S
     const float2* wHi = nullptr;    // multipass: W_M^(e 2^S) for e < M / 2^S
+};
+
+// 3-D plans: the depth transform's stage table (2 Dd points).
+struct Tables3 {
+    const float2* wD = nullptr;
 };
 
 // Constant tables of the tensor-core path, in per-lane fragment order.
@@ -45,11 +51,12 @@ struct C2TcTables {
 }  // namespace fftc
 
 struct fftconv_plan_s {
-    int kind = 1;          // 1: 1-D, 2: 2-D, 3: state-space filters, chunked, 4: partial, chunked
+    int kind = 1;          // 1: 1-D, 2: 2-D, 3: state-space filters, chunked, 4: partial, chunked, 5: 3-D
     int path = 0;          // fftc::Path
     int B = 0, H = 0;      // 1-D batch, channels (2-D: B images, H = C channels)
     int64_t N = 0;         // 1-D sequence length
-    int Hs = 0, Ws = 0;    // 2-D image size
+    int Hs = 0, Ws = 0;    // 2-D image size (3-D: the slices)
+    int Dd = 0;            // 3-D depth
     int dtype = 0;         // fftconv_dtype
     int gated = 0;
     int log2M = 0;         // 1-D transform length 2N
@@ -62,6 +69,7 @@ struct fftconv_plan_s {
     size_t workspace_bytes = 0;
     void* d_tables = nullptr;
     fftc::Tables tw;
+    fftc::Tables3 tw3;
     fftc::TcTablePtrs tc;
     bool umma = false;              // fused tensor-core path on tcgen05 (else mma.sync)
     bool t2 = false;                // two-stage tcgen05 kernel (2N = 8192)
@@ -98,6 +106,11 @@ namespace fftc {
 bool fused_tables(int log2M, std::vector<float2>& out, size_t* offL);
 bool multipass_tables(int log2M, std::vector<float2>& out, size_t* offC, size_t* offR);
 bool conv2d_tables(int Hs, int Ws, std::vector<float2>& out, size_t* offR, size_t* offC);
+bool conv3d_depth_tables(int Dd, std::vector<float2>& out, size_t* offD);
+cudaError_t launch_conv3d_fwd(const fftconv_plan_s& p, const void* u, const float2* khat3, void* y, float2* work,
+                              cudaStream_t s);
+cudaError_t launch_conv3d_spectrum(const fftconv_plan_s& p, const float* k, int Kd, int Kh, int Kw, float2* khat3,
+                                   float2* work, cudaStream_t s);
 
 // 1-D bf16 two-stage tcgen05 path (2N = 8192, ungated): tables, spectrum
 // (fp32 SIMT transform written in the kernel's bf16 layout), forward.

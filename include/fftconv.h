@@ -336,6 +336,32 @@ FFTCONV_API fftconv_status fftconv2d_fwd_dynamic(fftconv_plan_t plan, const void
                                                  void* y, void* workspace, void* stream);
 
 /*
+ * 3-D causal convolution (N-D beyond 2-D; "Native Multi-Dimensional
+ * Subquadratic Operators via Input Dependent Long Convolutions", abstract:
+ * the long convolution on native N-D geometry): the first-octant crop of the
+ * zero-padded linear convolution,
+ *     y[b,c,d,i,j] = sum_{e<=d, p<=i, q<=j} k[c,e,p,q] u[b,c,d-e,i-p,j-q],
+ * d < Dd, i < Hs, j < Ws, by a (2Dd) x (2Hs) x (2Ws) transform (fp32 SIMT).
+ * Dd, Hs, Ws powers of two in [FFTCONV3D_MIN_SIDE, FFTCONV3D_MAX_SIDE]
+ * (else FFTCONV_ERR_UNSUPPORTED).  u, y: [B][C][Dd][Hs][Ws] of the plan's
+ * dtype; k: [C][Kd][Kh][Kw] fp32, 1 <= Kd <= Dd, 1 <= Kh <= Hs, 1 <= Kw <= Ws.
+ * khat: fftconv_spectrum_bytes(plan) bytes, computed once by
+ * fftconv3d_kernel_spectrum; workspace: fftconv_workspace_bytes(plan) bytes
+ * (both calls need it).  All device pointers 16-byte aligned; y must not
+ * alias u.  FFTCONV_ERR_NOT_READY before the spectrum; FFTCONV_ERR_INVALID_ARG
+ * for other plans or when the current device is not the plan's.  Path name
+ * "3d".
+ */
+#define FFTCONV3D_MIN_SIDE 16
+#define FFTCONV3D_MAX_SIDE 256
+FFTCONV_API fftconv_status fftconv3d_plan_create(fftconv_plan_t* plan, int B, int C, int Dd, int Hs, int Ws,
+                                                 fftconv_dtype dtype);
+FFTCONV_API fftconv_status fftconv3d_kernel_spectrum(fftconv_plan_t plan, const float* k, int Kd, int Kh, int Kw,
+                                                     void* khat, void* workspace, void* stream);
+FFTCONV_API fftconv_status fftconv3d_fwd(fftconv_plan_t plan, const void* u, const void* khat, void* y,
+                                         void* workspace, void* stream);
+
+/*
  * Conjugate spectrum: khat_conj <- conj(khat) in the plan's layout, the
  * spectrum of the correlation with k (the backward pass's filter).  khat is
  * the output of fftconv_kernel_spectrum on this plan; khat_conj is a buffer of
