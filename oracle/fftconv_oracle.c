@@ -341,11 +341,11 @@ static double conv3d_point(int64_t Hs, int64_t Ws, int64_t Kd, int64_t Kh, int64
 {
     double acc = 0.0;
     int64_t emax = d < Kd - 1 ? d : Kd - 1;
-    int64_t pmax = i < Kh - 1 ? i : Kh - 1;
-    int64_t qmax = j < Kw - 1 ? j : Kw - 1;
+    int64_t hmax = i < Kh - 1 ? i : Kh - 1;
+    int64_t wmax = j < Kw - 1 ? j : Kw - 1;
     for (int64_t e = 0; e <= emax; ++e)
-        for (int64_t p = 0; p <= pmax; ++p)
-            for (int64_t q = 0; q <= qmax; ++q)
+        for (int64_t p = 0; p <= hmax; ++p)
+            for (int64_t q = 0; q <= wmax; ++q)
                 acc += k[(e * Kh + p) * Kw + q] * u[((d - e) * Hs + (i - p)) * Ws + (j - q)];
     return acc;
 }
