@@ -132,14 +132,9 @@ fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
     auto bar = [&](const uint64_t& b) { return tc::smem_u32(&b); };
     auto first_pair = [&](int slot) { return (int)blockIdx.x + slot * (int)gridDim.x; };
 
-    // ---- set-up: constant matrices and twiddles into shared memory (all
-    // copies in flight at once), barriers, TMEM
-    for (int i = tid; i < (int)(kOffX / 16); i += kThreads) tc::cp_async16(sbase + 16u * i, mats + i, 16);
-    for (int i = tid; i < 2048; i += kThreads)
-        tc::cp_async16(sbase + kOffTW + 16u * i, reinterpret_cast<const uint4*>(twid) + i, 16);
-    tc::cp_async_commit();
-    tc::cp_async_wait_all();
-    um::fence_proxy_async();
+    // ---- set-up: barriers; the first input rows of both slots (bulk copies)
+    // in flight while the constant matrices and twiddles come into shared
+    // memory; TMEM
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             um::mbar_init(bar(s_bar[s].dA), 1);
@@ -154,6 +149,24 @@ fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
         }
         s_abort = 0;
     }
+    __syncthreads();
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            const int q = first_pair(s);
+            if (q < pairs) {
+                const uint32_t xb = bar(s_bar[s].xfull);
+                um::mbar_arrive_expect_tx(xb, kXBytes);
+                um::tma_load_5d(sbase + kOffX + kXBytes * (uint32_t)s, &xmap, 0, 0, 0, 2 * (q % npp), 8 * (q / npp),
+                                xb);
+            }
+        }
+    }
+    for (int i = tid; i < (int)(kOffX / 16); i += kThreads) tc::cp_async16(sbase + 16u * i, mats + i, 16);
+    for (int i = tid; i < 2048; i += kThreads)
+        tc::cp_async16(sbase + kOffTW + 16u * i, reinterpret_cast<const uint4*>(twid) + i, 16);
+    tc::cp_async_commit();
+    tc::cp_async_wait_all();
+    um::fence_proxy_async();
     if (warp == 0) {
         um::tmem_alloc(tc::smem_u32(&s_tmem), 512);
         um::tmem_relinquish();
@@ -228,10 +241,7 @@ fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
             };
             const SlotBars& sb = s_bar[s];
             int q = first_pair(s);
-            if (q < pairs) {
-                load_x(s, q);
-                inflight = true;
-            }
+            inflight = q < pairs;  // the set-up issued this pair's copy
             for (; q < pairs && ok; q += qstep) {
                 if (!(ok = wait(bar(sb.xfull), px))) break;
                 inflight = false;
