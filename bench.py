@@ -37,7 +37,7 @@ uniform sample of the same workload's outputs.
 variants (N=1): the skipped-work forms on the long workload's shape, each
 timed against the dense multi-pass plan on the same inputs (partial
 convolution, frequency-sparse filter, state-space filters with chunked state
-passing).
+passing), and the backward pass of the Hyena-style layer against its forward.
 """
 import argparse
 import hashlib
@@ -600,6 +600,24 @@ def variants(torch, steps=5):
     pair("ssm_chunked_d16", lambda: ssm.fwd(u, kss, D=D, y=y), lambda: dense.fwd(u, kd, D=D, y=y, workspace=ws),
          "diagonal state-space filters, chunks of 8192 with the state passed vs the dense plan on the same filters")
     del ssm, kss, dense, ws, u, y
+    torch.cuda.empty_cache()
+    # the backward pass on the Hyena-style layer (B=8, H=768, N=4096 bf16): du through the
+    # forward kernel with the conjugated spectrum, then dk and dD; against the forward
+    Bh, Hh, Nh = 8, 768, 4096
+    plan = binding.Plan(Bh, Hh, Nh, "bf16")
+    kh = (torch.randn(Hh, Nh, generator=g) * torch.exp(-1e-3 * torch.arange(Nh, dtype=torch.float32))).to(dev)
+    khat = plan.kernel_spectrum(kh)
+    kconj = plan.spectrum_conjugate(khat)
+    uh = torch.randn(Bh, Hh, Nh, generator=g).to(dev, torch.bfloat16)
+    dyh = torch.randn(Bh, Hh, Nh, generator=g).to(dev, torch.bfloat16)
+    Dh = torch.randn(Hh, generator=g).to(dev)
+    yh = torch.empty_like(uh)
+    tb = _time_fn(lambda: plan.bwd(dyh, uh, khat, kconj, D=Dh), steps, 3, torch, flush)
+    tf = _time_fn(lambda: plan.fwd(uh, khat, D=Dh, y=yh), steps, 3, torch, flush)
+    out["backward_hyena"] = {"ms_backward": round(tb, 4), "ms_forward": round(tf, 4),
+                             "ratio": round(tb / tf, 3), "path": plan.path,
+                             "note": "du, dk, dD of the Hyena-style layer against its forward"}
+    del plan, khat, kconj, uh, dyh, yh
     torch.cuda.empty_cache()
     return out
 
