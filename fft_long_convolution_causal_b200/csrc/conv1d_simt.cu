@@ -28,6 +28,7 @@
 #include "fft_simt.cuh"
 #include "plan.h"
 #include "tables.h"
+#include "tc_common.cuh"
 
 namespace fftc {
 
@@ -644,6 +645,77 @@ mp_pass1(const IO* __restrict__ u, const IO* __restrict__ w, const float* __rest
     });
 }
 
+// Pass 1, persistent (ungated forward): a CTA walks column tiles t =
+// blockIdx.x, + gridDim.x, ... (consecutive tiles share a pair), staging the
+// next tile's input rows (both images, rows n1 < N1/2, 32 columns) with
+// cp.async into a second buffer while it transforms the current one.
+template <int LOG2N1, int LOG2N2, typename IO>
+constexpr size_t mp1p_raw_bytes() {
+    return (size_t)2 * ((1 << LOG2N1) / 2) * kColTile<LOG2N1> * sizeof(IO);
+}
+
+template <int LOG2N1, int LOG2N2, typename IO>
+__global__ void __launch_bounds__(ColG<LOG2N1>::T)
+mp_pass1p(const IO* __restrict__ u, float2* __restrict__ work, const float2* __restrict__ twC,
+          const float2* __restrict__ lo, const float2* __restrict__ hi, int log2S, int B, int H, int64_t first,
+          int g, const uint8_t* __restrict__ keep) {
+    using G = ColG<LOG2N1>;
+    using Lay = typename G::Lay;
+    constexpr int N1 = 1 << LOG2N1, N2 = 1 << LOG2N2, LOG2M = LOG2N1 + LOG2N2;
+    constexpr int64_t N = (int64_t)N1 * N2 / 2;
+    constexpr int CT = kColTile<LOG2N1>, TPP = N2 / CT;  // columns per tile, tiles per pair
+    constexpr int NS = G::Plan::kStages, R0 = first_radix<G>(), RL = last_radix<G>();
+    constexpr int CPR = CT * (int)sizeof(IO) / 16;      // 16-byte chunks per input row of a tile
+    extern __shared__ float2 smem[];
+    IO* raw = reinterpret_cast<IO*>(smem + Lay::kWords);  // [image 2][n1 < N1/2][CT]
+    const uint32_t raw_s = tc::smem_u32(raw);
+    const int tid = threadIdx.x;
+    const int tiles = TPP * g;
+    auto lds = [&](int i, int c) { return smem[Lay::at(i, c)]; };
+    auto sts = [&](int i, int c, float2 z) { smem[Lay::at(i, c)] = z; };
+    auto prefetch = [&](int t) {
+        const int64_t P = first + t / TPP;
+        const int n2_0 = (t % TPP) * CT;
+        const int h = (int)(P % H), b0 = (int)(P / H) * 2;
+        const bool has1 = b0 + 1 < B;
+        for (int j = tid; j < 2 * (N1 / 2) * CPR; j += G::T) {
+            const int im = j / ((N1 / 2) * CPR), rem = j % ((N1 / 2) * CPR), n1 = rem / CPR, ch = rem % CPR;
+            const bool ok = im == 0 || has1;
+            const size_t row = ((size_t)(b0 + (ok ? im : 0)) * H + h) * N;
+            const IO* src = u + row + (size_t)n1 * N2 + n2_0 + ch * (16 / (int)sizeof(IO));
+            tc::cp_async16(raw_s + (uint32_t)j * 16u, src, ok ? 16 : 0);
+        }
+        tc::cp_async_commit();
+    };
+    int t = blockIdx.x;
+    if (t < tiles) prefetch(t);
+    for (; t < tiles; t += gridDim.x) {
+        tc::cp_async_wait_all();
+        __syncthreads();  // the tile's input is in; the previous tile's transform is written out
+        const int64_t P = first + t / TPP;
+        const int n2_0 = (t % TPP) * CT;
+        stage<G, 0, false, R0 / 2, R0, false>(
+            tid, twC,
+            [&](int n1, int c) {
+                return make_float2(to_f(raw[(size_t)n1 * CT + c]), to_f(raw[(size_t)(N1 / 2 + n1) * CT + c]));
+            },
+            sts);
+        __syncthreads();  // the input buffer is free: stage the next tile's
+        if (t + (int)gridDim.x < tiles) prefetch(t + gridDim.x);
+        smem_stages<G, 1, NS - 1, false>(smem, tid, twC);
+        float2* __restrict__ out = work + (size_t)(t / TPP) * ((size_t)N1 * N2);
+        float2 tw = make_float2(1.f, 0.f), step = make_float2(1.f, 0.f);
+        stage<G, NS - 1, false, RL, RL, false>(tid, twC, lds, [&](int k1, int c, float2 z, int r) {
+            const uint32_t n2 = (uint32_t)(n2_0 + c);
+            if (r == 0) step = twiddle_M(lo, hi, n2 * (uint32_t)(N1 / RL), LOG2M, log2S);
+            tw = (r % kTwRun == 0) ? twiddle_M(lo, hi, n2 * (uint32_t)k1, LOG2M, log2S) : cmul(tw, step);
+            if (!keep || keep[k1]) out[(size_t)k1 * N2 + n2] = cmul(z, tw);
+        });
+        (void)P;
+    }
+    tc::cp_async_wait_all();
+}
+
 // Pass 2.  MODE 0: forward row DFT, product with Khat (+D/M), inverse, conj
 // twiddle, in place.  MODE 1: forward row DFT only, Khat[k1][k2] = X / M.
 // Three CTAs of up to 256 threads per SM (at most 85 registers; no spills).
@@ -751,11 +823,32 @@ static cudaError_t mp_fwd_go(const fftconv_plan_s& p, const void* u, const void*
     ensure_smem(k1, sc);
     ensure_smem(k2, sr);
     ensure_smem(k3, sc);
+    // ungated: the persistent pass 1 that stages the next tile's input while it
+    // transforms the current one (one CTA per SM)
+    auto k1p = mp_pass1p<LOG2N1, LOG2N2, IO>;
+    const size_t sp = sc + mp1p_raw_bytes<LOG2N1, LOG2N2, IO>();
+    static int sms = 0;
+    if (!GATED) {
+        ensure_smem(k1p, sp);
+        if (sms == 0) {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (sms <= 0) sms = 1;
+        }
+    }
     for (int64_t first = 0; first < p.pairs; first += p.group) {
         const int g = (int)((p.pairs - first) < p.group ? (p.pairs - first) : p.group);
-        k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0, work,
-                                                               p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S, p.B,
-                                                               p.H, first, p.d_keep);
+        if (!GATED) {
+            const int tiles = (N2 / kColTile<LOG2N1>) * g;
+            k1p<<<tiles < sms ? tiles : sms, ColG<LOG2N1>::T, sp, s>>>((const IO*)u, work, p.tw.wC, p.tw.wLo,
+                                                                      p.tw.wHi, p.log2S, p.B, p.H, first, g,
+                                                                      p.d_keep);
+        } else {
+            k1<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>((const IO*)u, (const IO*)w, nullptr, 0,
+                                                                   work, p.tw.wC, p.tw.wLo, p.tw.wHi, p.log2S,
+                                                                   p.B, p.H, first, p.d_keep);
+        }
         k2<<<dim3(N1 / RowG<LOG2N2>::C, g), RowG<LOG2N2>::T, sr, s>>>(work, khat, nullptr, D, p.tw.wL, p.tw.wLo, p.tw.wHi,
                                                     p.log2S, p.H, first, p.d_keep);
         k3<<<dim3(N2 / kColTile<LOG2N1>, g), ColG<LOG2N1>::T, sc, s>>>(work, (const IO*)v, (IO*)y, p.tw.wC, p.B,
