@@ -168,56 +168,70 @@ t2_spectrum_simt(const float* __restrict__ k, int L, uint16_t* __restrict__ khat
     });
 }
 
-// Filter gradient of the backward pass, one CTA per channel: for every pair
-// of batch rows, Zx = DFT_M(pad(x_b + i x_b+1)) and Zg = DFT_M(pad(g_b + i g_b+1))
-// (x = u or u w, g = dy or dy v), accumulated as T = sum conj(Zx) Zg in acc
-// ([H][M] fp32 complex, each thread its own frequencies f = tid + T m).  The
-// real part of the inverse of T is sum_b corr(g_b, x_b): the cross terms of
-// the packed pair land in the imaginary part.  dk[h][j] = that at lags
-// j < L, dD[h] = that at lag 0 (when dD is given).
+// Filter gradient of the backward pass, in two launches spread over every
+// (pair, channel).  For a pair of batch rows, Zx = DFT_M(pad(x_b + i x_b+1))
+// and Zg = DFT_M(pad(g_b + i g_b+1)) (x = u or u w, g = dy or dy v);
+// kgrad_pairs (one CTA per pair pp and channel h) writes the cross spectrum
+// conj(Zx) Zg to part[h][pp][f]; kgrad_finish (one CTA per channel) sums
+// the pairs' spectra in pair order into T.  The real part of the inverse of
+// T is sum_b corr(g_b, x_b): the cross terms of the packed pair land in the
+// imaginary part.  dk[h][j] = that at lags j < L, dD[h] = that at lag 0
+// (when dD is given).
 template <int LOG2M, typename IO, bool GATED>
 __global__ void __launch_bounds__(FusedG<LOG2M>::T)
-kgrad_simt(const IO* __restrict__ u, const IO* __restrict__ w, const IO* __restrict__ dy, const IO* __restrict__ v,
-           float2* __restrict__ acc, float* __restrict__ dk, float* __restrict__ dD, const float2* __restrict__ tw,
-           int B, int H, int L) {
+kgrad_pairs(const IO* __restrict__ u, const IO* __restrict__ w, const IO* __restrict__ dy, const IO* __restrict__ v,
+            float2* __restrict__ part, const float2* __restrict__ tw, int B, int H) {
     using G = FusedG<LOG2M>;
     using Lay = typename G::Lay;
     constexpr int M = G::L, N = M / 2, NS = G::Plan::kStages, T = G::T, FPT = M / T;
-    constexpr int R0 = first_radix<G>(), RL = last_radix<G>();
+    constexpr int R0 = first_radix<G>();
+    extern __shared__ float2 smem[];
+    const int tid = threadIdx.x, pp = blockIdx.x, h = blockIdx.y;
+    const int npp = (B + 1) / 2;
+    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
+    const int b0 = 2 * pp;
+    const bool has1 = b0 + 1 < B;
+    const size_t row0 = ((size_t)b0 * H + h) * N;
+    const size_t row1 = ((size_t)(b0 + 1) * H + h) * N;
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return load_pair<IO, GATED>(u, w, row0, row1, has1, n); }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(smem, tid, tw);
+    float2 zx[FPT];
+#pragma unroll
+    for (int m = 0; m < FPT; ++m) zx[m] = smem[Lay::at(tid + T * m, 0)];
+    __syncthreads();
+    stage<G, 0, false, R0 / 2, R0, false>(
+        tid, tw, [&](int n, int) { return load_pair<IO, GATED>(dy, v, row0, row1, has1, n); }, sts);
+    __syncthreads();
+    smem_stages<G, 1, NS, false>(smem, tid, tw);
+    float2* __restrict__ out = part + ((size_t)h * npp + pp) * M;
+#pragma unroll
+    for (int m = 0; m < FPT; ++m) {
+        const int f = tid + T * m;
+        out[f] = cmulc(smem[Lay::at(f, 0)], zx[m]);  // Zg conj(Zx)
+    }
+}
+
+template <int LOG2M>
+__global__ void __launch_bounds__(FusedG<LOG2M>::T)
+kgrad_finish(const float2* __restrict__ part, float* __restrict__ dk, float* __restrict__ dD,
+             const float2* __restrict__ tw, int npp, int L) {
+    using G = FusedG<LOG2M>;
+    using Lay = typename G::Lay;
+    constexpr int M = G::L, NS = G::Plan::kStages, T = G::T, FPT = M / T;
+    constexpr int RL = last_radix<G>();
     extern __shared__ float2 smem[];
     const int tid = threadIdx.x, h = blockIdx.x;
     auto lds = [&](int i, int) { return smem[Lay::at(i, 0)]; };
-    auto sts = [&](int i, int, float2 z) { smem[Lay::at(i, 0)] = z; };
-    float2* __restrict__ a = acc + (size_t)h * M;
-    const int npp = (B + 1) / 2;
-    for (int pp = 0; pp < npp; ++pp) {
-        const int b0 = 2 * pp;
-        const bool has1 = b0 + 1 < B;
-        const size_t row0 = ((size_t)b0 * H + h) * N;
-        const size_t row1 = ((size_t)(b0 + 1) * H + h) * N;
-        stage<G, 0, false, R0 / 2, R0, false>(
-            tid, tw, [&](int n, int) { return load_pair<IO, GATED>(u, w, row0, row1, has1, n); }, sts);
-        __syncthreads();
-        smem_stages<G, 1, NS, false>(smem, tid, tw);
-        float2 zx[FPT];
+    const float2* __restrict__ in = part + (size_t)h * npp * M;
 #pragma unroll
-        for (int m = 0; m < FPT; ++m) zx[m] = smem[Lay::at(tid + T * m, 0)];
-        __syncthreads();
-        stage<G, 0, false, R0 / 2, R0, false>(
-            tid, tw, [&](int n, int) { return load_pair<IO, GATED>(dy, v, row0, row1, has1, n); }, sts);
-        __syncthreads();
-        smem_stages<G, 1, NS, false>(smem, tid, tw);
-#pragma unroll
-        for (int m = 0; m < FPT; ++m) {
-            const int f = tid + T * m;
-            const float2 t = cmulc(smem[Lay::at(f, 0)], zx[m]);  // Zg conj(Zx)
-            a[f] = pp == 0 ? t : cadd(a[f], t);
-        }
-        __syncthreads();
+    for (int m = 0; m < FPT; ++m) {
+        const int f = tid + T * m;
+        float2 t = in[f];
+        for (int pp = 1; pp < npp; ++pp) t = cadd(t, in[(size_t)pp * M + f]);
+        smem[Lay::at(f, 0)] = t;
     }
-    // inverse DFT of T (unnormalised), real part / M at lags n < N
-#pragma unroll
-    for (int m = 0; m < FPT; ++m) smem[Lay::at(tid + T * m, 0)] = a[tid + T * m];
     __syncthreads();
     smem_stages<G, 0, NS - 1, true>(smem, tid, tw);
     stage<G, NS - 1, true, RL, RL / 2, false>(tid, tw, lds, [&](int n, int, float2 z) {
@@ -419,14 +433,19 @@ cudaError_t launch_fused_fwd(const fftconv_plan_s& p, const void* u, const void*
     }
 }
 
+// acc: [H][pairs per channel][M] fp32 complex (kgrad_workspace_elems)
 template <int LOG2M, typename IO, bool GATED>
 static cudaError_t kgrad_go(const fftconv_plan_s& p, const void* u, const void* w, const void* dy, const void* v,
                             float2* acc, float* dk, float* dD, int L, cudaStream_t s) {
-    auto kern = kgrad_simt<LOG2M, IO, GATED>;
+    auto k1 = kgrad_pairs<LOG2M, IO, GATED>;
+    auto k2 = kgrad_finish<LOG2M>;
     const size_t smem = fused_smem<LOG2M>();
-    ensure_smem(kern, smem);
-    kern<<<p.H, FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)w, (const IO*)dy, (const IO*)v, acc, dk, dD,
-                                              p.tw.wL, p.B, p.H, L);
+    ensure_smem(k1, smem);
+    ensure_smem(k2, smem);
+    const int npp = (p.B + 1) / 2;
+    k1<<<dim3(npp, p.H), FusedG<LOG2M>::T, smem, s>>>((const IO*)u, (const IO*)w, (const IO*)dy, (const IO*)v, acc,
+                                                      p.tw.wL, p.B, p.H);
+    k2<<<p.H, FusedG<LOG2M>::T, smem, s>>>(acc, dk, dD, p.tw.wL, npp, L);
     return cudaGetLastError();
 }
 

@@ -12,8 +12,9 @@
 //   dx = fwd(g, conj Khat, D) -> du = dx w, dw = dx u; s = fwd(x, Khat, D),
 //   the pre-gate output -> dv = dy s.
 // * Filter gradient: dk[j] = sum_b sum_t g x[t - j] = Re(iDFT(sum_pairs
-//   conj(DFT zx) DFT zg))[j] for the packed pairs zx, zg (kgrad_simt), and
-//   dD = the same at lag 0.
+//   conj(DFT zx) DFT zg))[j] for the packed pairs zx, zg (kgrad_pairs writes
+//   each pair's cross spectrum, kgrad_finish sums and inverts), and dD = the
+//   same at lag 0.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -82,7 +83,10 @@ struct BwdWs {
 BwdWs bwd_ws(const fftconv_plan_s& p) {
     BwdWs w;
     w.fwd = up256(p.workspace_bytes);
-    w.acc = fftc::kgrad_supported(p.log2M) ? up256((size_t)p.H * ((size_t)1 << p.log2M) * sizeof(float2)) : 0;
+    // the filter gradient's cross spectra, one per (channel, pair)
+    w.acc = fftc::kgrad_supported(p.log2M)
+                ? up256((size_t)p.H * ((p.B + 1) / 2) * ((size_t)1 << p.log2M) * sizeof(float2))
+                : 0;
     const size_t esz = p.dtype == FFTCONV_BF16 ? 2 : 4;
     w.gx = p.gated ? up256((size_t)p.B * p.H * p.N * esz) : 0;
     w.total = w.fwd + w.acc + 2 * w.gx;
