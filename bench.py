@@ -37,7 +37,8 @@ uniform sample of the same workload's outputs.
 variants (N=1): the skipped-work forms on the long workload's shape, each
 timed against the dense multi-pass plan on the same inputs (partial
 convolution, frequency-sparse filter, state-space filters with chunked state
-passing), and the backward pass of the Hyena-style layer against its forward.
+passing), the backward pass of the Hyena-style layer against its forward,
+and the 3-D causal convolution on 64^3 fp32 volumes.
 """
 import argparse
 import hashlib
@@ -618,6 +619,25 @@ def variants(torch, steps=5):
                              "ratio": round(tb / tf, 3), "path": plan.path,
                              "note": "du, dk, dD of the Hyena-style layer against its forward"}
     del plan, khat, kconj, uh, dyh, yh
+    torch.cuda.empty_cache()
+    # the 3-D causal convolution (no named workload is 3-D): B=2, C=8, 64^3 fp32
+    # volumes with full-size filters; output elements per second and the HBM
+    # fraction of u + y
+    B3, C3, S3 = 2, 8, 64
+    plan = binding.Plan3D(B3, C3, S3, S3, S3, "f32")
+    k3 = torch.randn(C3, S3, S3, S3, generator=g).to(dev)
+    kh3 = plan.kernel_spectrum(k3)
+    u3 = torch.randn(B3, C3, S3, S3, S3, generator=g).to(dev)
+    y3 = torch.empty_like(u3)
+    ws3 = plan.new_workspace()
+    t3 = _time_fn(lambda: plan.fwd(u3, kh3, y=y3, workspace=ws3), steps, 3, torch, flush)
+    n3 = B3 * C3 * S3 ** 3
+    hbm, _, _ = measured_peaks()
+    out["conv3d_b2_c8_64cubed_f32"] = {"ms": round(t3, 4), "elems_per_s": n3 / (t3 * 1e-3),
+                                      "hbm_frac": round(2 * n3 * 4 / (t3 * 1e-3) / 1e9 / hbm, 4), "path": plan.path,
+                                      "note": "five launches per group (rows, columns, depth with the product, "
+                                              "inverse columns, inverse rows) through an fp32 workspace"}
+    del plan, kh3, u3, y3, ws3, k3
     torch.cuda.empty_cache()
     return out
 
