@@ -596,10 +596,24 @@ def variants(torch, steps=5):
     lam64, c64 = lam.to(torch.complex128).to(dev), c.to(torch.complex128).to(dev)
     for j in range(d):  # the same filters materialised (fp64) for the dense plan
         kmat += (c64[:, j:j + 1] * torch.exp(tt[None, :] * torch.log(lam64[:, j:j + 1]))).real
-    kd = dense.kernel_spectrum(kmat.to(torch.float32), khat=kd)
+    kmat_f32 = kmat.to(torch.float32)
+    kd = dense.kernel_spectrum(kmat_f32, khat=kd)
     del kmat, tt
     pair("ssm_chunked_d16", lambda: ssm.fwd(u, kss, D=D, y=y), lambda: dense.fwd(u, kd, D=D, y=y, workspace=ws),
          "diagonal state-space filters, chunks of 8192 with the state passed vs the dense plan on the same filters")
+    # the same filters in bf16: chunks of 4096 on the two-stage tensor-core kernel,
+    # against the bf16 dense multi-pass plan
+    ub = u.to(torch.bfloat16)
+    yb = torch.empty_like(ub)
+    ssmb = binding.SSMPlan(B, H, N, "bf16", d_state=d, chunk=4096)
+    kssb = ssmb.set_filters(lam, c)
+    denseb = binding.Plan(B, H, N, "bf16")
+    wsb = denseb.new_workspace()
+    kdb = denseb.kernel_spectrum(kmat_f32)
+    pair("ssm_chunked_d16_bf16", lambda: ssmb.fwd(ub, kssb, D=D, y=yb),
+         lambda: denseb.fwd(ub, kdb, D=D, y=yb, workspace=wsb),
+         "bf16: chunks of 4096 on the two-stage tensor-core kernel with the state passed vs the bf16 dense plan")
+    del ssmb, kssb, denseb, wsb, kdb, ub, yb, kmat_f32
     del ssm, kss, dense, ws, u, y
     torch.cuda.empty_cache()
     # the backward pass on the Hyena-style layer (B=8, H=768, N=4096 bf16): du through the

@@ -190,9 +190,11 @@ cudaError_t launch_ssm_setup(const fftconv_plan_s& p, const float* lr, const flo
     ssm::ssm_setup<<<p.H, ssm::kThreads, 0, s>>>(lr, li, cr, ci, p.d_state, (int)p.T, v.lam, v.cc, v.pw, k);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // one spectrum per channel, of k[:T] zero-padded to 2T
+    // one spectrum per channel, of k[:T] zero-padded to 2T, in the layout of the
+    // chunk plan's forward kernel
     fftconv_plan_s q = *p.chunk;
     q.H = p.H;
+    if (q.t2) return launch_t2_spectrum(q, k, p.T, khat, s);
     return launch_fused_spectrum(q, k, p.T, (float2*)khat, s);
 }
 
@@ -218,7 +220,9 @@ cudaError_t launch_ssm_fwd(const fftconv_plan_s& p, const void* u, const void* k
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // intra-chunk convolutions: rows [B][H x nc][T], one spectrum and D per channel
-    e = launch_fused_fwd(*p.chunk, u, nullptr, nullptr, (const float2*)khat, D, y, s);
+    // (bf16 chunks of 4096: the two-stage tensor-core kernel; else the fp32 fused kernel)
+    e = p.chunk->t2 ? launch_t2_fwd(*p.chunk, u, khat, D, y, s)
+                    : launch_fused_fwd(*p.chunk, u, nullptr, nullptr, (const float2*)khat, D, y, s);
     if (e != cudaSuccess || nc <= 1) return e;
     const dim3 g(nc - 1, p.H, p.B);
     if (p.dtype == FFTCONV_BF16)

@@ -117,7 +117,8 @@ constexpr uint32_t kXBytes = 16384;
 __global__ void __launch_bounds__(kThreads, 1)
 fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
              __nv_bfloat16* __restrict__ y, const uint4* __restrict__ mats, const uint2* __restrict__ twid,
-             int* __restrict__ err, int B, int H, uint32_t wait_limit, const __grid_constant__ CUtensorMap xmap) {
+             int* __restrict__ err, int B, int H, uint32_t wait_limit, int kdiv,
+             const __grid_constant__ CUtensorMap xmap) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ __align__(8) SlotBars s_bar[2];
@@ -318,8 +319,11 @@ fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
         };
         for (int q = first_pair(slot); q < pairs; q += qstep) {
             const int h = q / npp, b0 = 2 * (q % npp);
+            // kdiv consecutive row channels share one spectrum and skip weight (the
+            // chunks of one channel in the chunked state-passing path; 1 otherwise)
+            const int hk = h / kdiv;
             // the skip weight, loaded here so that its latency passes before epilogue B
-            const float dh = D ? __ldg(&D[h]) : 0.f;
+            const float dh = D ? __ldg(&D[hk]) : 0.f;
             // ---- epilogue A: -> A operand of stage B (Ra columns 0..63)
             if (!wait(bar(sb.dA), pdA)) break;
             um::fence_after();
@@ -338,7 +342,7 @@ fused_fwd_t2(const uint4* __restrict__ khat, const float* __restrict__ D,
             // lanes of a warp read 512 contiguous bytes
             uint4 kv[8];
             {
-                const uint4* kp = khat + (size_t)(h * 4 + 2 * hf) * 4 * kP + r;
+                const uint4* kp = khat + (size_t)(hk * 4 + 2 * hf) * 4 * kP + r;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) kv[i] = __ldg(&kp[i * kP]);
             }
@@ -595,7 +599,7 @@ cudaError_t launch_t2_fwd(const fftconv_plan_s& p, const void* u, const void* kh
     const int pairs = ((p.B + 1) / 2) * p.H;  // each CTA walks its pairs alternately on its two slots
     dim3 grid(pairs < sms ? pairs : sms);
     kern<<<grid, t2::kThreads, t2::kSmemBytes, s>>>((const uint4*)khat, D, (__nv_bfloat16*)y, p.t2_mats, p.t2_twid,
-                                                    p.d_err, p.B, p.H, p.wait_limit, xmap);
+                                                    p.d_err, p.B, p.H, p.wait_limit, p.kdiv, xmap);
     return cudaGetLastError();
 }
 

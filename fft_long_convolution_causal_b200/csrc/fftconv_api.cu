@@ -340,12 +340,15 @@ fftconv_status fftconv_ssm_plan_create(fftconv_plan_t* out, int B, int H, int64_
     if (N < chunk || N % chunk != 0 || N / chunk > 65535) return FFTCONV_ERR_UNSUPPORTED;
     const int64_t nc = N / chunk;
     if ((int64_t)H * nc > 65535) return FFTCONV_ERR_UNSUPPORTED;
+    // the chunk plan: bf16 chunks of 4096 (2T = 8192) on the two-stage tensor-core
+    // kernel, every other chunk size on the fp32 fused kernel
     fftconv_plan_options o = defaults();
-    o.kernel = FFTCONV_KERNEL_SIMT;
+    const bool tc_chunks = dtype == FFTCONV_BF16 && chunk == 4096;
+    o.kernel = tc_chunks ? FFTCONV_KERNEL_TCGEN05 : FFTCONV_KERNEL_SIMT;
     fftconv_plan_t ch = nullptr;
     fftconv_status st = fftconv_plan_create_ex(&ch, B, (int)(H * nc), chunk, dtype, 0, &o);
     if (st != FFTCONV_OK) return st;
-    if (ch->path != fftc::PATH_FUSED) {
+    if (tc_chunks ? !ch->t2 : ch->path != fftc::PATH_FUSED) {
         fftconv_plan_destroy(ch);
         return FFTCONV_ERR_UNSUPPORTED;
     }
@@ -693,6 +696,7 @@ fftconv_status fftconv2d_fwd_offset(fftconv_plan_t p, const void* u, const void*
 fftconv_status fftconv_plan_set_wait_limit(fftconv_plan_t p, uint32_t probes) {
     if (!p) return FFTCONV_ERR_INVALID_ARG;
     p->wait_limit = probes;
+    if (p->chunk) p->chunk->wait_limit = probes;  // chunked plans launch their chunk plan's kernels
     return FFTCONV_OK;
 }
 

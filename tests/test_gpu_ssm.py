@@ -69,6 +69,25 @@ def test_ssm_long_sampled(N, T, d):
     assert_close(y[b, h, t], want, "f32", f"ssm N={N} T={T} d={d}", scale=row_scale_1d(wl, b, h))
 
 
+@pytest.mark.parametrize("B,H,N", [(3, 2, 16384), (2, 3, 4096)])
+def test_ssm_bf16_tensor_core_chunks(B, H, N):
+    """bf16 plans with chunks of 4096 run the chunk convolutions on the
+    two-stage tcgen05 kernel (chunks of one channel share its spectrum); every
+    output compared, odd B, a single chunk."""
+    y, u, k, D, wl = run(B, H, N, "bf16", 16, 4096, seed=N + B)
+    want = oracle.causal_conv1d(u, k, D=D)
+    assert_close(y, want, "bf16", f"ssm bf16 tensor-core chunks B={B} H={H} N={N}", scale=row_scale_1d(wl))
+
+
+def test_ssm_bf16_tensor_core_chunks_long():
+    """2^20 bf16 (256 chunks of 4096 on the tensor cores), sampled outputs."""
+    B, H, N = 2, 3, 1 << 20
+    y, u, k, D, wl = run(B, H, N, "bf16", 16, 4096, seed=17)
+    b, h, t = wlmod.sample_points_1d(B, H, N, 64, seed=N + 1)
+    want = oracle.causal_conv1d_points(u, k, b, h, t, D=D)
+    assert_close(y[b, h, t], want, "bf16", "ssm bf16 2^20 tensor-core chunks", scale=row_scale_1d(wl, b, h))
+
+
 def test_ssm_rejects_bad_shapes():
     from fft_long_convolution_causal_b200 import binding
     for args in ((2, 2, 1000, "f32", 4, 256), (2, 2, 4096, "f32", 4, 16384), (2, 2, 4096, "f32", 0, 256),
