@@ -121,3 +121,76 @@ def test_null_plan_option_calls(lib):
     assert lib.fftconv_plan_mma_flops(None) == 0.0
     assert lib.fftconv_device_status(None, None) == 1
     assert lib.fftconv_fwd_static_workspace(None, None, None, None, None, None, None, None) == 1
+
+
+def _out():
+    h = ctypes.c_void_p()
+    return h, ctypes.byref(h)
+
+
+@pytest.mark.parametrize("B,H,N,dtype,d,chunk,want", [
+    (0, 4, 1 << 16, 0, 16, 8192, 1),          # no rows
+    (1, 4, 1 << 16, 2, 16, 8192, 1),          # fp16 is not a state-passing dtype
+    (1, 4, 1 << 16, 0, 0, 8192, 1),           # no state
+    (1, 4, 1 << 16, 0, 65, 8192, 1),          # state above the largest supported
+    (1, 4, 1 << 16, 0, 16, 6144, 2),          # chunk not a power of two
+    (1, 4, 1 << 16, 0, 16, 32, 2),            # chunk below the smallest
+    (1, 4, 1 << 16, 0, 16, 16384, 2),         # chunk above the largest
+    (1, 4, 4096, 0, 16, 8192, 2),             # sequence shorter than one chunk
+    (1, 4, 12288, 0, 16, 8192, 2),            # sequence not a whole number of chunks
+    (1, 64, 1 << 20, 0, 16, 64, 2),           # channels x chunks past the launch grid
+])
+def test_ssm_plan_create_rejects(lib, B, H, N, dtype, d, chunk, want):
+    h, ref = _out()
+    assert lib.fftconv_ssm_plan_create(ref, B, H, N, dtype, d, chunk) == want
+    assert not h.value
+    assert lib.fftconv_ssm_plan_create(None, 1, 4, 1 << 16, 0, 16, 8192) == 1
+
+
+@pytest.mark.parametrize("B,H,N,dtype,L,want", [
+    (0, 4, 1 << 16, 0, 1024, 1), (1, 4, 1 << 16, 2, 1024, 1), (1, 4, 1 << 16, 0, 0, 1),
+    (1, 4, 1 << 16, 0, 16384, 2),   # the on-chip chunk would exceed 8192
+    (1, 4, 1024, 0, 2048, 2),       # sequence shorter than the chunk
+])
+def test_partial_plan_create_rejects(lib, B, H, N, dtype, L, want):
+    h, ref = _out()
+    assert lib.fftconv_partial_plan_create(ref, B, H, N, dtype, 0, L) == want
+    assert not h.value
+
+
+@pytest.mark.parametrize("B,C,Hs,Ws,want", [
+    (0, 1, 64, 64, 1), (1, 0, 64, 64, 1), (1 << 16, 1 << 15, 64, 64, 1),
+    (1, 1, 8, 64, 2), (1, 1, 64, 512, 2), (1, 1, 48, 64, 2),
+])
+def test_plan2d_dynamic_create_rejects(lib, B, C, Hs, Ws, want):
+    h, ref = _out()
+    assert lib.fftconv2d_dynamic_plan_create(ref, B, C, Hs, Ws, 1) == want
+    assert not h.value
+
+
+@pytest.mark.parametrize("B,C,Dd,Hs,Ws,dtype,want", [
+    (0, 1, 16, 16, 16, 0, 1), (1, 0, 16, 16, 16, 0, 1), (1, 1, 16, 16, 16, 2, 1),
+    (1, 1 << 25, 64, 16, 16, 0, 1),   # C x Dd slices past 2^30
+    (1, 1, 8, 16, 16, 0, 2), (1, 1, 16, 48, 16, 0, 2), (1, 1, 16, 16, 512, 0, 2),
+])
+def test_plan3d_create_rejects(lib, B, C, Dd, Hs, Ws, dtype, want):
+    h, ref = _out()
+    assert lib.fftconv3d_plan_create(ref, B, C, Dd, Hs, Ws, dtype) == want
+    assert not h.value
+    assert lib.fftconv3d_plan_create(None, 1, 1, 16, 16, 16, 0) == 1
+
+
+def test_null_plan_calls_of_the_extended_paths(lib):
+    """Every entry point beyond the four core calls reports a NULL plan as an
+    invalid argument (sizes as 0) without touching the device."""
+    assert lib.fftconv_fwd_dynamic(None, None, None, None, None, 1, None, None, None) == 1
+    assert lib.fftconv_spectrum_blocks(None) == 0
+    assert lib.fftconv_spectrum_sparsify(None, None, None, 0, None) == 1
+    assert lib.fftconv_ssm_spectrum(None, None, None, None, None, None, None, None) == 1
+    assert lib.fftconv2d_fwd_offset(None, None, None, None, None, None, 0, 0) == 1
+    assert lib.fftconv2d_fwd_dynamic(None, None, None, 1, 1, None, None, None) == 1
+    assert lib.fftconv3d_kernel_spectrum(None, None, 1, 1, 1, None, None, None) == 1
+    assert lib.fftconv3d_fwd(None, None, None, None, None, None) == 1
+    assert lib.fftconv_spectrum_conjugate(None, None, None, None) == 1
+    assert lib.fftconv_bwd_workspace_bytes(None) == 0
+    assert lib.fftconv_bwd(*([None] * 8), 1, *([None] * 7)) == 1
