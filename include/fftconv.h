@@ -41,6 +41,15 @@
  * plan may be used by several streams for fftconv_fwd at once provided each
  * call gets its own workspace; plan creation and destruction are not
  * thread-safe with respect to other calls on the same plan.
+ *
+ * Graph capture.  The forward calls (fftconv_fwd, fftconv2d_fwd(_offset),
+ * fftconv2d_fwd_dynamic, fftconv3d_fwd, and the forward of partial and
+ * state-passing plans) and fftconv_bwd enqueue only kernel launches on the
+ * given stream, so they may be captured into a CUDA graph once the same kind
+ * of call has run eagerly in the process (that first call sets the kernels'
+ * shared-memory limits).  A replay reads and writes the buffers named at
+ * capture.  Plan creation, fftconv_spectrum_sparsify and
+ * fftconv_device_status synchronise and are not capturable.
  */
 #ifndef FFTCONV_H
 #define FFTCONV_H
