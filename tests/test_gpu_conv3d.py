@@ -100,6 +100,26 @@ def test_conv3d_several_groups():
     assert_close(y[idx], ref, "f32", "3d groups", scale=_scale(u, k, idx[0], idx[1]))
 
 
+@pytest.mark.parametrize("B,dtype", [(1, "f32"), (2, "bf16")])
+def test_conv3d_max_side_full_filters(B, dtype):
+    """256 x 256 x 256 volumes, the largest side on every axis, with filters
+    as large as the volume: the eight corners of each volume (the far corner
+    sums all 256^3 taps) plus uniformly drawn voxels."""
+    C, S = 1, 256
+    u, k = _volume(B, C, S, S, S, S, S, S, dtype, seed=95, sigma=48.0)
+    y, _ = _run(u, k, dtype)
+    r = np.random.default_rng(96)
+    corners = np.array([(d, h, w) for d in (0, S - 1) for h in (0, S - 1) for w in (0, S - 1)])
+    n = 96
+    bi = np.concatenate([np.repeat(np.arange(B), len(corners)), r.integers(0, B, n)])
+    di = np.concatenate([np.tile(corners[:, 0], B), r.integers(0, S, n)])
+    hi = np.concatenate([np.tile(corners[:, 1], B), r.integers(0, S, n)])
+    wi = np.concatenate([np.tile(corners[:, 2], B), r.integers(0, S, n)])
+    ci = np.zeros_like(bi)
+    ref = oracle.causal_conv3d_points(u, k, bi, ci, di, hi, wi)
+    assert_close(y[bi, ci, di, hi, wi], ref, dtype, f"3d 256^3 {dtype}", scale=_scale(u, k, bi, ci))
+
+
 def test_conv3d_errors():
     from fft_long_convolution_causal_b200 import binding
     with pytest.raises(binding.FFTConvError):
