@@ -122,8 +122,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
 }
-// One bulk tensor copy (no multicast) of a 5-D box at the given coordinates
-// into shared memory at dst, completing its bytes on the barrier at mbar.
+// One bulk tensor copy of a 5-D box at the given coordinates into this CTA's
+// own shared memory at dst, completing its bytes on the barrier at mbar.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* map, int c0, int c1, int c2, int c3, int c4,
                                             uint32_t mbar) {
     asm volatile(
