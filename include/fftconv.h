@@ -282,10 +282,12 @@ FFTCONV_API fftconv_status fftconv_partial_plan_create(fftconv_plan_t* plan, int
 FFTCONV_API fftconv_status fftconv_ssm_plan_create(fftconv_plan_t* plan, int B, int H, int64_t N,
                                                    fftconv_dtype dtype, int d_state, int64_t chunk);
 
-/* Set the filters: lam and c are [H][d] fp32 device arrays (real and
- * imaginary parts separately).  Materialises k[:T], writes khat and keeps
- * lam, c and their power table in the plan.  Then fftconv_fwd(plan, u, NULL,
- * NULL, khat, D, y, workspace, stream) runs the chunked convolution. */
+/* Set the filters of a state-passing plan (the state-space filters of
+ * "FlashConv", Mechanism, defined above): lam and c are [H][d] fp32 device
+ * arrays (real and imaginary parts separately).  Materialises k[:T], writes
+ * khat and keeps lam, c and their power table in the plan.  Then
+ * fftconv_fwd(plan, u, NULL, NULL, khat, D, y, workspace, stream) runs the
+ * chunked convolution. */
 FFTCONV_API fftconv_status fftconv_ssm_spectrum(fftconv_plan_t plan, const float* lam_re, const float* lam_im,
                                                 const float* c_re, const float* c_im, void* khat, void* workspace,
                                                 void* stream);
@@ -302,7 +304,8 @@ FFTCONV_API fftconv_status fftconv2d_kernel_spectrum(fftconv_plan_t plan, const 
 /*
  * 2-D forward: y[b,c,i,j] = sum_{p<=i, q<=j} k[c,p,q] u[b,c,i-p,j-q] for
  * 0 <= i < Hs, 0 <= j < Ws (the first-quadrant crop of the zero-padded
- * linear convolution, the 2-D analogue of [:N]; same page as the spectrum).
+ * linear convolution, the 2-D analogue of [:N]; "Native Multi-Dimensional
+ * Subquadratic Operators via Input Dependent Long Convolutions", abstract).
  * u, y: [B][C][Hs][Ws] of the plan's dtype.  FFTCONV_ERR_INVALID_ARG also
  * when the current device is not the plan's.
  */
@@ -315,7 +318,9 @@ FFTCONV_API fftconv_status fftconv2d_fwd(fftconv_plan_t plan, const void* u, con
  * linear convolution full[r][s] = sum_{p,q} k[c,p,q] u[b,c,r-p,s-q] (indices
  * inside both arrays).  (0, 0) is fftconv2d_fwd's first-quadrant crop;
  * (Hs/2, Ws/2) the centred reading of a kernel anchored at its middle (the
- * pages' zero-padded convolution does not say which window).  0 <= oy <= Hs,
+ * zero-padded multi-dimensional convolution of "Native Multi-Dimensional
+ * Subquadratic Operators via Input Dependent Long Convolutions", abstract,
+ * does not say which window).  0 <= oy <= Hs,
  * 0 <= ox <= Ws, both multiples of 8 (else FFTCONV_ERR_INVALID_ARG).  The
  * transform of length 2Hs x 2Ws holds the full convolution without
  * wrap-around, so only the last inverse passes change: they keep rows
@@ -372,7 +377,9 @@ FFTCONV_API fftconv_status fftconv3d_fwd(fftconv_plan_t plan, const void* u, con
 
 /*
  * Conjugate spectrum: khat_conj <- conj(khat) in the plan's layout, the
- * spectrum of the correlation with k (the backward pass's filter).  khat is
+ * spectrum of the correlation with k (the backward pass's filter, below; the
+ * training of "Simple Hardware-Efficient Long Convolutions for Sequence
+ * Modeling", abstract).  khat is
  * the output of fftconv_kernel_spectrum on this plan; khat_conj is a buffer of
  * fftconv_spectrum_bytes() bytes and may equal khat (in place).
  */
