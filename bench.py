@@ -44,6 +44,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -59,15 +60,19 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 # Source files each dominant kernel is built from: a recorded DRAM-traffic
 # figure is valid only while the hash of these files matches.
-KERNEL_SOURCES = {
-    "fused_fwd_simt": ["fft_simt.cuh", "conv1d_simt.cu"],
-    "mp_pass2": ["fft_simt.cuh", "conv1d_simt.cu"],
-    "c2_pass2": ["fft_simt.cuh", "conv2d_simt.cu"],
-    "fused_fwd_tc": ["tc_common.cuh", "umma.cuh", "conv1d_mma.cu"],
-    "fused_fwd_umma": ["tc_common.cuh", "umma.cuh", "conv1d_umma.cu"],
-    "fused_fwd_t2": ["umma.cuh", "conv1d_t2.cu"],
-    "c2tc_cols": ["tc_common.cuh", "tables.h", "conv2d_tc.cu"],
+# The translation unit of each dominant kernel; its sources are that file and
+# every header under csrc/ it includes, directly or through other headers.
+KERNEL_UNITS = {
+    "fused_fwd_simt": "conv1d_simt.cu",
+    "mp_pass2": "conv1d_simt.cu",
+    "c2_pass2": "conv2d_simt.cu",
+    "fused_fwd_tc": "conv1d_mma.cu",
+    "fused_fwd_umma": "conv1d_umma.cu",
+    "fused_fwd_t2": "conv1d_t2.cu",
+    "c2tc_cols": "conv2d_tc.cu",
 }
+KERNEL_SOURCES = KERNEL_UNITS  # kernel names recognised in an ncu capture
+CSRC = os.path.join(ROOT, "fft_long_convolution_causal_b200", "csrc")
 
 
 def parse():
@@ -118,11 +123,28 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def kernel_sources(kernel):
+    """The kernel's translation unit and the csrc/ headers it includes,
+    transitively, sorted.  The public API header (include/) declares entry
+    points and status codes only and is not followed."""
+    unit = KERNEL_UNITS.get(kernel)
+    if unit is None:
+        return []
+    seen, todo = set(), [unit]
+    while todo:
+        f = todo.pop()
+        path = os.path.join(CSRC, f)
+        if f in seen or not os.path.exists(path):
+            continue
+        seen.add(f)
+        todo += re.findall(r'#include "([^"]+)"', open(path, encoding="utf-8").read())
+    return sorted(seen)
+
+
 def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES.get(kernel, []):
-        path = os.path.join(ROOT, "fft_long_convolution_causal_b200", "csrc", f)
-        h.update(open(path, "rb").read() if os.path.exists(path) else b"")
+    for f in kernel_sources(kernel):
+        h.update(f.encode() + b"\0" + open(os.path.join(CSRC, f), "rb").read())
     return h.hexdigest()[:16]
 
 
