@@ -271,6 +271,8 @@ def build_workload(name, channels=0, rank=0, world=1, shard="weak"):
     wl = workloads.make_1d(name=label, **c) if kind == "1d" else workloads.make_2d(name=label, **c)
     if world > 1 and shard == "strong":
         nch = wl.H if kind == "1d" else wl.C
+        if nch < world:  # every rank reaches this, so all of them stop together
+            raise SystemExit(f"--shard strong: {world} ranks for {nch} channels leaves ranks without work")
         a, b = fdist.shard_channels(nch, world, rank)
         wl = fdist.slice_channels_1d(wl, a, b) if kind == "1d" else fdist.slice_channels_2d(wl, a, b)
     return wl
@@ -501,16 +503,18 @@ def measure(wl, args, torch, steps, warmup, pg=None, world=1, clocks=False, e2e=
     if pg:
         pg.barrier()
     clk = sampler.stop() if sampler else None
-    from fft_long_convolution_causal_b200.dist import job_throughput, max_over_ranks
+    from fft_long_convolution_causal_b200.dist import max_over_ranks, sum_over_ranks
     total_ms = max_over_ranks(float(np.sum(per_step)), pg, device="cuda")
     ms_per_step = total_ms / steps
-    value = job_throughput(r.outputs, world, ms_per_step * 1e-3)
+    # every rank's outputs (shards may differ by a channel) over the slowest rank's time
+    job_outputs = sum_over_ranks(float(r.outputs), pg, device="cuda")
+    value = job_outputs / (ms_per_step * 1e-3)
 
     e2e_d = None
     if e2e:
         e2e_ms, h2d, d2h = time_e2e(r, max(3, min(steps, 20)), torch)
         e2e_ms = max_over_ranks(e2e_ms, pg, device="cuda")
-        e2e_d = {"value": job_throughput(r.outputs, world, e2e_ms * 1e-3), "unit": "elems/s",
+        e2e_d = {"value": job_outputs / (e2e_ms * 1e-3), "unit": "elems/s",
                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     hbm, bf16, peak_kind = measured_peaks()

@@ -54,6 +54,16 @@ def max_over_ranks(value, dist=None, device=None):
     return float(t.item())
 
 
+def sum_over_ranks(value, dist=None, device=None):
+    """Sum of a float over all ranks of the default process group (identity when single)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def job_throughput(outputs_per_rank, world, max_seconds):
     """Whole-job outputs per second: every rank's outputs over the slowest rank's time."""
     return outputs_per_rank * world / max_seconds

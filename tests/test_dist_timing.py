@@ -23,7 +23,9 @@ def _worker(rank, world, port, q):
     try:
         r, w, _ = fdist.rank_env()
         mx = fdist.max_over_ranks(1.5 + r, d)
-        q.put((r, w, mx, fdist.job_throughput(1000, w, mx)))
+        # uneven shards: rank r holds 1000 + 7 r outputs; the job holds their sum
+        total = fdist.sum_over_ranks(1000 + 7 * r, d)
+        q.put((r, w, mx, fdist.job_throughput(1000, w, mx), total))
     finally:
         d.destroy_process_group()
 
@@ -40,12 +42,14 @@ def test_max_over_ranks_two_gloo_ranks():
         assert p.exitcode == 0
     got = sorted(q.get(timeout=10) for _ in range(2))
     assert [g[0] for g in got] == [0, 1]
-    for _, w, mx, thr in got:
+    for _, w, mx, thr, total in got:
         assert w == 2 and mx == pytest.approx(2.5) and thr == pytest.approx(2000 / 2.5)
+        assert total == 2007.0
 
 
 def test_single_process_is_identity():
     assert fdist.max_over_ranks(3.25) == 3.25
+    assert fdist.sum_over_ranks(3.25) == 3.25
     assert fdist.job_throughput(10, 1, 2.0) == 5.0
 
 
