@@ -11,8 +11,8 @@ The CUDA library is loaded on first use; if it is missing the call raises.
 from . import workloads  # noqa: F401  (pure numpy, no arithmetic of the method)
 
 _BINDING_NAMES = {
-    "Plan", "Plan2D", "load_library", "library_path", "FFTConvError",
-    "fftconv", "fftconv2d", "status_string",
+    "Plan", "Plan2D", "Plan2DDynamic", "Plan3D", "PartialPlan", "SSMPlan", "PlanOptions",
+    "load_library", "library_path", "FFTConvError", "fftconv", "fftconv2d", "status_string",
 }
 
 
